@@ -1,0 +1,447 @@
+#!/usr/bin/env python3
+"""Benchmark of the decode-time Gated DeltaNet state update on B200.
+
+Workload (one "step"): the large L2-busting decode -- 8 independent GDN layer
+instances, each a call of gdn_decode_step on B=256 requests x Hv=32 value heads
+(Hk=16, dk=dv=128, bf16 q/k/v, fp32 state), in place on a random slot
+permutation of a 2048-slot pool (2 MiB of state per request per layer, 4 GiB
+per pool, 32 GiB allocated, 4 GiB touched per step: far beyond the 126 MB L2,
+so no flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  ``value`` is tokens*heads per second over the
+whole job (device-timed with CUDA events, max over ranks); ``e2e`` is the same
+metric through the public API with each step's inputs copied from pinned host
+memory and its outputs copied back inside the timed region.  With N > 1 every
+rank runs an independent replica (the update has no exchange step), so scaling
+is weak.  ``--impl reference`` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import os
+import pathlib
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "GDN state-update tokens·heads/s and achieved HBM GB/s vs B200 peak, 1 GPU"
+UNIT = "tokens*heads/s"
+WORKLOAD = "large L2-busting decode: B=256 x 8 GDN layers, Hk=16 Hv=32 dk=dv=128, in-place"
+KERNEL_SOURCE = ROOT / "hybrid_linear_attention_step_b200" / "csrc" / "gdn_step.cu"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
+# source it was taken on (sha256 of gdn_step.cu).  See profiles/.
+NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "profile": None}
+
+
+def algorithmic_bytes_per_unit(dk: int, dv: int, G: int, in_bytes: int = 2, T: int = 1) -> float:
+    """Bytes one (request, token, value head) must move: its state tile read once
+    per request and written once per token, plus its share of q/k (shared by the
+    G value heads of a key head), v, alpha, beta and the fp32 output."""
+    state = 4.0 * dk * dv * (1.0 / T + 1.0)
+    qk = 2.0 * dk * in_bytes / G
+    return state + qk + dv * in_bytes + 8.0 + 4.0 * dv
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            d = json.loads(p.read_text())
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_sha256() -> str:
+    return hashlib.sha256(KERNEL_SOURCE.read_bytes()).hexdigest()
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str, interval_ms: int = 50):
+        self.proc = None
+        self.gpu_index = gpu_index
+        self.interval_ms = interval_ms
+        self.window = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", f"-lms={self.interval_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for r in csv.reader(io.StringIO(out)):
+            if len(r) < 11:
+                continue
+            try:
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append(dict(ts=ts, sm=float(r[2]), sm_max=float(r[3]), power=float(r[4]),
+                                 util=float(r[5]), hw=r[7].strip(), hw_th=r[8].strip(),
+                                 sw_th=r[9].strip(), pcap=r[10].strip()))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        picked, where = rows, "all"
+        if self.window:
+            inside = [r for r in rows if self.window[0] - 0.05 <= r["ts"] <= self.window[1] + 0.05]
+            if len(inside) >= 3:
+                picked, where = inside, "timed"
+            else:
+                busy = [r for r in rows if r["util"] >= 50]
+                if busy:
+                    picked, where = busy, "busy"
+        reasons = set()
+        for r in picked:
+            for key, name in (("hw", "hw_slowdown"), ("hw_th", "hw_thermal_slowdown"),
+                              ("sw_th", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in picked),
+                "sm_max_mhz": max(r["sm_max"] for r in picked),
+                "reasons": sorted(reasons), "samples": len(picked), "window": where}
+
+
+# ----------------------------------------------------------- the workload
+
+class LargeDecode:
+    """Device-resident large decode: ``layers`` pools, per-layer inputs, one step = ``layers`` calls."""
+
+    def __init__(self, layers: int = 8, num_slots: int = 2048, B: int = 256, device: str = "cuda",
+                 seed: int = 4):
+        import numpy as np
+        import torch
+
+        from hybrid_linear_attention_step_b200 import gdn, workloads as wl
+
+        c = wl.LARGE
+        self.gdn = gdn
+        self.layers, self.num_slots, self.B = layers, num_slots, B
+        self.Hk, self.Hv, self.dk, self.dv = c["Hk"], c["Hv"], c["dk"], c["dv"]
+        self.seed = seed
+        self.device = torch.device(device)
+        self.host_steps = [wl.large_layer_step(l, seed, B, num_slots) for l in range(layers)]
+        self.pools, self.inputs, self.outs = [], [], []
+        for l in range(layers):
+            pool = torch.empty((num_slots, self.Hv, self.dk, self.dv), dtype=torch.float32, device=self.device)
+            wl.fill_pool_device(pool, seed, l)
+            self.pools.append(pool)
+            s = self.host_steps[l]
+            bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+            self.inputs.append(dict(
+                q=bf(s.q).to(self.device), k=bf(s.k).to(self.device), v=bf(s.v).to(self.device),
+                alpha=torch.from_numpy(s.alpha).to(self.device), beta=torch.from_numpy(s.beta).to(self.device),
+                src=torch.from_numpy(s.src_idx).to(self.device), dst=torch.from_numpy(s.dst_idx).to(self.device)))
+            self.outs.append(torch.zeros((B, 1, self.Hv, self.dv), dtype=torch.float32, device=self.device))
+        self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        torch.cuda.synchronize(self.device)
+
+    @property
+    def units_per_step(self) -> int:
+        return self.layers * self.B * self.Hv
+
+    @property
+    def units_per_launch(self) -> int:
+        return self.B * self.Hv
+
+    def launch(self, l: int, stream=None):
+        x = self.inputs[l]
+        self.gdn.gdn_decode_step(self.pools[l], x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"],
+                                 x["beta"], self.outs[l], err_word=self.err, stream=stream)
+
+    def step(self, stream=None):
+        for l in range(self.layers):
+            self.launch(l, stream)
+
+    # -- end to end: inputs from pinned host memory, outputs back to pinned host memory
+    def make_host_io(self):
+        import torch
+
+        self.h_in = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in self.inputs]
+        self.h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for x in self.h_in for t in x.values())
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def step_e2e(self, stream):
+        for l in range(self.layers):
+            x, hx = self.inputs[l], self.h_in[l]
+            for key in ("q", "k", "v", "alpha", "beta", "src", "dst"):
+                x[key].copy_(hx[key], non_blocking=True)
+            self.launch(l, stream)
+            self.h_out[l].copy_(self.outs[l], non_blocking=True)
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_setup(n_gpus: int):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def _oracle_sample_inputs(n_req: int, seed: int = 4):
+    import numpy as np
+
+    from hybrid_linear_attention_step_b200 import workloads as wl
+
+    s = wl.large_layer_step(0, seed)
+    rng = np.random.default_rng([seed, 99])
+    pool = wl.init_pool(rng, n_req, s.Hv, s.dk, s.dv)
+    idx = np.arange(n_req, dtype=np.int32)
+    sl = lambda a: np.ascontiguousarray(a[:n_req])
+    return pool, idx, sl(s.q), sl(s.k), sl(s.v), sl(s.alpha), sl(s.beta), s.Hv, s.dv
+
+
+def oracle_time(n_req: int, threads: int) -> float:
+    """Seconds the oracle takes for one in-place call on ``n_req`` requests of the large decode."""
+    import numpy as np
+
+    import oracle
+
+    pool, idx, q, k, v, a, b, Hv, dv = _oracle_sample_inputs(n_req)
+    out = np.zeros((n_req, 1, Hv, dv), np.float32)
+    t0 = time.perf_counter()
+    oracle.decode_step(pool, idx, idx.reshape(-1, 1).copy(), q, k, v, a, b, out, nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float = 12.0, Hv: int = 32):
+    """The oracle as it stands, timed on the host cores on a bounded sample of the workload."""
+    cores = cpu_cores()
+    t1 = oracle_time(1, 1)  # one request (32 units), single thread: calibration
+    n_req = int(max(1, min(256, budget_s * cores / max(t1, 1e-6) * 0.8)))
+    threads = min(cores, n_req)
+    t = oracle_time(n_req, threads)
+    return {"value": n_req * Hv / t, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one in-place call on {n_req} of the 256 requests of layer 0 ({n_req * Hv} "
+                      f"tokens*heads), C++ double-precision oracle, {threads} threads, {t:.1f} s"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, timed for K steps on a bounded per-step sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cores = cpu_cores()
+    t1 = oracle_time(1, 1)
+    per_step_budget = max(0.2, 150.0 / (args.steps + args.warmup))
+    n_req = int(max(1, min(256, per_step_budget * cores / max(t1, 1e-6) * 0.8)))
+    threads = min(cores, n_req)
+    for _ in range(args.warmup):
+        oracle_time(n_req, threads)
+    total = 0.0
+    for _ in range(args.steps):
+        total += oracle_time(n_req, threads)
+    units = args.steps * n_req * 32
+    value = units / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_requests_per_step": n_req, "layers_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"each step: one in-place call on {n_req} requests of layer 0"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    hbm_peak, peak_kind = peaks()
+    wk = LargeDecode(layers=args.layers, num_slots=args.slots, B=args.batch)
+    stream = torch.cuda.current_stream()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    smi_id = vis.split(",")[local].strip() if vis else str(local)
+    sampler = ClockSampler(smi_id)
+    sampler.start()
+
+    for _ in range(args.warmup):
+        wk.step(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    K, L = args.steps, wk.layers
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+          for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    w0 = time.time()
+    start.record(stream)
+    for s in range(K):
+        for l in range(L):
+            ev[s][l][0].record(stream)
+            wk.launch(l, stream)
+            ev[s][l][1].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    barrier(world)
+    sampler.mark(w0, w1)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
+    launch_ms = statistics.mean(e0.elapsed_time(e1) for row in ev for (e0, e1) in row)
+    launch_ms = max_over_ranks(launch_ms, world)
+    code = wk.gdn.gdn_get_error(wk.err)
+    if code != 0:
+        raise RuntimeError(f"device error word set during the benchmark: {wk.gdn.status_string(code)}")
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        wk.make_host_io()
+        for _ in range(max(3, args.warmup // 2)):
+            wk.step_e2e(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_start.record(stream)
+        for _ in range(K):
+            wk.step_e2e(stream)
+        e_stop.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e_start.elapsed_time(e_stop), world)
+        e2e = {"value": world * K * wk.units_per_step / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": wk.h2d_bytes, "d2h_bytes_per_step": wk.d2h_bytes,
+               "ms_per_step": e2e_ms / K}
+    clocks = sampler.stop()
+
+    G = wk.Hv // wk.Hk
+    bytes_per_unit = algorithmic_bytes_per_unit(wk.dk, wk.dv, G)
+    bytes_per_launch = bytes_per_unit * wk.units_per_launch
+    achieved = bytes_per_launch / (launch_ms / 1e3) / 1e9
+    traffic = None
+    if NCU_TRAFFIC["source_sha256"] == source_sha256() and NCU_TRAFFIC["bytes_per_launch"]:
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    value = world * K * wk.units_per_step / (elapsed_ms / 1e3)
+    step_gbs = bytes_per_launch * L * K / (elapsed_ms / 1e3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": wk.B, "layers": L, "Hk": wk.Hk, "Hv": wk.Hv, "dk": wk.dk,
+                   "dv": wk.dv, "qkv": "bf16", "state": "f32", "slots_per_layer": wk.num_slots,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (4 GiB of state touched per step), no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "gdn_tile_kernel<128,128,256,bf16>",
+                     "bytes_per_launch": bytes_per_launch, "launch_us": launch_ms * 1e3},
+        "hbm_gbs_step": step_gbs, "frac_of_8tbs_step": step_gbs / 8000.0,
+        "e2e": e2e, "gpu_launches": K * L, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--slots", type=int, default=2048)
+    ap.add_argument("--batch", type=int, default=256)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,139 @@
+"""Thin ctypes binding of ``libgdn_b200.so`` (C ABI declared in include/gdn_step.h).
+
+The functions here carry the C entry points' names and only marshal arguments:
+torch CUDA tensors become device pointers, sizes are read off their shapes, and
+the stream defaults to torch's current stream.  All compute runs in the CUDA
+library; there is no fallback.  Loading fails loudly if the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import pathlib
+from typing import Optional
+
+import torch
+
+LIB_PATH = pathlib.Path(__file__).resolve().parent / "libgdn_b200.so"
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARG = 1
+GDN_ERR_CUDA = 2
+GDN_ERR_INDEX = 3
+GDN_ERR_TIMEOUT = 4
+
+GDN_F32 = 0
+GDN_BF16 = 1
+
+_DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"CUDA extension {LIB_PATH.name} is missing: run "
+                           "`python -m hybrid_linear_attention_step_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    lib.gdn_decode_step.restype = i32
+    lib.gdn_decode_step.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                    i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    lib.gdn_commit.restype = i32
+    lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
+    lib.gdn_get_error.restype = i32
+    lib.gdn_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_status_string.argtypes = [i32]
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().gdn_status_string(int(status)).decode()
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _ptr_or_null(t: Optional[torch.Tensor], name: str) -> Optional[int]:
+    return None if t is None else _dev(t, name, torch.int32)
+
+
+def gdn_decode_step(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
+                    q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
+                    err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """Enqueue one GDN decode step (see gdn_decode_step in include/gdn_step.h).
+
+    pool [num_slots, Hv, dk, dv] fp32; src_idx [B] int32; dst_idx [B, T] (or [B]) int32;
+    q, k [B, T, Hk, dk] and v [B, T, Hv, dv] bf16 or fp32; alpha, beta [B, T, Hv] fp32;
+    out [B, T, Hv, dv] fp32.  Returns the status; raises GdnError on failure when ``check``.
+    """
+    if pool.dim() != 4 or q.dim() != 4 or v.dim() != 4:
+        raise ValueError("pool, q, k, v must be 4-D")
+    num_slots, Hv, dk, dv = pool.shape
+    B, T, Hk = q.shape[0], q.shape[1], q.shape[2]
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype: bfloat16 or float32")
+    status = load_library().gdn_decode_step(
+        _dev(pool, "pool", torch.float32), int(num_slots),
+        _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32),
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+        _dev(alpha, "alpha", torch.float32), _dev(beta, "beta", torch.float32),
+        _dev(out, "out", torch.float32),
+        int(B), int(T), int(Hk), int(Hv), int(dk), int(dv), _DTYPES[q.dtype],
+        _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_decode_step")
+    return status
+
+
+def gdn_commit(accept_len: torch.Tensor, committed: torch.Tensor, cur: torch.Tensor, num_slots: int,
+               err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """Enqueue the accept-length commit (see gdn_commit in include/gdn_step.h).
+
+    accept_len [B] int32; committed [B] int32 (updated in place); cur [B, T] int32.
+    """
+    if cur.dim() != 2:
+        raise ValueError("cur must be [B, T]")
+    B, T = cur.shape
+    status = load_library().gdn_commit(
+        _dev(accept_len, "accept_len", torch.int32), _dev(committed, "committed", torch.int32),
+        _dev(cur, "cur", torch.int32), int(B), int(T), int(num_slots),
+        _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_commit")
+    return status
+
+
+def gdn_get_error(err_word: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream, return the device error word's status code and clear it."""
+    code = ctypes.c_int32(-1)
+    status = load_library().gdn_get_error(_dev(err_word, "err_word", torch.int32), ctypes.byref(code),
+                                          _stream_handle(stream))
+    if status != GDN_OK:
+        raise GdnError(status, "gdn_get_error")
+    return int(code.value)

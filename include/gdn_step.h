@@ -1,0 +1,154 @@
+/*
+ * gdn_step.h -- C ABI of the decode-time Gated DeltaNet state update for B200 (sm_100a).
+ *
+ * What is computed.  A hybrid full/linear-attention model keeps, in each Gated
+ * DeltaNet (GDN) linear-attention layer, a recurrent state per request and value
+ * head (TokenSpeed 580 tok/s article, 24-ai.news English edition, opening section
+ * "What is TokenSpeed and how does it differ from vLLM?").  One decode token
+ * updates it with the gated delta rule (Yang, Kautz & Hatamizadeh, "Gated Delta
+ * Networks", ICLR 2025):
+ *
+ *     S' = alpha * S * (I - beta * k k^T) + beta * v k^T,      o = S' q,
+ *
+ * with S the dv x dk fp32 state, k, q in R^dk, v in R^dv and scalar gates alpha,
+ * beta per token and value head.  The library evaluates it in the equivalent
+ * rank-one form u = S k, c = beta * (v - alpha * u), S' = alpha * S + c k^T,
+ * o = alpha * (S q) + c * (k . q), streaming each state through the SM once.
+ *
+ * Where states live.  States sit in a slot pool and are addressed through int32
+ * indices: each request reads slot src and writes slot dst, which may differ.
+ * This is the index indirection that replaces per-step state copies ("Mamba
+ * State Update optimization" item of the 24-ai.news article's "What are the key
+ * optimizations behind the record?"), the copy-on-write reuse of cached prefix
+ * checkpoints (same section, "Hybrid prefix caching for GDN/Mamba"; zubnet.ai
+ * LightSeek TokenSpeed article, second paragraph), and the speculative path in
+ * which per-draft-token states go to the slots named by current_input_indices
+ * (zubnet.ai article, second paragraph).
+ *
+ * Layouts (all row-major, innermost last):
+ *   pool    float [num_slots][Hv][dk][dv]   element [s][h][i][j] = S_h[j][i] of slot s
+ *                                           (the stored tile is S transposed: dv contiguous)
+ *   q, k    [B][T][Hk][dk]   bf16 or fp32 (qkv_dtype)
+ *   v       [B][T][Hv][dv]   bf16 or fp32 (qkv_dtype)
+ *   alpha, beta  float [B][T][Hv]
+ *   out     float [B][T][Hv][dv]
+ *   src_idx int32 [B];  dst_idx int32 [B][T] (current_input_indices when T > 1)
+ * Value head h reads key head h / (Hv / Hk) (contiguous groups); Hv % Hk == 0.
+ * No scaling or normalisation of q and k happens inside the step.
+ *
+ * Ownership and execution.  Every pointer is device memory owned by the caller;
+ * the library allocates nothing, frees nothing and keeps no state between calls.
+ * All work is enqueued on `stream` (0 = legacy default stream); no call
+ * synchronises except gdn_get_error.
+ *
+ * Errors.  Each entry returns a gdn_status.  Bad sizes, a null pointer or an
+ * unknown dtype return GDN_ERR_INVALID_ARG before anything is enqueued; a failed
+ * launch returns GDN_ERR_CUDA.  Index errors are found on the device: the
+ * affected request is skipped (nothing of it is written) and GDN_ERR_INDEX is
+ * recorded in *err_word (first error wins) when err_word is not NULL; read and
+ * clear it with gdn_get_error.  Kernels never trap, assert or wait unboundedly.
+ */
+#ifndef GDN_STEP_H
+#define GDN_STEP_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* sizes, null pointers, dtype: rejected before launch */
+    GDN_ERR_CUDA = 2,        /* a CUDA runtime call or launch failed */
+    GDN_ERR_INDEX = 3,       /* device-side: a slot index or accept length was out of range */
+    GDN_ERR_TIMEOUT = 4      /* device-side: a bounded wait gave up (reserved) */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/*
+ * gdn_decode_step -- one GDN layer's decode update for B requests and T tokens each.
+ *
+ * Defined by the gated delta rule above and the slot scheme of the 24-ai.news
+ * article ("Mamba State Update optimization", "Hybrid prefix caching for
+ * GDN/Mamba") and the zubnet.ai article (second paragraph: state slots,
+ * current_input_indices, copy-on-write checkpoints).
+ *
+ * For each request b, value head h and token t = 0..T-1 the state carried from
+ * pool[src_idx[b]][h] (token 0) or from the previous token is updated with
+ * token t's q, k, v, alpha, beta; the fp32 result is stored to
+ * pool[dst_idx[b*T + t]][h] and carried to token t+1, and o is written to
+ * out[b][t][h][:].  The src slot is only read (copy-on-write) unless it is
+ * also the destination (T == 1 in-place update).
+ *
+ *   pool       device, [num_slots][Hv][dk][dv] fp32, read and written
+ *   num_slots  number of slots in pool (>= 1)
+ *   src_idx    device, int32 [B]
+ *   dst_idx    device, int32 [B*T]
+ *   q, k, v    device, layouts above, element type qkv_dtype
+ *   alpha, beta device, fp32 [B][T][Hv]
+ *   out        device, fp32 [B][T][Hv][dv], written
+ *   B >= 0 (0 is a no-op), T >= 1, Hk >= 1, Hv >= 1 with Hv % Hk == 0,
+ *   1 <= dk <= 4096, dv >= 1, B*Hv < 2^31
+ *   qkv_dtype  GDN_F32 or GDN_BF16
+ *   err_word   device int32, may be NULL (index errors then skip silently)
+ *   stream     CUDA stream the work is enqueued on
+ *
+ * Preconditions (results are unspecified if violated; nothing is written out of
+ * bounds either way): the B*T destination slots are pairwise distinct; no
+ * destination equals another request's source; for T > 1 no destination equals
+ * the request's own source.  Many requests may share one source slot.
+ * Index check: a request whose src or any of its T dst entries lies outside
+ * [0, num_slots) is skipped entirely (no state, no output) and GDN_ERR_INDEX is
+ * recorded.
+ */
+gdn_status gdn_decode_step(float* pool, int32_t num_slots, const int32_t* src_idx,
+                           const int32_t* dst_idx, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta, float* out, int32_t B, int32_t T,
+                           int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int32_t qkv_dtype,
+                           int32_t* err_word, cudaStream_t stream);
+
+/*
+ * gdn_commit -- accept speculative draft tokens by rewriting an int32 index table.
+ *
+ * Defined by the O(1) index update that replaces an O(L*D) state copy (24-ai.news
+ * article, "Mamba State Update optimization") and by speculative decoding through
+ * current_input_indices (zubnet.ai article, second paragraph).  No state byte moves.
+ *
+ * For each request b with a = accept_len[b]:
+ *   a == 0          committed[b] is kept (the pre-draft state stays current);
+ *   1 <= a <= T     committed[b] = cur[b*T + a - 1] (the state after draft token a-1).
+ * The call is idempotent.  The committed table is what the next decode step
+ * passes as src_idx.
+ *
+ *   accept_len device int32 [B]
+ *   committed  device int32 [B], updated in place
+ *   cur        device int32 [B*T] (current_input_indices of the decode call)
+ *   B >= 0 (0 is a no-op), T >= 1, num_slots >= 1
+ *   err_word   device int32, may be NULL
+ * Errors: accept_len outside [0, T], or a selected slot outside [0, num_slots),
+ * leaves committed[b] unchanged and records GDN_ERR_INDEX.
+ */
+gdn_status gdn_commit(const int32_t* accept_len, int32_t* committed, const int32_t* cur, int32_t B,
+                      int32_t T, int32_t num_slots, int32_t* err_word, cudaStream_t stream);
+
+/*
+ * gdn_get_error -- read and clear a device error word.
+ *
+ * Synchronises `stream`, copies *err_word (device) to *host_code (host) and
+ * resets the device word to 0.  *host_code is a gdn_status value (GDN_OK when no
+ * device-side error was recorded).  Returns GDN_ERR_INVALID_ARG for null
+ * pointers and GDN_ERR_CUDA when a runtime call fails.
+ */
+gdn_status gdn_get_error(int32_t* err_word, int32_t* host_code, cudaStream_t stream);
+
+/* Static, NUL-terminated name of a status code ("GDN_OK", ...); never NULL. */
+const char* gdn_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_STEP_H */

@@ -1,0 +1,97 @@
+"""The C-ABI library builds, loads without a GPU, exports every declared entry point,
+and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import pathlib
+import re
+
+import pytest
+
+ROOT = pathlib.Path(__file__).resolve().parent.parent
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hybrid_linear_attention_step_b200 import build
+
+    path = build.build()
+    return ctypes.CDLL(str(path))
+
+
+def declared_functions():
+    names = []
+    for h in sorted((ROOT / "include").glob("*.h")):
+        text = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
+        names += re.findall(r"^\s*(?:gdn_status|const\s+char\s*\*)\s*(gdn_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gdn_decode_step", "gdn_commit", "gdn_get_error", "gdn_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_status_string.argtypes = [ctypes.c_int32]
+    assert [lib.gdn_status_string(i).decode() for i in range(5)] == [
+        "GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_CUDA", "GDN_ERR_INDEX", "GDN_ERR_TIMEOUT"]
+    assert lib.gdn_status_string(99).decode() == "GDN_UNKNOWN_STATUS"
+
+
+def _decode(lib, **kw):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    f = lib.gdn_decode_step
+    f.restype = i32
+    f.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    a = dict(pool=8, num_slots=4, src=8, dst=8, q=8, k=8, v=8, alpha=8, beta=8, out=8,
+             B=1, T=1, Hk=1, Hv=1, dk=16, dv=16, dtype=1, err=None, stream=None)
+    a.update(kw)
+    return f(*a.values())
+
+
+def test_host_validation_before_any_cuda_call(lib):
+    # Each of these must be rejected on the host (no device is present here).
+    assert _decode(lib, B=-1) == 1
+    assert _decode(lib, T=0) == 1
+    assert _decode(lib, Hk=3, Hv=4) == 1
+    assert _decode(lib, dk=5000) == 1
+    assert _decode(lib, dtype=7) == 1
+    assert _decode(lib, num_slots=0) == 1
+    assert _decode(lib, pool=None) == 1
+    assert _decode(lib, out=None) == 1
+    assert _decode(lib, B=0, pool=None, src=None, dst=None) == 0  # empty batch: no-op
+    f = lib.gdn_commit
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int32] * 3 + [ctypes.c_void_p] * 2
+    assert f(8, 8, 8, -1, 1, 4, None, None) == 1
+    assert f(8, 8, 8, 1, 0, 4, None, None) == 1
+    assert f(None, 8, 8, 1, 1, 4, None, None) == 1
+    assert f(None, None, None, 0, 1, 4, None, None) == 0
+    g = lib.gdn_get_error
+    g.restype = ctypes.c_int32
+    g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert g(None, None, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    pytest.importorskip("torch")
+    from hybrid_linear_attention_step_b200 import gdn
+
+    monkeypatch.setattr(gdn, "LIB_PATH", tmp_path / "missing.so")
+    monkeypatch.setattr(gdn, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        gdn.load_library()
+
+
+def test_product_path_never_imports_the_oracle():
+    pkg = ROOT / "hybrid_linear_attention_step_b200"
+    for p in list(pkg.rglob("*.py")) + list(pkg.rglob("*.cu")) + list((ROOT / "include").glob("*.h")):
+        text = p.read_text()
+        assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), p
+        assert "gdn_oracle" not in text, p

@@ -1,0 +1,243 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded bytes.
+
+Bit-exact: which slots are written, untouched slots' bytes, committed index
+tables, error reporting.  Within tolerance: fp32 states (1e-4) and outputs
+(2e-3 with bf16 inputs, 1e-4 with fp32 inputs), as max relative error with the
+reference RMS as floor.
+"""
+import zlib
+
+import numpy as np
+import pytest
+
+from hybrid_linear_attention_step_b200 import workloads as wl
+from tests.gpu_helpers import (TOL_OUT_BF16, TOL_OUT_F32, TOL_STATE, check_pool, rel_err, run_gpu, run_oracle,
+                               step_to_device, to_torch)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+
+    from hybrid_linear_attention_step_b200 import gdn
+
+    gdn.load_library()
+    return torch
+
+
+def _tol_out(s):
+    return TOL_OUT_BF16 if s.dtype == wl.BF16 else TOL_OUT_F32
+
+
+def test_tiny_chain_matches_oracle_and_golden(torch_cuda):
+    from tests.golden import make_golden
+
+    w = wl.tiny(0)
+    dev = to_torch(w.pool)
+    ref_pool = w.pool.copy()
+    outs = []
+    for s in w.steps:
+        before = dev.cpu().numpy()
+        out = run_gpu(dev, s)
+        ref_pool, ref_out, _ = run_oracle(ref_pool, s)
+        assert rel_err(out, ref_out) <= TOL_OUT_F32
+        check_pool(dev.cpu().numpy(), ref_pool, before, s.dst_idx)
+        outs.append(out.reshape(-1))
+    g_outs, g_pool = make_golden.load()
+    assert rel_err(np.stack(outs), g_outs) <= TOL_OUT_F32
+    assert rel_err(dev.cpu().numpy(), g_pool) <= TOL_STATE
+
+
+@pytest.mark.parametrize("name", ["decode_b16", "prefix_cow"])
+def test_decode_workloads(torch_cuda, name):
+    w = wl.WORKLOADS[name]()
+    s = w.steps[0]
+    dev = to_torch(w.pool)
+    out = run_gpu(dev, s)
+    ref_pool, ref_out, skipped = run_oracle(w.pool, s)
+    assert skipped == 0
+    got = dev.cpu().numpy()
+    check_pool(got, ref_pool, w.pool, s.dst_idx)
+    assert rel_err(out, ref_out) <= _tol_out(s)
+    # copy-on-write: every source slot is byte-identical after the call unless it is also written
+    src_only = np.setdiff1d(s.src_idx, s.dst_idx.ravel())
+    assert np.array_equal(got[src_only].view(np.uint32), w.pool[src_only].view(np.uint32))
+
+
+def test_speculative_and_commit(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    w = wl.speculative()
+    s = w.steps[0]
+    dev = to_torch(w.pool)
+    out = run_gpu(dev, s)
+    ref_pool, ref_out, _ = run_oracle(w.pool, s)
+    got = dev.cpu().numpy()
+    check_pool(got, ref_pool, w.pool, s.dst_idx)
+    assert rel_err(out, ref_out) <= TOL_OUT_BF16
+
+    # commit: bit-exact index table, no pool byte changes
+    import oracle
+
+    committed = torch.from_numpy(s.src_idx.copy()).cuda()
+    cur = torch.from_numpy(s.dst_idx.copy()).cuda()
+    accept = torch.from_numpy(s.accept_len.copy()).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool_before = dev.clone()
+    gdn.gdn_commit(accept, committed, cur, w.num_slots, err_word=err)
+    want = s.src_idx.copy()
+    assert oracle.commit(s.accept_len, want, s.dst_idx, w.num_slots) == 0
+    assert np.array_equal(committed.cpu().numpy(), want)
+    assert torch.equal(dev.view(torch.int32), pool_before.view(torch.int32))
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    gdn.gdn_commit(accept, committed, cur, w.num_slots)  # idempotent
+    assert np.array_equal(committed.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F32])
+def test_sequential_equals_speculative_bitwise(torch_cuda, dtype):
+    """T chained single-token calls and one T-token call give identical bits on the GPU."""
+    rng = np.random.default_rng(40)
+    num_slots, B, T, Hk, Hv, dk, dv = 40, 4, 4, 2, 4, 128, 128
+    pool = wl.init_pool(rng, num_slots, Hv, dk, dv)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, T, Hk, Hv, dk, dv, dtype)
+    src = np.arange(B, dtype=np.int32)
+    cur = (B + np.arange(B * T, dtype=np.int32)).reshape(B, T)
+    spec = to_torch(pool)
+    out_spec = run_gpu(spec, wl.Step(q, k, v, a, b, src, cur))
+    seq = to_torch(pool)
+    prev = src
+    for t in range(T):
+        sl = lambda x: np.ascontiguousarray(x[:, t:t + 1])
+        o = run_gpu(seq, wl.Step(sl(q), sl(k), sl(v), sl(a), sl(b), prev.copy(), sl(cur)))
+        assert np.array_equal(o[:, 0], out_spec[:, t])
+        prev = cur[:, t].copy()
+    assert np.array_equal(seq.cpu().numpy().view(np.uint32), spec.cpu().numpy().view(np.uint32))
+
+
+SHAPES = [
+    # (B, T, Hk, Hv, dk, dv, dtype, in_place)
+    (3, 1, 1, 1, 16, 16, wl.F32, False),
+    (5, 2, 2, 4, 3, 5, wl.BF16, False),
+    (4, 1, 2, 2, 64, 64, wl.BF16, True),
+    (3, 3, 1, 3, 64, 64, wl.F32, False),
+    (2, 2, 1, 2, 100, 72, wl.BF16, False),
+    (6, 1, 4, 8, 128, 128, wl.F32, True),
+    (3, 2, 2, 2, 256, 128, wl.BF16, False),
+    (2, 1, 1, 1, 128, 300, wl.BF16, True),
+    (1, 5, 1, 1, 1, 1, wl.F32, False),
+    (7, 1, 1, 2, 33, 257, wl.F32, False),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}T{}Hk{}Hv{}dk{}dv{}{}{}".format(*s[:7], "ip" if s[7] else ""))
+def test_shapes_and_ragged_tails(torch_cuda, shape):
+    B, T, Hk, Hv, dk, dv, dtype, in_place = shape
+    rng = np.random.default_rng(zlib.crc32(repr(shape).encode()))
+    num_slots = B * (T + 1) + 3
+    pool = wl.init_pool(rng, num_slots, Hv, dk, dv)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, T, Hk, Hv, dk, dv, dtype)
+    perm = rng.permutation(num_slots).astype(np.int32)
+    src = perm[:B].copy()
+    dst = src.reshape(B, 1).copy() if in_place else perm[B:B + B * T].reshape(B, T).copy()
+    s = wl.Step(q, k, v, a, b, src, dst)
+    dev = to_torch(pool)
+    out = run_gpu(dev, s)
+    ref_pool, ref_out, _ = run_oracle(pool, s)
+    check_pool(dev.cpu().numpy(), ref_pool, pool, dst)
+    assert rel_err(out, ref_out) <= _tol_out(s)
+
+
+def test_empty_batch_is_a_no_op(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    pool = torch.ones((2, 1, 128, 128), device="cuda")
+    e = torch.zeros((0, 1, 1, 128), dtype=torch.bfloat16, device="cuda")
+    ab = torch.zeros((0, 1, 1), device="cuda")
+    idx = torch.zeros((0,), dtype=torch.int32, device="cuda")
+    out = torch.zeros((0, 1, 1, 128), device="cuda")
+    assert gdn.gdn_decode_step(pool, idx, idx.view(0, 1), e, e, e, ab, ab, out) == gdn.GDN_OK
+    assert gdn.gdn_commit(idx, idx, idx.view(0, 1), 2) == gdn.GDN_OK
+    torch.cuda.synchronize()
+    assert bool((pool == 1).all())
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (20, 24)])
+def test_out_of_range_indices_skip_and_report(torch_cuda, dk, dv):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(50)
+    num_slots, B, T = 12, 4, 2
+    pool = wl.init_pool(rng, num_slots, 2, dk, dv)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, T, 1, 2, dk, dv, wl.BF16)
+    src = np.array([0, num_slots, 2, -1], np.int32)
+    dst = np.array([[4, 5], [6, 7], [8, 99], [10, 11]], np.int32)
+    s = wl.Step(q, k, v, a, b, src, dst)
+    dev = to_torch(pool)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_gpu(dev, s, err=err)
+    ref_pool, ref_out, skipped = run_oracle(pool, s)
+    assert skipped == 3
+    assert gdn.gdn_get_error(err) == gdn.GDN_ERR_INDEX
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK  # read-and-clear
+    got = dev.cpu().numpy()
+    check_pool(got, ref_pool, pool, dst[:1])
+    assert np.all(out[1:] == -7.0)
+    assert rel_err(out[:1], ref_out[:1]) <= TOL_OUT_BF16
+
+    accept = torch.tensor([1, -1, T + 1, 2], dtype=torch.int32, device="cuda")
+    cur = torch.tensor([[4, 5], [6, 7], [8, 9], [10, num_slots + 4]], dtype=torch.int32, device="cuda")
+    committed = torch.tensor([0, 1, 2, 3], dtype=torch.int32, device="cuda")
+    gdn.gdn_commit(accept, committed, cur, num_slots, err_word=err)
+    assert committed.cpu().tolist() == [4, 1, 2, 3]
+    assert gdn.gdn_get_error(err) == gdn.GDN_ERR_INDEX
+
+
+def test_unaligned_pool_uses_column_path(torch_cuda):
+    """A pool that starts off a 16-byte boundary still gives oracle results."""
+    torch = torch_cuda
+    w = wl.decode_b16()
+    s = w.steps[0]
+    n = w.pool.size
+    buf = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    dev = buf[1:].view(w.pool.shape)
+    dev.copy_(torch.from_numpy(w.pool))
+    out = run_gpu(dev, s)
+    ref_pool, ref_out, _ = run_oracle(w.pool, s)
+    check_pool(dev.cpu().numpy(), ref_pool, w.pool, s.dst_idx)
+    assert rel_err(out, ref_out) <= TOL_OUT_BF16
+
+
+def test_side_stream(torch_cuda):
+    torch = torch_cuda
+    w = wl.decode_b16()
+    s = w.steps[0]
+    dev = to_torch(w.pool)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        out = run_gpu(dev, s, stream=st)
+    ref_pool, ref_out, _ = run_oracle(w.pool, s)
+    check_pool(dev.cpu().numpy(), ref_pool, w.pool, s.dst_idx)
+    assert rel_err(out, ref_out) <= TOL_OUT_BF16
+
+
+def test_invalid_arguments_raise(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    w = wl.decode_b16()
+    s = w.steps[0]
+    x = step_to_device(s)
+    pool = torch.zeros((4, 32, 128, 128), device="cuda")
+    out = torch.zeros((16, 1, 32, 128), device="cuda")
+    with pytest.raises(gdn.GdnError) as ei:  # Hv = 32 not a multiple of Hk = 3
+        gdn.gdn_decode_step(pool, x["src"], x["dst"], x["q"][:, :, :3].contiguous(), x["k"][:, :, :3].contiguous(),
+                            x["v"], x["alpha"], x["beta"], out)
+    assert ei.value.status == gdn.GDN_ERR_INVALID_ARG
+    with pytest.raises(TypeError):
+        gdn.gdn_decode_step(pool, x["src"], x["dst"], x["q"], x["k"], x["v"].float(), x["alpha"], x["beta"], out)
