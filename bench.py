@@ -44,7 +44,9 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).  See profiles/.
-NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "profile": None}
+NCU_TRAFFIC = {"source_sha256": "0601db0eb8524fa0b331ef6c8f4e6583bcfbaff0676f759b9efbe997185a500e",
+               "bytes_per_launch": 541150720 + 483911936,
+               "profile": "profiles/gdn_tile_kernel_large_decode.md"}
 
 
 def algorithmic_bytes_per_unit(dk: int, dv: int, G: int, in_bytes: int = 2, T: int = 1) -> float:

@@ -70,17 +70,22 @@ def run_oracle(pool: np.ndarray, s: wl.Step, out_fill=-7.0, nthreads=8):
     return pool, out, skipped
 
 
-def check_pool(got: np.ndarray, ref: np.ndarray, before: np.ndarray, written: np.ndarray):
+def check_pool(got: np.ndarray, ref: np.ndarray, before: np.ndarray, written: np.ndarray,
+               ref_before: np.ndarray = None):
     """Bit-exact slot behaviour plus in-tolerance state values.
 
-    * every slot outside ``written`` is byte-identical to ``before`` on both sides;
+    * every slot outside ``written`` keeps its bytes: ``got`` against ``before``
+      (the device pool before the call) and ``ref`` against ``ref_before`` (the
+      oracle's pool before the call, by default the same array);
     * the written slots agree with the oracle within TOL_STATE.
     """
+    if ref_before is None:
+        ref_before = before
     num_slots = before.shape[0]
     untouched = np.setdiff1d(np.arange(num_slots), np.asarray(written).ravel())
     assert np.array_equal(got[untouched].view(np.uint32), before[untouched].view(np.uint32)), \
         "CUDA path changed a slot it does not own"
-    assert np.array_equal(ref[untouched].view(np.uint32), before[untouched].view(np.uint32))
+    assert np.array_equal(ref[untouched].view(np.uint32), ref_before[untouched].view(np.uint32))
     w = np.unique(np.asarray(written).ravel())
     e = rel_err(got[w], ref[w])
     assert e <= TOL_STATE, f"state rel err {e:.3g} > {TOL_STATE}"

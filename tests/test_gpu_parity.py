@@ -39,11 +39,11 @@ def test_tiny_chain_matches_oracle_and_golden(torch_cuda):
     ref_pool = w.pool.copy()
     outs = []
     for s in w.steps:
-        before = dev.cpu().numpy()
+        before, ref_before = dev.cpu().numpy(), ref_pool
         out = run_gpu(dev, s)
         ref_pool, ref_out, _ = run_oracle(ref_pool, s)
         assert rel_err(out, ref_out) <= TOL_OUT_F32
-        check_pool(dev.cpu().numpy(), ref_pool, before, s.dst_idx)
+        check_pool(dev.cpu().numpy(), ref_pool, before, s.dst_idx, ref_before)
         outs.append(out.reshape(-1))
     g_outs, g_pool = make_golden.load()
     assert rel_err(np.stack(outs), g_outs) <= TOL_OUT_F32
