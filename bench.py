@@ -44,9 +44,15 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).  See profiles/.
-NCU_TRAFFIC = {"source_sha256": "0601db0eb8524fa0b331ef6c8f4e6583bcfbaff0676f759b9efbe997185a500e",
+NCU_TRAFFIC = {"kernel": "gdn_tile_kernel<128,128,256,bf16>",
+               "source_sha256": "0601db0eb8524fa0b331ef6c8f4e6583bcfbaff0676f759b9efbe997185a500e",
                "bytes_per_launch": 541150720 + 483911936,
                "profile": "profiles/gdn_tile_kernel_large_decode.md"}
+
+# Kernel that serves the large decode for each --variant ("auto" picks the
+# single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
+KERNEL_NAMES = {"auto": "gdn_tile1_kernel<128,128,64,128,5,bf16>", "tile": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
+                "stream": "gdn_stream_kernel<256,bf16>", "column": "gdn_column_kernel<bf16>"}
 
 
 def algorithmic_bytes_per_unit(dk: int, dv: int, G: int, in_bytes: int = 2, T: int = 1) -> float:
@@ -76,7 +82,11 @@ def source_sha256() -> str:
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works."""
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works.
+
+    A reader thread collects one CSV line per sample; ``start`` returns once the
+    first sample has arrived (or after a few seconds if nvidia-smi is absent).
+    """
 
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
               "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -88,8 +98,16 @@ class ClockSampler:
         self.gpu_index = gpu_index
         self.interval_ms = interval_ms
         self.window = None
+        self.lines = []
+        self.thread = None
 
-    def start(self):
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line))
+
+    def start(self, wait_s: float = 5.0):
+        import threading
+
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
@@ -97,6 +115,12 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < wait_s and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def mark(self, t0: float, t1: float):
         self.window = (t0, t1)
@@ -106,17 +130,18 @@ class ClockSampler:
             return None
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=10)
+            self.proc.wait(timeout=10)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
         rows = []
-        for r in csv.reader(io.StringIO(out)):
+        for t_host, line in list(self.lines):
+            r = next(csv.reader([line]), [])
             if len(r) < 11:
                 continue
             try:
-                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                rows.append(dict(ts=ts, sm=float(r[2]), sm_max=float(r[3]), power=float(r[4]),
+                rows.append(dict(ts=t_host, sm=float(r[2]), sm_max=float(r[3]), power=float(r[4]),
                                  util=float(r[5]), hw=r[7].strip(), hw_th=r[8].strip(),
                                  sw_th=r[9].strip(), pcap=r[10].strip()))
             except ValueError:
@@ -125,7 +150,7 @@ class ClockSampler:
             return None
         picked, where = rows, "all"
         if self.window:
-            inside = [r for r in rows if self.window[0] - 0.05 <= r["ts"] <= self.window[1] + 0.05]
+            inside = [r for r in rows if self.window[0] <= r["ts"] <= self.window[1] + 0.1]
             if len(inside) >= 3:
                 picked, where = inside, "timed"
             else:
@@ -149,7 +174,7 @@ class LargeDecode:
     """Device-resident large decode: ``layers`` pools, per-layer inputs, one step = ``layers`` calls."""
 
     def __init__(self, layers: int = 8, num_slots: int = 2048, B: int = 256, device: str = "cuda",
-                 seed: int = 4):
+                 seed: int = 4, variant: str = "auto"):
         import numpy as np
         import torch
 
@@ -160,6 +185,7 @@ class LargeDecode:
         self.layers, self.num_slots, self.B = layers, num_slots, B
         self.Hk, self.Hv, self.dk, self.dv = c["Hk"], c["Hv"], c["dk"], c["dv"]
         self.seed = seed
+        self.variant = variant
         self.device = torch.device(device)
         self.host_steps = [wl.large_layer_step(l, seed, B, num_slots) for l in range(layers)]
         self.pools, self.inputs, self.outs = [], [], []
@@ -187,8 +213,11 @@ class LargeDecode:
 
     def launch(self, l: int, stream=None):
         x = self.inputs[l]
-        self.gdn.gdn_decode_step(self.pools[l], x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"],
-                                 x["beta"], self.outs[l], err_word=self.err, stream=stream)
+        args = (self.pools[l], x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], self.outs[l])
+        if self.variant == "auto":
+            self.gdn.gdn_decode_step(*args, err_word=self.err, stream=stream)
+        else:
+            self.gdn.gdn_decode_step_variant(*args, self.variant, err_word=self.err, stream=stream)
 
     def step(self, stream=None):
         for l in range(self.layers):
@@ -203,13 +232,47 @@ class LargeDecode:
         self.h2d_bytes = sum(t.numel() * t.element_size() for x in self.h_in for t in x.values())
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.h_out)
 
+    def make_e2e_streams(self):
+        """Copy-in, compute and copy-out streams plus the per-layer events that
+        order them (inputs of layer l are overwritten only after the previous
+        step's kernel l has read them; out[l] only after it has been copied out)."""
+        import torch
+
+        self.s_in, self.s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        self.ev_in = [torch.cuda.Event() for _ in range(self.layers)]
+        self.ev_run = [torch.cuda.Event() for _ in range(self.layers)]
+        self.ev_out = [torch.cuda.Event() for _ in range(self.layers)]
+        self.e2e_primed = False
+
     def step_e2e(self, stream):
+        """One step end to end: per layer, H2D of its inputs (pinned host -> device),
+        the decode call, D2H of its output; copies of other layers overlap the
+        kernels (the pages' async H2D with event-based layer barriers)."""
+        import torch
+
         for l in range(self.layers):
             x, hx = self.inputs[l], self.h_in[l]
-            for key in ("q", "k", "v", "alpha", "beta", "src", "dst"):
-                x[key].copy_(hx[key], non_blocking=True)
+            with torch.cuda.stream(self.s_in):
+                if self.e2e_primed:
+                    self.s_in.wait_event(self.ev_run[l])
+                for key in ("q", "k", "v", "alpha", "beta", "src", "dst"):
+                    x[key].copy_(hx[key], non_blocking=True)
+                self.ev_in[l].record(self.s_in)
+            stream.wait_event(self.ev_in[l])
+            if self.e2e_primed:
+                stream.wait_event(self.ev_out[l])
             self.launch(l, stream)
-            self.h_out[l].copy_(self.outs[l], non_blocking=True)
+            self.ev_run[l].record(stream)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.ev_run[l])
+                self.h_out[l].copy_(self.outs[l], non_blocking=True)
+                self.ev_out[l].record(self.s_out)
+        self.e2e_primed = True
+
+    def join_e2e(self, stream):
+        """Make ``stream`` wait for every copy of the steps issued so far."""
+        stream.wait_stream(self.s_in)
+        stream.wait_stream(self.s_out)
 
 
 # ----------------------------------------------------------------- ranks
@@ -332,7 +395,8 @@ def run_ours(args):
     rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     hbm_peak, peak_kind = peaks()
-    wk = LargeDecode(layers=args.layers, num_slots=args.slots, B=args.batch)
+    wk = LargeDecode(layers=args.layers, num_slots=args.slots, B=args.batch, variant=args.variant)
+    kernel = KERNEL_NAMES[args.variant]
     stream = torch.cuda.current_stream()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
     smi_id = vis.split(",")[local].strip() if vis else str(local)
@@ -345,26 +409,36 @@ def run_ours(args):
     barrier(world)
 
     K, L = args.steps, wk.layers
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-          for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(world)
     w0 = time.time()
     start.record(stream)
-    for s in range(K):
-        for l in range(L):
-            ev[s][l][0].record(stream)
-            wk.launch(l, stream)
-            ev[s][l][1].record(stream)
+    for _ in range(K):
+        wk.step(stream)
     stop.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
     barrier(world)
     sampler.mark(w0, w1)
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
-    launch_ms = statistics.mean(e0.elapsed_time(e1) for row in ev for (e0, e1) in row)
-    launch_ms = max_over_ranks(launch_ms, world)
+    # Every launch in the timed region is the same kernel on the same stream:
+    # its average duration is the region over the launch count (gaps included).
+    launch_ms = elapsed_ms / (K * L)
+
+    # Diagnostic pass, outside the timed region: the same K steps with an
+    # event pair around every launch (the events themselves add a few us each).
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K * L)]
+    for s_ in range(K):
+        for l in range(L):
+            e0, e1 = ev[s_ * L + l]
+            e0.record(stream)
+            wk.launch(l, stream)
+            e1.record(stream)
+    torch.cuda.synchronize()
+    durs = sorted(e0.elapsed_time(e1) for e0, e1 in ev)
+    launch_events = {"mean_us": 1e3 * statistics.mean(durs), "median_us": 1e3 * durs[len(durs) // 2],
+                     "min_us": 1e3 * durs[0], "max_us": 1e3 * durs[-1]}
     code = wk.gdn.gdn_get_error(wk.err)
     if code != 0:
         raise RuntimeError(f"device error word set during the benchmark: {wk.gdn.status_string(code)}")
@@ -373,14 +447,19 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         wk.make_host_io()
+        wk.make_e2e_streams()
         for _ in range(max(3, args.warmup // 2)):
             wk.step_e2e(stream)
+        wk.join_e2e(stream)
         torch.cuda.synchronize()
         barrier(world)
         e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e_start.record(stream)
+        wk.s_in.wait_event(e_start)
+        wk.s_out.wait_event(e_start)
         for _ in range(K):
             wk.step_e2e(stream)
+        wk.join_e2e(stream)
         e_stop.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -395,24 +474,25 @@ def run_ours(args):
     bytes_per_launch = bytes_per_unit * wk.units_per_launch
     achieved = bytes_per_launch / (launch_ms / 1e3) / 1e9
     traffic = None
-    if NCU_TRAFFIC["source_sha256"] == source_sha256() and NCU_TRAFFIC["bytes_per_launch"]:
+    if (NCU_TRAFFIC["source_sha256"] == source_sha256() and NCU_TRAFFIC["kernel"] == kernel
+            and NCU_TRAFFIC["bytes_per_launch"]):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
     value = world * K * wk.units_per_step / (elapsed_ms / 1e3)
-    step_gbs = bytes_per_launch * L * K / (elapsed_ms / 1e3) / 1e9
+    step_gbs = bytes_per_launch * L * K / (elapsed_ms / 1e3) / 1e9  # equals roofline.achieved here
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": wk.B, "layers": L, "Hk": wk.Hk, "Hv": wk.Hv, "dk": wk.dk,
+        "config": {"workload": WORKLOAD, "variant": args.variant, "B": wk.B, "layers": L, "Hk": wk.Hk, "Hv": wk.Hv, "dk": wk.dk,
                    "dv": wk.dv, "qkv": "bf16", "state": "f32", "slots_per_layer": wk.num_slots,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (4 GiB of state touched per step), no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
-                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "gdn_tile_kernel<128,128,256,bf16>",
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": kernel,
                      "bytes_per_launch": bytes_per_launch, "launch_us": launch_ms * 1e3},
-        "hbm_gbs_step": step_gbs, "frac_of_8tbs_step": step_gbs / 8000.0,
+        "hbm_gbs_step": step_gbs, "launch_events": launch_events, "frac_of_8tbs_step": step_gbs / 8000.0,
         "e2e": e2e, "gpu_launches": K * L, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -434,6 +514,8 @@ def main():
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--slots", type=int, default=2048)
     ap.add_argument("--batch", type=int, default=256)
+    ap.add_argument("--variant", choices=["auto", "stream", "tile", "column"], default="auto",
+                    help="kernel for the decode calls (auto = what gdn_decode_step picks)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

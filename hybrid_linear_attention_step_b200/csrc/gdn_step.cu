@@ -198,6 +198,132 @@ __global__ void __launch_bounds__(NT, 2) gdn_tile_kernel(StepArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Single-token register-tile kernel.  Value columns are independent, so a
+// (b, h) tile is split into DV / DVC column blocks, one CTA each (a column
+// block's rows are DVC * 4 contiguous bytes, read and written as float4 runs).
+// Thread layout per CTA: CG = DVC / 4 column groups x RG = NT / CG row groups,
+// rows i = m * RG + rg.  Every input the CTA needs (tile block, k and q rows,
+// its v columns, the gates, the slot indices) is requested at kernel start, so
+// after the tile lands the only waits are two barriers; shared memory stays
+// small, leaving the unified L1 large enough to track the outstanding misses
+// of the MINB CTAs resident per SM.
+// ---------------------------------------------------------------------------
+template <int DK, int DV, int DVC, int NT, int MINB, typename InT>
+__global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
+    constexpr int CG = DVC / 4;
+    static_assert(DV % DVC == 0 && DVC % 4 == 0 && NT % CG == 0 && NT >= 32, "tile shape");
+    constexpr int RG = NT / CG;
+    static_assert(DK % RG == 0, "tile shape");
+    constexpr int RPT = DK / RG;
+    constexpr int NC = DV / DVC;
+
+    __shared__ float ks[DK];
+    __shared__ float qs[DK];
+    __shared__ float vs[DVC];
+    __shared__ float gates[2];
+    __shared__ int dst_s;
+    __shared__ float4 red_u[RG][CG];
+    __shared__ float4 red_w[RG][CG];
+    __shared__ float kq_s;
+
+    const int tid = threadIdx.x;
+    const int cg = tid % CG;
+    const int rg = tid / CG;
+    const int chunk = blockIdx.x % NC;
+    const int unit = blockIdx.x / NC;
+    const int h = unit % a.Hv;
+    const int b = unit / a.Hv;
+
+    const int src = __ldg(a.src_idx + b);
+    const int dst = __ldg(a.dst_idx + b);
+    if (src < 0 || src >= a.num_slots || dst < 0 || dst >= a.num_slots) {
+        if (tid == 0) record_error(a.err, GDN_ERR_INDEX);
+        return;
+    }
+
+    // float4 offset of (row i, this thread's columns) inside a tile: i * DV / 4 + chunk * CG + cg;
+    // the thread's rows are rg + m * RG, so its base is row rg and the step is RG rows.
+    const int col4 = chunk * CG + cg;
+    const int toff = rg * (DV / 4) + col4;
+    constexpr int kRowStep = RG * (DV / 4);
+    const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV)) + toff;
+    float4 s[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+
+    const size_t gh = (size_t)b * a.Hv + h;  // token index = b for a single token
+    const size_t kbase = ((size_t)b * a.Hk + h / a.G) * DK;
+    for (int i = tid; i < DK; i += NT) {
+        ks[i] = load_in<InT>(a.k, kbase + i);
+        qs[i] = load_in<InT>(a.q, kbase + i);
+    }
+    // v and the gates go through shared memory too: staged now, read after
+    // the reduction, they cost no registers while the tile is in flight.
+    for (int j = tid; j < DVC; j += NT) vs[j] = load_in<InT>(a.v, gh * DV + (size_t)chunk * DVC + j);
+    if (tid == 0) {
+        gates[0] = __ldg(a.alpha + gh);
+        gates[1] = __ldg(a.beta + gh);
+        dst_s = dst;  // re-read after the reduction instead of holding a register
+    }
+    __syncthreads();
+
+    float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const int i = m * RG + rg;
+        fma4(pu, s[m], ks[i]);
+        fma4(pw, s[m], qs[i]);
+    }
+    red_u[rg][cg] = pu;
+    red_w[rg][cg] = pw;
+    if (tid < 32) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = tid; i < DK; i += 32) acc = fmaf(ks[i], qs[i], acc);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (tid == 0) kq_s = acc;
+    }
+    __syncthreads();
+
+    float4 u = red_u[0][cg];
+    float4 w = red_w[0][cg];
+#pragma unroll
+    for (int r = 1; r < RG; ++r) {
+        add4(u, red_u[r][cg]);
+        add4(w, red_w[r][cg]);
+    }
+    const float al = gates[0];
+    const float be = gates[1];
+    const float4 vv = reinterpret_cast<const float4*>(vs)[cg];
+    float4 c;
+    c.x = be * (vv.x - al * u.x);
+    c.y = be * (vv.y - al * u.y);
+    c.z = be * (vv.z - al * u.z);
+    c.w = be * (vv.w - al * u.w);
+    if (rg == 0) {
+        const float kq = kq_s;
+        float4 o;
+        o.x = fmaf(c.x, kq, al * w.x);
+        o.y = fmaf(c.y, kq, al * w.y);
+        o.z = fmaf(c.z, kq, al * w.z);
+        o.w = fmaf(c.w, kq, al * w.w);
+        __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + col4, o);
+    }
+    float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst_s * a.Hv + h) * (DK * DV)) + toff;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const float ki = ks[m * RG + rg];
+        s[m].x = fmaf(ki, c.x, al * s[m].x);
+        s[m].y = fmaf(ki, c.y, al * s[m].y);
+        s[m].z = fmaf(ki, c.z, al * s[m].z);
+        s[m].w = fmaf(ki, c.w, al * s[m].w);
+        __stcs(D + m * kRowStep, s[m]);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Column kernel for any (dk, dv): one thread per value column j, one CTA per
 // (b, h, chunk of columns).  Pass 1 reduces u_j, w_j down column j; pass 2
 // re-reads the column and writes the update.  Token t > 0 reads the slot token
@@ -258,6 +384,288 @@ __global__ void gdn_column_kernel(StepArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Bulk-copy helpers (sm_90+ PTX, used on sm_100a): mbarrier transaction
+// counting and one-dimensional cp.async.bulk global -> shared copies.  No
+// multicast and no tensor maps: every copy is a contiguous, 16-byte aligned
+// range of this GPU's own memory.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Every wait on a copy gives up after this long and reports GDN_ERR_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Waits for the phase with the given parity; false if the limit ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+template <typename InT>
+__device__ __forceinline__ float smem_in(const InT* p, int i);
+template <>
+__device__ __forceinline__ float smem_in<float>(const float* p, int i) {
+    return p[i];
+}
+template <>
+__device__ __forceinline__ float smem_in<__nv_bfloat16>(const __nv_bfloat16* p, int i) {
+    return __bfloat162float(p[i]);
+}
+
+// Shared-memory plan of the streaming kernel (dk = dv = 128, one token).
+// Each of the STAGES buffers holds one unit's state tile plus its q, k and v
+// rows and the 16-byte chunks of alpha and beta that contain its gate values.
+// The cross-row-group reduction buffers and k.q are double-buffered by unit
+// parity, so one barrier per unit suffices.
+template <int NT, typename InT>
+struct StreamPlan {
+    static constexpr int DK = 128, DV = 128, STAGES = 3;
+    static constexpr int CG = DV / 4, RG = NT / CG, RPT = DK / RG;
+    static constexpr uint32_t TILE_BYTES = DK * DV * 4;
+    static constexpr uint32_t ROW_BYTES = 128 * sizeof(InT);
+    static constexpr uint32_t Q_OFF = TILE_BYTES, K_OFF = Q_OFF + ROW_BYTES, V_OFF = K_OFF + ROW_BYTES;
+    static constexpr uint32_t A_OFF = V_OFF + ROW_BYTES, B_OFF = A_OFF + 16;
+    static constexpr uint32_t STAGE_TX = B_OFF + 16;  // bytes landed per unit
+    static constexpr uint32_t STAGE_STRIDE = (STAGE_TX + 127) / 128 * 128;
+    static constexpr uint32_t RED_OFF = STAGES * STAGE_STRIDE;
+    static constexpr uint32_t RED_BYTES = 2 * RG * CG * 16;  // u and w partials of one unit
+    static constexpr uint32_t BAR_OFF = RED_OFF + 2 * RED_BYTES;
+    static constexpr uint32_t META_OFF = BAR_OFF + STAGES * 8;
+    static constexpr uint32_t KQ_OFF = META_OFF + STAGES * 8;
+    static constexpr uint32_t SMEM_BYTES = KQ_OFF + 16;
+    static_assert(NT % CG == 0 && DK % RG == 0, "thread layout");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory plan exceeds the per-CTA limit");
+};
+
+// ---------------------------------------------------------------------------
+// Streaming kernel for single-token decode at dk = dv = 128.  Persistent: one
+// CTA per SM walks units u = blockIdx.x + n * gridDim.x (u = b * Hv + h).
+// Thread 0 keeps STAGES units in flight with bulk copies (state tile, q/k/v
+// rows, gate chunks) and prefetches slot indices one unit ahead.  All threads
+// consume one landed unit at a time: tile, k, v and gates -> registers and
+// partial reductions; one barrier, after which the stage is refilled with the
+// unit STAGES ahead while the threads finish the reduction, update the tile in
+// registers and stream it straight to the destination slot.  The tile is read
+// from HBM once and written once; the next STAGES tiles are in flight while
+// the current one is reduced and stored.
+// ---------------------------------------------------------------------------
+template <int NT, typename InT>
+__global__ void __launch_bounds__(NT, 1) gdn_stream_kernel(StepArgs a) {
+    using P = StreamPlan<NT, InT>;
+    constexpr int CG = P::CG, RG = P::RG, RPT = P::RPT, STAGES = P::STAGES;
+    extern __shared__ __align__(128) unsigned char sbuf[];
+    float4* red_base = reinterpret_cast<float4*>(sbuf + P::RED_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sbuf + P::BAR_OFF);
+    int2* meta = reinterpret_cast<int2*>(sbuf + P::META_OFF);
+    float* kq_s = reinterpret_cast<float*>(sbuf + P::KQ_OFF);
+
+    const int tid = threadIdx.x;
+    const int cg = tid % CG;
+    const int rg = tid / CG;
+    const int units = a.B * a.Hv;
+    const int grid = gridDim.x;
+    const int n_local = (units - (int)blockIdx.x + grid - 1) / grid;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    // Producer state, meaningful in thread 0 only.
+    int p_next = 0;
+    int nx_src = 0, nx_dst = 0;
+    auto fetch_indices = [&](int n) {
+        const int b = ((int)blockIdx.x + n * grid) / a.Hv;
+        nx_src = __ldg(a.src_idx + b);
+        nx_dst = __ldg(a.dst_idx + b);
+    };
+    auto issue = [&]() {
+        const int n = p_next;
+        const int u = (int)blockIdx.x + n * grid;
+        const int b = u / a.Hv, h = u % a.Hv;
+        const int src = nx_src, dst = nx_dst;
+        ++p_next;
+        if (p_next < n_local) fetch_indices(p_next);
+        const int stage = n % STAGES;
+        const bool valid = src >= 0 && src < a.num_slots && dst >= 0 && dst < a.num_slots;
+        meta[stage] = make_int2(dst, valid ? 1 : 0);
+        uint64_t* bar = &bars[stage];
+        if (!valid) {
+            mbar_arrive(bar);
+            return;
+        }
+        unsigned char* st = sbuf + stage * P::STAGE_STRIDE;
+        const size_t gh = (size_t)b * a.Hv + h;
+        const size_t row = ((size_t)b * a.Hk + h / a.G) * P::DK;
+        mbar_arrive_expect_tx(bar, P::STAGE_TX);
+        bulk_g2s(st, a.pool + ((size_t)src * a.Hv + h) * (P::DK * P::DV), P::TILE_BYTES, bar);
+        bulk_g2s(st + P::Q_OFF, static_cast<const InT*>(a.q) + row, P::ROW_BYTES, bar);
+        bulk_g2s(st + P::K_OFF, static_cast<const InT*>(a.k) + row, P::ROW_BYTES, bar);
+        bulk_g2s(st + P::V_OFF, static_cast<const InT*>(a.v) + gh * P::DV, P::ROW_BYTES, bar);
+        bulk_g2s(st + P::A_OFF, a.alpha + (gh & ~(size_t)3), 16, bar);
+        bulk_g2s(st + P::B_OFF, a.beta + (gh & ~(size_t)3), 16, bar);
+    };
+
+    if (tid == 0) {
+        if (n_local > 0) fetch_indices(0);
+        while (p_next < n_local && p_next < STAGES) issue();
+    }
+    __syncthreads();  // meta[] of the prologue's units is visible to every thread
+
+    for (int n = 0; n < n_local; ++n) {
+        const int stage = n % STAGES;
+        const uint32_t parity = (uint32_t)(n / STAGES) & 1u;
+        const int2 m = meta[stage];
+        const bool landed = mbar_wait_bounded(&bars[stage], parity);
+
+        const unsigned char* st = sbuf + stage * P::STAGE_STRIDE;
+        const float4* tile = reinterpret_cast<const float4*>(st);
+        const InT* qsm = reinterpret_cast<const InT*>(st + P::Q_OFF);
+        const InT* ksm = reinterpret_cast<const InT*>(st + P::K_OFF);
+        const InT* vsm = reinterpret_cast<const InT*>(st + P::V_OFF);
+        float4* red_u = red_base + (n & 1) * (2 * RG * CG);
+        float4* red_w = red_u + RG * CG;
+        const int u = (int)blockIdx.x + n * grid;  // = b * Hv + h = gh for a single token
+
+        // Everything this unit needs from its stage goes to registers before
+        // the barrier.  The reads happen whether or not this thread saw the
+        // copy land, so warp 0's shuffles never diverge; a unit that did not
+        // land is abandoned at the barrier, its values unused.
+        float4 s[RPT];
+        float kr[RPT];
+        float4 vr = make_float4(0.f, 0.f, 0.f, 0.f);
+        float al = 0.f, be = 0.f;
+        if (m.y) {
+            float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const int i = r * RG + rg;
+                s[r] = tile[i * CG + cg];
+                kr[r] = smem_in<InT>(ksm, i);
+                fma4(pu, s[r], kr[r]);
+                fma4(pw, s[r], smem_in<InT>(qsm, i));
+            }
+            red_u[rg * CG + cg] = pu;
+            red_w[rg * CG + cg] = pw;
+            vr = make_float4(smem_in<InT>(vsm, cg * 4 + 0), smem_in<InT>(vsm, cg * 4 + 1),
+                             smem_in<InT>(vsm, cg * 4 + 2), smem_in<InT>(vsm, cg * 4 + 3));
+            al = reinterpret_cast<const float*>(st + P::A_OFF)[u & 3];
+            be = reinterpret_cast<const float*>(st + P::B_OFF)[u & 3];
+            if (tid < 32) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = tid; i < P::DK; i += 32) acc = fmaf(smem_in<InT>(ksm, i), smem_in<InT>(qsm, i), acc);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                if (tid == 0) kq_s[n & 1] = acc;
+            }
+        }
+        if (__syncthreads_or(landed ? 0 : 1)) {
+            // A copy never completed: report, let thread 0 wait (bounded) for
+            // the copies it has issued so none lands in freed shared memory.
+            if (tid == 0) {
+                record_error(a.err, GDN_ERR_TIMEOUT);
+                for (int j = n; j < p_next; ++j)
+                    if (!mbar_wait_bounded(&bars[j % STAGES], (uint32_t)(j / STAGES) & 1u)) break;
+            }
+            return;
+        }
+        // The stage is consumed: refill it with the unit STAGES ahead.
+        if (tid == 0 && p_next < n_local) issue();
+
+        if (m.y) {
+            float4 uu = red_u[cg];
+            float4 ww = red_w[cg];
+#pragma unroll
+            for (int r = 1; r < RG; ++r) {
+                add4(uu, red_u[r * CG + cg]);
+                add4(ww, red_w[r * CG + cg]);
+            }
+            float4 c;
+            c.x = be * (vr.x - al * uu.x);
+            c.y = be * (vr.y - al * uu.y);
+            c.z = be * (vr.z - al * uu.z);
+            c.w = be * (vr.w - al * uu.w);
+            if (rg == 0) {
+                const float kq = kq_s[n & 1];
+                float4 o;
+                o.x = fmaf(c.x, kq, al * ww.x);
+                o.y = fmaf(c.y, kq, al * ww.y);
+                o.z = fmaf(c.z, kq, al * ww.z);
+                o.w = fmaf(c.w, kq, al * ww.w);
+                __stcs(reinterpret_cast<float4*>(a.out + (size_t)u * P::DV) + cg, o);
+            }
+            const int h = u % a.Hv;
+            float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)m.x * a.Hv + h) * (P::DK * P::DV));
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                s[r].x = fmaf(kr[r], c.x, al * s[r].x);
+                s[r].y = fmaf(kr[r], c.y, al * s[r].y);
+                s[r].z = fmaf(kr[r], c.z, al * s[r].z);
+                s[r].w = fmaf(kr[r], c.w, al * s[r].w);
+                __stcs(D + (size_t)(r * RG + rg) * CG + cg, s[r]);
+            }
+        } else if (tid == 0) {
+            record_error(a.err, GDN_ERR_INDEX);
+        }
+        // No second barrier: the next unit writes the other reduction buffer,
+        // and this one is rewritten only after every thread has passed the
+        // next unit's barrier, i.e. has finished reading it here.
+    }
+}
+
 __global__ void gdn_commit_kernel(const int32_t* __restrict__ accept_len, int32_t* __restrict__ committed,
                                   const int32_t* __restrict__ cur, int B, int T, int num_slots, int32_t* err) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -278,8 +686,30 @@ __global__ void gdn_commit_kernel(const int32_t* __restrict__ accept_len, int32_
 
 constexpr int kMaxDk = 4096;
 
+// Column-block width of the single-token tile kernel (value columns per CTA)
+// and its per-thread register budget, which sets how many CTAs stay resident
+// per SM.  Compile-time tunables; the defaults are the measured best on B200.
+#ifndef GDN_TILE1_COLS
+#define GDN_TILE1_COLS 64
+#endif
+#ifndef GDN_TILE1_MAXREG
+#define GDN_TILE1_MAXREG 100
+#endif
+constexpr int kTile1Cols = GDN_TILE1_COLS;
+
 template <int DK, int DV, int NT>
 gdn_status launch_tile(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
+    if (a.T == 1) {
+        constexpr int DVC = DV < kTile1Cols ? DV : kTile1Cols;
+        constexpr int NT1 = (DVC / 4) * 8;               // 8 row groups
+        constexpr int MINB = (65536 / (NT1 * GDN_TILE1_MAXREG)) < 16 ? (65536 / (NT1 * GDN_TILE1_MAXREG)) : 16;
+        const dim3 grid((unsigned)(a.B * a.Hv * (DV / DVC)));
+        if (dtype == GDN_BF16)
+            gdn_tile1_kernel<DK, DV, DVC, NT1, MINB, __nv_bfloat16><<<grid, NT1, 0, stream>>>(a);
+        else
+            gdn_tile1_kernel<DK, DV, DVC, NT1, MINB, float><<<grid, NT1, 0, stream>>>(a);
+        return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
     const dim3 grid((unsigned)(a.B * a.Hv));
     if (dtype == GDN_BF16)
         gdn_tile_kernel<DK, DV, NT, __nv_bfloat16><<<grid, NT, 0, stream>>>(a);
@@ -302,26 +732,105 @@ gdn_status launch_column(const StepArgs& a, int32_t dtype, cudaStream_t stream) 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr int kMaxDevices = 64;
+
+int sm_count() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev < kMaxDevices) cache[dev] = n;
+    return n;
+}
+
+template <int NT, typename InT>
+gdn_status launch_stream(const StepArgs& a, cudaStream_t stream) {
+    using P = StreamPlan<NT, InT>;
+    const int sms = sm_count();
+    if (sms <= 0) return GDN_ERR_CUDA;
+    // The opt-in above 48 KiB is a per-function attribute: setting it on every
+    // launch keeps the library free of device-state caches and costs ~1 us.
+    if (cudaFuncSetAttribute(gdn_stream_kernel<NT, InT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)P::SMEM_BYTES) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int units = a.B * a.Hv;
+    const int grid = units < sms ? units : sms;
+    gdn_stream_kernel<NT, InT><<<grid, NT, P::SMEM_BYTES, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// Which kernel serves a call: the streaming kernel needs one token, 128 x 128
+// tiles, 16-byte aligned buffers (bulk copies) and B * Hv a multiple of 4 (the
+// 16-byte gate chunks stay inside alpha/beta); the register-tile kernel needs
+// a compiled tile shape and 16-byte aligned pool/out; the column kernel takes
+// anything.
+bool stream_ok(const StepArgs& a) {
+    return a.T == 1 && a.dk == 128 && a.dv == 128 && ((int64_t)a.B * a.Hv) % 4 == 0 && aligned16(a.pool) &&
+           aligned16(a.out) && aligned16(a.q) && aligned16(a.k) && aligned16(a.v) && aligned16(a.alpha) &&
+           aligned16(a.beta);
+}
+
+bool tile_ok(const StepArgs& a) {
+    return ((a.dk == 128 && a.dv == 128) || (a.dk == 64 && a.dv == 64)) && aligned16(a.pool) && aligned16(a.out);
+}
+
+gdn_status launch(const StepArgs& a, int32_t dtype, int32_t variant, cudaStream_t stream) {
+    const bool bf = dtype == GDN_BF16;
+    if (variant == GDN_VARIANT_AUTO) {
+        // Measured on B200 (large decode, 8192 tiles per call): register tiles
+        // 164.8 us per call, bulk-copy pipeline 184.4 us, so the register-tile
+        // family serves every shape it supports.
+        if (tile_ok(a))
+            variant = GDN_VARIANT_TILE;
+        else if (stream_ok(a))
+            variant = GDN_VARIANT_STREAM;
+        else
+            variant = GDN_VARIANT_COLUMN;
+    }
+    switch (variant) {
+        case GDN_VARIANT_STREAM:
+            if (!stream_ok(a)) return GDN_ERR_INVALID_ARG;
+            return bf ? launch_stream<256, __nv_bfloat16>(a, stream) : launch_stream<256, float>(a, stream);
+        case GDN_VARIANT_TILE:
+            if (!tile_ok(a)) return GDN_ERR_INVALID_ARG;
+            return a.dk == 128 ? launch_tile<128, 128, 256>(a, dtype, stream) : launch_tile<64, 64, 128>(a, dtype, stream);
+        case GDN_VARIANT_COLUMN:
+            return launch_column(a, dtype, stream);
+        default:
+            return GDN_ERR_INVALID_ARG;
+    }
+}
+
 }  // namespace
+
+extern "C" gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t* src_idx,
+                                              const int32_t* dst_idx, const void* q, const void* k, const void* v,
+                                              const float* alpha, const float* beta, float* out, int32_t B,
+                                              int32_t T, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                                              int32_t qkv_dtype, int32_t* err_word, int32_t variant,
+                                              cudaStream_t stream) {
+    if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return GDN_ERR_INVALID_ARG;
+    if (Hv % Hk != 0 || dk > kMaxDk) return GDN_ERR_INVALID_ARG;
+    if (qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (variant < GDN_VARIANT_AUTO || variant > GDN_VARIANT_COLUMN) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)B * Hv * 4 >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;  // grid: up to 4 CTAs per (b, h)
+    if (B == 0) return GDN_OK;
+    if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out) return GDN_ERR_INVALID_ARG;
+
+    const StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word,
+                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk};
+    return launch(a, qkv_dtype, variant, stream);
+}
 
 extern "C" gdn_status gdn_decode_step(float* pool, int32_t num_slots, const int32_t* src_idx,
                                       const int32_t* dst_idx, const void* q, const void* k, const void* v,
                                       const float* alpha, const float* beta, float* out, int32_t B, int32_t T,
                                       int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int32_t qkv_dtype,
                                       int32_t* err_word, cudaStream_t stream) {
-    if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return GDN_ERR_INVALID_ARG;
-    if (Hv % Hk != 0 || dk > kMaxDk) return GDN_ERR_INVALID_ARG;
-    if (qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
-    if ((int64_t)B * Hv >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
-    if (B == 0) return GDN_OK;
-    if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out) return GDN_ERR_INVALID_ARG;
-
-    StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word,
-               num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk};
-    const bool vec_ok = aligned16(pool) && aligned16(out);
-    if (dk == 128 && dv == 128 && vec_ok) return launch_tile<128, 128, 256>(a, qkv_dtype, stream);
-    if (dk == 64 && dv == 64 && vec_ok) return launch_tile<64, 64, 128>(a, qkv_dtype, stream);
-    return launch_column(a, qkv_dtype, stream);
+    return gdn_decode_step_variant(pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, out, B, T, Hk, Hv, dk,
+                                   dv, qkv_dtype, err_word, GDN_VARIANT_AUTO, stream);
 }
 
 extern "C" gdn_status gdn_commit(const int32_t* accept_len, int32_t* committed, const int32_t* cur, int32_t B,

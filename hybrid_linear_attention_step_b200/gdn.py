@@ -24,6 +24,13 @@ GDN_ERR_TIMEOUT = 4
 GDN_F32 = 0
 GDN_BF16 = 1
 
+GDN_VARIANT_AUTO = 0
+GDN_VARIANT_STREAM = 1
+GDN_VARIANT_TILE = 2
+GDN_VARIANT_COLUMN = 3
+VARIANTS = {"auto": GDN_VARIANT_AUTO, "stream": GDN_VARIANT_STREAM, "tile": GDN_VARIANT_TILE,
+            "column": GDN_VARIANT_COLUMN}
+
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
 
 _lib = None
@@ -48,6 +55,9 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_decode_step.restype = i32
     lib.gdn_decode_step.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                     i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    lib.gdn_decode_step_variant.restype = i32
+    lib.gdn_decode_step_variant.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     lib.gdn_commit.restype = i32
     lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
     lib.gdn_get_error.restype = i32
@@ -82,6 +92,21 @@ def _ptr_or_null(t: Optional[torch.Tensor], name: str) -> Optional[int]:
     return None if t is None else _dev(t, name, torch.int32)
 
 
+def _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out):
+    if pool.dim() != 4 or q.dim() != 4 or v.dim() != 4:
+        raise ValueError("pool, q, k, v must be 4-D")
+    num_slots, Hv, dk, dv = pool.shape
+    B, T, Hk = q.shape[0], q.shape[1], q.shape[2]
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype: bfloat16 or float32")
+    return (_dev(pool, "pool", torch.float32), int(num_slots),
+            _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32),
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+            _dev(alpha, "alpha", torch.float32), _dev(beta, "beta", torch.float32),
+            _dev(out, "out", torch.float32),
+            int(B), int(T), int(Hk), int(Hv), int(dk), int(dv), _DTYPES[q.dtype])
+
+
 def gdn_decode_step(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
                     q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
@@ -92,22 +117,26 @@ def gdn_decode_step(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Te
     q, k [B, T, Hk, dk] and v [B, T, Hv, dv] bf16 or fp32; alpha, beta [B, T, Hv] fp32;
     out [B, T, Hv, dv] fp32.  Returns the status; raises GdnError on failure when ``check``.
     """
-    if pool.dim() != 4 or q.dim() != 4 or v.dim() != 4:
-        raise ValueError("pool, q, k, v must be 4-D")
-    num_slots, Hv, dk, dv = pool.shape
-    B, T, Hk = q.shape[0], q.shape[1], q.shape[2]
-    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
-        raise TypeError("q, k, v must share one dtype: bfloat16 or float32")
-    status = load_library().gdn_decode_step(
-        _dev(pool, "pool", torch.float32), int(num_slots),
-        _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32),
-        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
-        _dev(alpha, "alpha", torch.float32), _dev(beta, "beta", torch.float32),
-        _dev(out, "out", torch.float32),
-        int(B), int(T), int(Hk), int(Hv), int(dk), int(dv), _DTYPES[q.dtype],
-        _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+    status = load_library().gdn_decode_step(*args, _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_decode_step")
+    return status
+
+
+def gdn_decode_step_variant(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
+                            q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor, variant,
+                            err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """gdn_decode_step with an explicit kernel: ``variant`` is a GDN_VARIANT_* value or a name
+    ("auto", "stream", "tile", "column")."""
+    if isinstance(variant, str):
+        variant = VARIANTS[variant]
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+    status = load_library().gdn_decode_step_variant(*args, _ptr_or_null(err_word, "err_word"), int(variant),
+                                                    _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_decode_step_variant")
     return status
 
 

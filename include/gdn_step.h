@@ -68,6 +68,18 @@ typedef enum gdn_status {
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
+/* Kernel choice for gdn_decode_step_variant. */
+typedef enum gdn_variant {
+    GDN_VARIANT_AUTO = 0,   /* what gdn_decode_step uses: the first of TILE, STREAM, COLUMN that applies */
+    GDN_VARIANT_STREAM = 1, /* persistent bulk-copy pipeline through shared memory: T == 1,
+                               dk == dv == 128, every buffer 16-byte aligned, B*Hv % 4 == 0 */
+    GDN_VARIANT_TILE = 2,   /* state tile held in registers: (dk, dv) in {(128, 128), (64, 64)},
+                               pool and out 16-byte aligned, any T (T == 1: one CTA per 64-column
+                               block of a (request, head) tile; T > 1: one CTA per tile, carried
+                               across the tokens) */
+    GDN_VARIANT_COLUMN = 3  /* one thread per value column: any shape and alignment */
+} gdn_variant;
+
 /*
  * gdn_decode_step -- one GDN layer's decode update for B requests and T tokens each.
  *
@@ -109,6 +121,22 @@ gdn_status gdn_decode_step(float* pool, int32_t num_slots, const int32_t* src_id
                            const float* alpha, const float* beta, float* out, int32_t B, int32_t T,
                            int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int32_t qkv_dtype,
                            int32_t* err_word, cudaStream_t stream);
+
+/*
+ * gdn_decode_step_variant -- gdn_decode_step with an explicit kernel choice.
+ *
+ * Same operation, arguments, preconditions and errors as gdn_decode_step, plus
+ * `variant` (a gdn_variant).  All variants compute the same update; they differ
+ * in how work maps onto the GPU and may differ in floating-point rounding order
+ * (never in which slots are written).  A variant whose conditions (listed with
+ * gdn_variant) the call does not meet returns GDN_ERR_INVALID_ARG before any
+ * launch.  Meant for tests and measurements that pin one kernel.
+ */
+gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t* src_idx,
+                                   const int32_t* dst_idx, const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta, float* out, int32_t B, int32_t T,
+                                   int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int32_t qkv_dtype,
+                                   int32_t* err_word, int32_t variant, cudaStream_t stream);
 
 /*
  * gdn_commit -- accept speculative draft tokens by rewriting an int32 index table.

@@ -47,16 +47,22 @@ def step_to_device(s: wl.Step, device="cuda"):
                 src=to_torch(s.src_idx, device), dst=to_torch(np.ascontiguousarray(s.dst_idx.reshape(s.B, s.T)), device))
 
 
-def run_gpu(pool_dev, s: wl.Step, out_fill=-7.0, err=None, stream=None):
-    """Runs one CUDA decode call on ``pool_dev`` (updated in place); returns out (host)."""
+def run_gpu(pool_dev, s: wl.Step, out_fill=-7.0, err=None, stream=None, variant=None):
+    """Runs one CUDA decode call on ``pool_dev`` (updated in place); returns out (host).
+
+    ``variant`` None goes through gdn_decode_step; a name pins one kernel through
+    gdn_decode_step_variant."""
     import torch
 
     from hybrid_linear_attention_step_b200 import gdn
 
     x = step_to_device(s, pool_dev.device)
     out = torch.full((s.B, s.T, s.Hv, s.dv), out_fill, dtype=torch.float32, device=pool_dev.device)
-    gdn.gdn_decode_step(pool_dev, x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], out,
-                        err_word=err, stream=stream)
+    args = (pool_dev, x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+    if variant is None:
+        gdn.gdn_decode_step(*args, err_word=err, stream=stream)
+    else:
+        gdn.gdn_decode_step_variant(*args, variant, err_word=err, stream=stream)
     torch.cuda.synchronize()
     return out.cpu().numpy()
 

@@ -50,12 +50,13 @@ def test_tiny_chain_matches_oracle_and_golden(torch_cuda):
     assert rel_err(dev.cpu().numpy(), g_pool) <= TOL_STATE
 
 
+@pytest.mark.parametrize("variant", [None, "stream", "tile", "column"])
 @pytest.mark.parametrize("name", ["decode_b16", "prefix_cow"])
-def test_decode_workloads(torch_cuda, name):
+def test_decode_workloads(torch_cuda, name, variant):
     w = wl.WORKLOADS[name]()
     s = w.steps[0]
     dev = to_torch(w.pool)
-    out = run_gpu(dev, s)
+    out = run_gpu(dev, s, variant=variant)
     ref_pool, ref_out, skipped = run_oracle(w.pool, s)
     assert skipped == 0
     got = dev.cpu().numpy()
@@ -66,14 +67,15 @@ def test_decode_workloads(torch_cuda, name):
     assert np.array_equal(got[src_only].view(np.uint32), w.pool[src_only].view(np.uint32))
 
 
-def test_speculative_and_commit(torch_cuda):
+@pytest.mark.parametrize("variant", [None, "column"])
+def test_speculative_and_commit(torch_cuda, variant):
     torch = torch_cuda
     from hybrid_linear_attention_step_b200 import gdn
 
     w = wl.speculative()
     s = w.steps[0]
     dev = to_torch(w.pool)
-    out = run_gpu(dev, s)
+    out = run_gpu(dev, s, variant=variant)
     ref_pool, ref_out, _ = run_oracle(w.pool, s)
     got = dev.cpu().numpy()
     check_pool(got, ref_pool, w.pool, s.dst_idx)
@@ -166,17 +168,19 @@ def test_empty_batch_is_a_no_op(torch_cuda):
     assert bool((pool == 1).all())
 
 
-@pytest.mark.parametrize("dk,dv", [(128, 128), (20, 24)])
-def test_out_of_range_indices_skip_and_report(torch_cuda, dk, dv):
+@pytest.mark.parametrize("dk,dv,T", [(128, 128, 2), (20, 24, 2), (128, 128, 1)])
+def test_out_of_range_indices_skip_and_report(torch_cuda, dk, dv, T):
     torch = torch_cuda
     from hybrid_linear_attention_step_b200 import gdn
 
     rng = np.random.default_rng(50)
-    num_slots, B, T = 12, 4, 2
+    num_slots, B = 12, 4
     pool = wl.init_pool(rng, num_slots, 2, dk, dv)
     q, k, v, a, b = wl.random_step_inputs(rng, B, T, 1, 2, dk, dv, wl.BF16)
     src = np.array([0, num_slots, 2, -1], np.int32)
-    dst = np.array([[4, 5], [6, 7], [8, 99], [10, 11]], np.int32)
+    dst = np.array([[4, 5], [6, 7], [8, 99], [10, 11]], np.int32)[:, :T].copy()
+    if T == 1:
+        dst[2, 0] = 99
     s = wl.Step(q, k, v, a, b, src, dst)
     dev = to_torch(pool)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -190,6 +194,7 @@ def test_out_of_range_indices_skip_and_report(torch_cuda, dk, dv):
     assert np.all(out[1:] == -7.0)
     assert rel_err(out[:1], ref_out[:1]) <= TOL_OUT_BF16
 
+    T = 2
     accept = torch.tensor([1, -1, T + 1, 2], dtype=torch.int32, device="cuda")
     cur = torch.tensor([[4, 5], [6, 7], [8, 9], [10, num_slots + 4]], dtype=torch.int32, device="cuda")
     committed = torch.tensor([0, 1, 2, 3], dtype=torch.int32, device="cuda")
@@ -241,3 +246,38 @@ def test_invalid_arguments_raise(torch_cuda):
     assert ei.value.status == gdn.GDN_ERR_INVALID_ARG
     with pytest.raises(TypeError):
         gdn.gdn_decode_step(pool, x["src"], x["dst"], x["q"], x["k"], x["v"].float(), x["alpha"], x["beta"], out)
+
+
+def test_variant_conditions_are_checked(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    w = wl.speculative()
+    s = w.steps[0]
+    x = step_to_device(s)
+    pool = to_torch(w.pool)
+    out = torch.zeros((s.B, s.T, s.Hv, s.dv), device="cuda")
+    args = (pool, x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+    for bad in ("stream", 9):  # the streaming kernel serves single-token calls only; 9 is no variant
+        with pytest.raises(gdn.GdnError) as ei:
+            gdn.gdn_decode_step_variant(*args, bad)
+        assert ei.value.status == gdn.GDN_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert np.array_equal(pool.cpu().numpy(), w.pool)  # nothing ran
+
+
+@pytest.mark.parametrize("B", [1, 3, 37, 300])
+def test_stream_kernel_partial_waves(torch_cuda, B):
+    """Unit counts below, at and above one unit per SM, and not a multiple of the grid."""
+    rng = np.random.default_rng(60 + B)
+    Hk, Hv = 2, 4
+    num_slots = 2 * B + 5
+    pool = wl.init_pool(rng, num_slots, Hv, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, 1, Hk, Hv, 128, 128, wl.BF16)
+    perm = rng.permutation(num_slots).astype(np.int32)
+    s = wl.Step(q, k, v, a, b, perm[:B].copy(), perm[B:2 * B].reshape(B, 1).copy())
+    dev = to_torch(pool)
+    out = run_gpu(dev, s, variant="stream")
+    ref_pool, ref_out, _ = run_oracle(pool, s)
+    check_pool(dev.cpu().numpy(), ref_pool, pool, s.dst_idx)
+    assert rel_err(out, ref_out) <= TOL_OUT_BF16
