@@ -44,14 +44,15 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).  See profiles/.
-NCU_TRAFFIC = {"kernel": "gdn_tile_kernel<128,128,256,bf16>",
-               "source_sha256": "0601db0eb8524fa0b331ef6c8f4e6583bcfbaff0676f759b9efbe997185a500e",
-               "bytes_per_launch": 541150720 + 483911936,
-               "profile": "profiles/gdn_tile_kernel_large_decode.md"}
+NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
+               "source_sha256": "4839168da5fe371a7512349ae486f777fb52b16b0fd84890dd76a88eed4244a9",
+               "bytes_per_launch": 541148928 + 483413504,
+               "profile": "profiles/gdn_tile1_kernel_large_decode.md"}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
-KERNEL_NAMES = {"auto": "gdn_tile1_kernel<128,128,64,128,5,bf16>", "tile": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
+KERNEL_NAMES = {"auto": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
+                "tile": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
                 "stream": "gdn_stream_kernel<256,bf16>", "column": "gdn_column_kernel<bf16>"}
 
 
@@ -402,6 +403,125 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------- other workloads
+
+def workload_bytes(w, s) -> dict:
+    """Algorithmic bytes of one call of a host workload: nominal (every unit reads
+    its own source tile) and minimum (each distinct source tile read once)."""
+    G = s.Hv // s.Hk
+    in_bytes = 2 if s.dtype == "bf16" else 4
+    per_req_tok = s.Hv * (2.0 * s.dk * in_bytes / G + s.dv * in_bytes + 8.0 + 4.0 * s.dv)
+    tile = 4.0 * s.dk * s.dv
+    writes = s.B * s.T * s.Hv * tile
+    nominal = s.B * s.Hv * tile + writes + s.B * s.T * per_req_tok
+    distinct = len(set(int(x) for x in s.src_idx if x >= 0))
+    minimum = distinct * s.Hv * tile + writes + s.B * s.T * per_req_tok
+    return {"nominal": nominal, "minimum": minimum, "units": s.B * s.T * s.Hv}
+
+
+def run_workload(args):
+    """Times one of the smaller workloads (decode_b16, prefix_cow, speculative):
+    ``--steps`` decode calls, back to back (warm L2) and, separately, each call
+    after an L2-flushing write (cold), optionally replayed from a CUDA graph."""
+    import numpy as np
+    import torch
+
+    from hybrid_linear_attention_step_b200 import gdn, workloads as wl
+
+    torch.cuda.set_device(0)
+    w = wl.WORKLOADS[args.workload]()
+    s = w.steps[0]
+    to_dev = lambda a: (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+                        if a.dtype == np.uint16 else torch.from_numpy(np.ascontiguousarray(a)).cuda())
+    pool = torch.from_numpy(w.pool).cuda()
+    x = {k_: to_dev(getattr(s, k_)) for k_ in ("q", "k", "v", "alpha", "beta", "src_idx")}
+    dst = to_dev(np.ascontiguousarray(s.dst_idx.reshape(s.B, s.T)))
+    out = torch.zeros((s.B, s.T, s.Hv, s.dv), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def call():
+        args_ = (pool, x["src_idx"], dst, x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+        if args.variant == "auto":
+            gdn.gdn_decode_step(*args_, err_word=err)
+        else:
+            gdn.gdn_decode_step_variant(*args_, args.variant, err_word=err)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    if args.graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            call()  # one eager call on the capture stream before capturing
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(K):
+                call()
+        graph.replay()
+        torch.cuda.synchronize()
+    ev0.record(stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        for _ in range(K):
+            call()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    warm_us = 1e3 * ev0.elapsed_time(ev1) / K
+
+    # cold: an L2-sized write before every call, the call alone bracketed by events
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    cold = []
+    for _ in range(min(K, 50)):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cold.append(1e3 * e0.elapsed_time(e1))
+    cold_us = statistics.median(cold)
+    code = gdn.gdn_get_error(err)
+    if code != 0:
+        raise RuntimeError(f"device error word set: {gdn.status_string(code)}")
+
+    commit_us = None
+    if s.accept_len is not None:
+        committed = x["src_idx"].clone()
+        acc = to_dev(s.accept_len)
+        for _ in range(3):
+            gdn.gdn_commit(acc, committed, dst, w.num_slots)
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(100):
+            gdn.gdn_commit(acc, committed, dst, w.num_slots)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        commit_us = 1e3 * c0.elapsed_time(c1) / 100
+
+    hbm_peak, peak_kind = peaks()
+    nb = workload_bytes(w, s)
+    line = {
+        "metric": METRIC, "workload": args.workload, "unit": UNIT, "variant": args.variant,
+        "graph": bool(args.graph), "steps": K, "warmup": args.warmup,
+        "value": nb["units"] / (warm_us / 1e6), "us_per_call_warm": warm_us, "us_per_call_cold": cold_us,
+        "bytes_per_call_nominal": nb["nominal"], "bytes_per_call_min": nb["minimum"],
+        "gbs_warm_nominal": nb["nominal"] / warm_us / 1e3, "gbs_cold_nominal": nb["nominal"] / cold_us / 1e3,
+        "gbs_cold_min": nb["minimum"] / cold_us / 1e3, "peak_gbs": hbm_peak, "peak_kind": peak_kind,
+        "commit_us": commit_us,
+        "config": {"B": s.B, "T": s.T, "Hk": s.Hk, "Hv": s.Hv, "dk": s.dk, "dv": s.dv, "slots": w.num_slots,
+                   "dtype": s.dtype},
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def run_ours(args):
@@ -531,6 +651,10 @@ def main():
     ap.add_argument("--batch", type=int, default=256)
     ap.add_argument("--variant", choices=["auto", "stream", "tile", "column"], default="auto",
                     help="kernel for the decode calls (auto = what gdn_decode_step picks)")
+    ap.add_argument("--workload", choices=["large", "decode_b16", "prefix_cow", "speculative"], default="large",
+                    help="large = the headline 8-layer decode; the others time one call of that workload")
+    ap.add_argument("--graph", action="store_true", help="replay the timed calls from a CUDA graph "
+                    "(smaller workloads only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -538,6 +662,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != "large":
+        run_workload(args)
     else:
         run_ours(args)
 

@@ -61,16 +61,26 @@ __device__ __forceinline__ float load_in<__nv_bfloat16>(const void* base, size_t
     return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(base) + idx));
 }
 
-// True when src and all T destination slots of request b are inside the pool.
-// Every thread of a block evaluates the same indices, so the result is uniform.
-__device__ __forceinline__ bool request_in_range(const StepArgs& a, int b, int& src) {
+// Request status: kRun when src and all T destination slots of request b lie
+// inside the pool; kPad when src is the padding sentinel GDN_SLOT_NONE (the
+// request is skipped silently, its destinations are not looked at); kBad
+// otherwise (skipped and reported).  Every thread of a block evaluates the
+// same indices, so the result is uniform across the block.
+enum RequestStatus { kRun = 0, kPad = 1, kBad = 2 };
+
+// All index loads are issued before any branch on their values, so a CTA
+// pays one load latency here, not one per index.
+__device__ __forceinline__ int request_status(const StepArgs& a, int b, int T, int& src, int& dst0) {
     src = __ldg(a.src_idx + b);
-    bool ok = src >= 0 && src < a.num_slots;
-    for (int t = 0; t < a.T; ++t) {
-        const int d = __ldg(a.dst_idx + (size_t)b * a.T + t);
-        ok = ok && d >= 0 && d < a.num_slots;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+        const int d = __ldg(a.dst_idx + (size_t)b * T + t);
+        if (t == 0) dst0 = d;
+        ok &= (d >= 0) & (d < a.num_slots);
     }
-    return ok;
+    if (src == GDN_SLOT_NONE) return kPad;
+    ok &= (src >= 0) & (src < a.num_slots);
+    return ok ? kRun : kBad;
 }
 
 __device__ __forceinline__ void fma4(float4& acc, const float4& m, float x) {
@@ -78,6 +88,13 @@ __device__ __forceinline__ void fma4(float4& acc, const float4& m, float x) {
     acc.y = fmaf(m.y, x, acc.y);
     acc.z = fmaf(m.z, x, acc.z);
     acc.w = fmaf(m.w, x, acc.w);
+}
+
+__device__ __forceinline__ void add4_rn(float4& acc, const float4& x) {
+    acc.x = __fadd_rn(acc.x, x.x);
+    acc.y = __fadd_rn(acc.y, x.y);
+    acc.z = __fadd_rn(acc.z, x.z);
+    acc.w = __fadd_rn(acc.w, x.w);
 }
 
 __device__ __forceinline__ void add4(float4& acc, const float4& x) {
@@ -88,125 +105,13 @@ __device__ __forceinline__ void add4(float4& acc, const float4& x) {
 }
 
 // ---------------------------------------------------------------------------
-// Register-tile kernel for fixed (DK, DV).  One CTA owns one (b, h) state tile
-// and keeps it in registers across all T tokens.  Thread layout: CG = DV/4
-// column groups (one float4 each) x RG = NT/CG row groups; thread (rg, cg)
-// holds rows i = m*RG + rg, m < DK/RG, so each warp-wide load instruction
-// reads whole 512-byte rows and the CTA sweeps the 64 KiB tile front to back.
-// Reductions over i: in-thread over its rows, then across row groups through
-// shared memory.  The tile is read once from HBM and written once per token.
-// ---------------------------------------------------------------------------
-template <int DK, int DV, int NT, typename InT>
-__global__ void __launch_bounds__(NT, 2) gdn_tile_kernel(StepArgs a) {
-    constexpr int CG = DV / 4;
-    static_assert(DV % 4 == 0 && NT % CG == 0, "tile shape");
-    constexpr int RG = NT / CG;
-    static_assert(DK % RG == 0, "tile shape");
-    constexpr int RPT = DK / RG;
-
-    __shared__ float ks[DK];
-    __shared__ float qs[DK];
-    __shared__ float4 red_u[RG][CG];
-    __shared__ float4 red_w[RG][CG];
-    __shared__ float kq_s;
-
-    const int tid = threadIdx.x;
-    const int cg = tid % CG;
-    const int rg = tid / CG;
-    const int h = blockIdx.x % a.Hv;
-    const int b = blockIdx.x / a.Hv;
-    const int hk = h / a.G;
-
-    int src;
-    if (!request_in_range(a, b, src)) {
-        if (tid == 0) record_error(a.err, GDN_ERR_INDEX);
-        return;
-    }
-
-    const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV));
-    float4 s[RPT];
-#pragma unroll
-    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + (size_t)(m * RG + rg) * CG + cg);
-
-    for (int t = 0; t < a.T; ++t) {
-        const size_t tok = (size_t)b * a.T + t;
-        if (t > 0) __syncthreads();  // the previous token is done with ks/qs/red
-        const size_t kbase = (tok * a.Hk + hk) * DK;
-        for (int i = tid; i < DK; i += NT) {
-            ks[i] = load_in<InT>(a.k, kbase + i);
-            qs[i] = load_in<InT>(a.q, kbase + i);
-        }
-        __syncthreads();
-
-        float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int m = 0; m < RPT; ++m) {
-            const int i = m * RG + rg;
-            fma4(pu, s[m], ks[i]);
-            fma4(pw, s[m], qs[i]);
-        }
-        red_u[rg][cg] = pu;
-        red_w[rg][cg] = pw;
-        if (tid < 32) {
-            float acc = 0.f;
-            for (int i = tid; i < DK; i += 32) acc = fmaf(ks[i], qs[i], acc);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (tid == 0) kq_s = acc;
-        }
-        __syncthreads();
-
-        float4 u = red_u[0][cg];
-        float4 w = red_w[0][cg];
-#pragma unroll
-        for (int r = 1; r < RG; ++r) {
-            add4(u, red_u[r][cg]);
-            add4(w, red_w[r][cg]);
-        }
-        const size_t gh = tok * a.Hv + h;
-        const float al = __ldg(a.alpha + gh);
-        const float be = __ldg(a.beta + gh);
-        const size_t vb = gh * DV + (size_t)cg * 4;
-        float4 c;
-        c.x = be * (load_in<InT>(a.v, vb + 0) - al * u.x);
-        c.y = be * (load_in<InT>(a.v, vb + 1) - al * u.y);
-        c.z = be * (load_in<InT>(a.v, vb + 2) - al * u.z);
-        c.w = be * (load_in<InT>(a.v, vb + 3) - al * u.w);
-        if (rg == 0) {
-            const float kq = kq_s;
-            float4 o;
-            o.x = fmaf(c.x, kq, al * w.x);
-            o.y = fmaf(c.y, kq, al * w.y);
-            o.z = fmaf(c.z, kq, al * w.z);
-            o.w = fmaf(c.w, kq, al * w.w);
-            __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + cg, o);
-        }
-
-        const int dst = __ldg(a.dst_idx + tok);
-        float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst * a.Hv + h) * (DK * DV));
-#pragma unroll
-        for (int m = 0; m < RPT; ++m) {
-            const float ki = ks[m * RG + rg];
-            s[m].x = fmaf(ki, c.x, al * s[m].x);
-            s[m].y = fmaf(ki, c.y, al * s[m].y);
-            s[m].z = fmaf(ki, c.z, al * s[m].z);
-            s[m].w = fmaf(ki, c.w, al * s[m].w);
-            __stcs(D + (size_t)(m * RG + rg) * CG + cg, s[m]);
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Single-token register-tile kernel.  Value columns are independent, so a
-// (b, h) tile is split into DV / DVC column blocks, one CTA each (a column
-// block's rows are DVC * 4 contiguous bytes, read and written as float4 runs).
-// Thread layout per CTA: CG = DVC / 4 column groups x RG = NT / CG row groups,
-// rows i = m * RG + rg.  Every input the CTA needs (tile block, k and q rows,
-// its v columns, the gates, the slot indices) is requested at kernel start, so
-// after the tile lands the only waits are two barriers; shared memory stays
-// small, leaving the unified L1 large enough to track the outstanding misses
-// of the MINB CTAs resident per SM.
+// Single-token form of the register-tile kernel below (same thread layout, same
+// per-token arithmetic in the same order, hence identical bits), written out
+// on its own: with 5 CTAs per SM the budget is 96 registers, and the general
+// form's token bookkeeping tips the single-token case into spills.  The slot
+// indices are loaded together and branched on once; the destination slot, v
+// and the gates are staged in shared memory so that no register holds them
+// while the tile is in flight.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, int DVC, int NT, int MINB, typename InT>
 __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
@@ -236,13 +141,13 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
 
     const int src = __ldg(a.src_idx + b);
     const int dst = __ldg(a.dst_idx + b);
+    if (src == GDN_SLOT_NONE) return;
     if (src < 0 || src >= a.num_slots || dst < 0 || dst >= a.num_slots) {
         if (tid == 0) record_error(a.err, GDN_ERR_INDEX);
         return;
     }
 
-    // float4 offset of (row i, this thread's columns) inside a tile: i * DV / 4 + chunk * CG + cg;
-    // the thread's rows are rg + m * RG, so its base is row rg and the step is RG rows.
+    // float4 offset of (row i, this thread's columns) in a tile: i * DV / 4 + chunk * CG + cg.
     const int col4 = chunk * CG + cg;
     const int toff = rg * (DV / 4) + col4;
     constexpr int kRowStep = RG * (DV / 4);
@@ -257,13 +162,11 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
         ks[i] = load_in<InT>(a.k, kbase + i);
         qs[i] = load_in<InT>(a.q, kbase + i);
     }
-    // v and the gates go through shared memory too: staged now, read after
-    // the reduction, they cost no registers while the tile is in flight.
     for (int j = tid; j < DVC; j += NT) vs[j] = load_in<InT>(a.v, gh * DV + (size_t)chunk * DVC + j);
     if (tid == 0) {
         gates[0] = __ldg(a.alpha + gh);
         gates[1] = __ldg(a.beta + gh);
-        dst_s = dst;  // re-read after the reduction instead of holding a register
+        dst_s = dst;
     }
     __syncthreads();
 
@@ -282,7 +185,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
 #pragma unroll
         for (int i = tid; i < DK; i += 32) acc = fmaf(ks[i], qs[i], acc);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
         if (tid == 0) kq_s = acc;
     }
     __syncthreads();
@@ -291,35 +194,233 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     float4 w = red_w[0][cg];
 #pragma unroll
     for (int r = 1; r < RG; ++r) {
-        add4(u, red_u[r][cg]);
-        add4(w, red_w[r][cg]);
+        add4_rn(u, red_u[r][cg]);
+        add4_rn(w, red_w[r][cg]);
     }
     const float al = gates[0];
     const float be = gates[1];
     const float4 vv = reinterpret_cast<const float4*>(vs)[cg];
     float4 c;
-    c.x = be * (vv.x - al * u.x);
-    c.y = be * (vv.y - al * u.y);
-    c.z = be * (vv.z - al * u.z);
-    c.w = be * (vv.w - al * u.w);
+    c.x = __fmul_rn(be, fmaf(-al, u.x, vv.x));
+    c.y = __fmul_rn(be, fmaf(-al, u.y, vv.y));
+    c.z = __fmul_rn(be, fmaf(-al, u.z, vv.z));
+    c.w = __fmul_rn(be, fmaf(-al, u.w, vv.w));
     if (rg == 0) {
         const float kq = kq_s;
         float4 o;
-        o.x = fmaf(c.x, kq, al * w.x);
-        o.y = fmaf(c.y, kq, al * w.y);
-        o.z = fmaf(c.z, kq, al * w.z);
-        o.w = fmaf(c.w, kq, al * w.w);
+        o.x = fmaf(c.x, kq, __fmul_rn(al, w.x));
+        o.y = fmaf(c.y, kq, __fmul_rn(al, w.y));
+        o.z = fmaf(c.z, kq, __fmul_rn(al, w.z));
+        o.w = fmaf(c.w, kq, __fmul_rn(al, w.w));
         __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + col4, o);
     }
     float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst_s * a.Hv + h) * (DK * DV)) + toff;
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
         const float ki = ks[m * RG + rg];
-        s[m].x = fmaf(ki, c.x, al * s[m].x);
-        s[m].y = fmaf(ki, c.y, al * s[m].y);
-        s[m].z = fmaf(ki, c.z, al * s[m].z);
-        s[m].w = fmaf(ki, c.w, al * s[m].w);
+        s[m].x = fmaf(ki, c.x, __fmul_rn(al, s[m].x));
+        s[m].y = fmaf(ki, c.y, __fmul_rn(al, s[m].y));
+        s[m].z = fmaf(ki, c.z, __fmul_rn(al, s[m].z));
+        s[m].w = fmaf(ki, c.w, __fmul_rn(al, s[m].w));
         __stcs(D + m * kRowStep, s[m]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Register-tile kernel.  Value columns are independent, so a (b, h) tile is
+// split into DV / DVC column blocks, one CTA each (a column block's rows are
+// DVC * 4 contiguous bytes, read and written as float4 runs).  Thread layout
+// per CTA: CG = DVC / 4 column groups x RG = NT / CG row groups; thread
+// (rg, cg) holds rows i = m * RG + rg of its four columns in registers for
+// the whole call.
+//
+// Per token: partial sums of u = S k and w = S q over the thread's rows (k.q
+// alongside, in warp 0), one barrier, the cross-row-group sums from shared
+// memory, then c = beta (v - alpha u), o = alpha w + c (k.q) and the update
+// S' = alpha S + k c^T in registers, streamed to the token's destination slot.
+//
+// Everything a token needs besides the tile (k and q rows, its v columns, the
+// gates) is staged in shared memory.  Token 0's inputs are requested together
+// with the tile at kernel start; token t+1's are fetched while token t's tile
+// is being stored.  Shared memory stays small (a few KiB), which leaves the
+// unified L1 large enough to track the outstanding misses of the MINB CTAs
+// resident per SM -- measured on B200, a large shared-memory footprint caps
+// read+write streaming well below what register-resident tiles reach.
+//
+// MULTI = false is a single-token form of the same template (not launched:
+// gdn_tile1_kernel above serves T = 1).  Every form runs the same per-token
+// arithmetic in the same order, so T chained single-token calls and one
+// T-token call give identical bits.
+// ---------------------------------------------------------------------------
+template <int DK, int DV, int DVC, int NT, int MINB, typename InT, bool MULTI>
+__global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
+    constexpr int CG = DVC / 4;
+    static_assert(DV % DVC == 0 && DVC % 4 == 0 && NT % CG == 0 && NT >= 32 && NT >= DVC, "tile shape");
+    constexpr int RG = NT / CG;
+    static_assert(DK % RG == 0, "tile shape");
+    constexpr int RPT = DK / RG;
+    constexpr int NC = DV / DVC;
+    constexpr int NB = MULTI ? 2 : 1;  // token-input and reduction buffers (by token parity)
+
+    __shared__ float ks[NB][DK];
+    __shared__ float qs[NB][DK];
+    __shared__ float vs[NB][DVC];
+    __shared__ float gates[NB][2];
+    __shared__ int dst_s[NB];
+    __shared__ float4 red_u[NB][RG][CG];
+    __shared__ float4 red_w[NB][RG][CG];
+    __shared__ float kq_s[NB];
+
+    const int tid = threadIdx.x;
+    const int cg = tid % CG;
+    const int rg = tid / CG;
+    const int chunk = blockIdx.x % NC;
+    const int unit = blockIdx.x / NC;
+    const int h = unit % a.Hv;
+    const int b = unit / a.Hv;
+    const int T = MULTI ? a.T : 1;
+
+    int src, dst0 = 0;
+    const int status = request_status(a, b, T, src, dst0);
+    if (status != kRun) {
+        if (status == kBad && tid == 0) record_error(a.err, GDN_ERR_INDEX);
+        return;
+    }
+
+    // float4 offset of (row i, this thread's columns) in a tile: i * DV / 4 + chunk * CG + cg.
+    const int col4 = chunk * CG + cg;
+    const int toff = rg * (DV / 4) + col4;
+    constexpr int kRowStep = RG * (DV / 4);
+    const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV)) + toff;
+    float4 s[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+
+    const int hk = h / a.G;
+    // Token t's inputs: thread j < DK fetches k_j and q_j, thread j < DVC its v
+    // column, thread 0 the gates.
+    auto fetch = [&](int t, float& kx, float& qx, float& vx, float& ax, float& bx, int& dx) {
+        const size_t tok = (size_t)b * T + t;
+        if (tid < DK) {
+            kx = load_in<InT>(a.k, (tok * a.Hk + hk) * DK + tid);
+            qx = load_in<InT>(a.q, (tok * a.Hk + hk) * DK + tid);
+        }
+        if (tid < DVC) vx = load_in<InT>(a.v, (tok * a.Hv + h) * DV + (size_t)chunk * DVC + tid);
+        if (tid == 0) {
+            ax = __ldg(a.alpha + tok * a.Hv + h);
+            bx = __ldg(a.beta + tok * a.Hv + h);
+            dx = t == 0 ? dst0 : __ldg(a.dst_idx + tok);
+        }
+    };
+    // The destination slot goes through shared memory as well: re-reading it
+    // from global memory at store time would put a cache miss in front of the
+    // stores, and holding it in a register costs occupancy.
+    auto stage = [&](int buf, float kx, float qx, float vx, float ax, float bx, int dx) {
+        if (tid < DK) {
+            ks[buf][tid] = kx;
+            qs[buf][tid] = qx;
+        }
+        if (tid < DVC) vs[buf][tid] = vx;
+        if (tid == 0) {
+            gates[buf][0] = ax;
+            gates[buf][1] = bx;
+            dst_s[buf] = dx;
+        }
+    };
+    static_assert(NT >= DK || !MULTI, "one thread per k/q element when staging tokens");
+    {
+        float kx = 0.f, qx = 0.f, vx = 0.f, ax = 0.f, bx = 0.f;
+        int dx = 0;
+        if (NT >= DK) {
+            fetch(0, kx, qx, vx, ax, bx, dx);
+            stage(0, kx, qx, vx, ax, bx, dx);
+        } else {
+            const size_t kbase = ((size_t)b * a.Hk + hk) * DK;
+            for (int i = tid; i < DK; i += NT) {
+                ks[0][i] = load_in<InT>(a.k, kbase + i);
+                qs[0][i] = load_in<InT>(a.q, kbase + i);
+            }
+            fetch(0, kx, qx, vx, ax, bx, dx);
+            if (tid < DVC) vs[0][tid] = vx;
+            if (tid == 0) {
+                gates[0][0] = ax;
+                gates[0][1] = bx;
+                dst_s[0] = dx;
+            }
+        }
+    }
+    __syncthreads();
+
+    for (int t = 0; t < T; ++t) {
+        const int cb = MULTI ? (t & 1) : 0;
+        float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const int i = m * RG + rg;
+            fma4(pu, s[m], ks[cb][i]);
+            fma4(pw, s[m], qs[cb][i]);
+        }
+        red_u[cb][rg][cg] = pu;
+        red_w[cb][rg][cg] = pw;
+        if (tid < 32) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = tid; i < DK; i += 32) acc = fmaf(ks[cb][i], qs[cb][i], acc);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+            if (tid == 0) kq_s[cb] = acc;
+        }
+        __syncthreads();
+
+        // Next token's inputs are requested now; their latency hides behind this token's stores.
+        float kx = 0.f, qx = 0.f, vx = 0.f, ax = 0.f, bx = 0.f;
+        int dx = 0;
+        if (MULTI && t + 1 < T) fetch(t + 1, kx, qx, vx, ax, bx, dx);
+
+        float4 u = red_u[cb][0][cg];
+        float4 w = red_w[cb][0][cg];
+#pragma unroll
+        for (int r = 1; r < RG; ++r) {
+            add4_rn(u, red_u[cb][r][cg]);
+            add4_rn(w, red_w[cb][r][cg]);
+        }
+        const float al = gates[cb][0];
+        const float be = gates[cb][1];
+        const float4 vv = reinterpret_cast<const float4*>(vs[cb])[cg];
+        // Rounding is spelled out (fmaf / __fmul_rn) so that every form of this
+        // kernel, and every compiler context, evaluates the same operations.
+        float4 c;
+        c.x = __fmul_rn(be, fmaf(-al, u.x, vv.x));
+        c.y = __fmul_rn(be, fmaf(-al, u.y, vv.y));
+        c.z = __fmul_rn(be, fmaf(-al, u.z, vv.z));
+        c.w = __fmul_rn(be, fmaf(-al, u.w, vv.w));
+        const size_t gh = ((size_t)b * T + t) * a.Hv + h;
+        if (rg == 0) {
+            const float kq = kq_s[cb];
+            float4 o;
+            o.x = fmaf(c.x, kq, __fmul_rn(al, w.x));
+            o.y = fmaf(c.y, kq, __fmul_rn(al, w.y));
+            o.z = fmaf(c.z, kq, __fmul_rn(al, w.z));
+            o.w = fmaf(c.w, kq, __fmul_rn(al, w.w));
+            __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + col4, o);
+        }
+        const int dst = dst_s[cb];
+        float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst * a.Hv + h) * (DK * DV)) + toff;
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const float ki = ks[cb][m * RG + rg];
+            s[m].x = fmaf(ki, c.x, __fmul_rn(al, s[m].x));
+            s[m].y = fmaf(ki, c.y, __fmul_rn(al, s[m].y));
+            s[m].z = fmaf(ki, c.z, __fmul_rn(al, s[m].z));
+            s[m].w = fmaf(ki, c.w, __fmul_rn(al, s[m].w));
+            __stcs(D + m * kRowStep, s[m]);
+        }
+        if (MULTI && t + 1 < T) {
+            // The other buffer was last read during token t-1, before this token's barrier.
+            stage(cb ^ 1, kx, qx, vx, ax, bx, dx);
+            __syncthreads();
+        }
     }
 }
 
@@ -343,9 +444,10 @@ __global__ void gdn_column_kernel(StepArgs a) {
     const bool active = j < a.dv;
     const size_t tile = (size_t)a.dk * a.dv;
 
-    int src;
-    if (!request_in_range(a, b, src)) {
-        if (threadIdx.x == 0) record_error(a.err, GDN_ERR_INDEX);
+    int src, dst0 = 0;
+    const int status = request_status(a, b, a.T, src, dst0);
+    if (status != kRun) {
+        if (status == kBad && threadIdx.x == 0) record_error(a.err, GDN_ERR_INDEX);
         return;
     }
 
@@ -539,7 +641,8 @@ __global__ void __launch_bounds__(NT, 1) gdn_stream_kernel(StepArgs a) {
         if (p_next < n_local) fetch_indices(p_next);
         const int stage = n % STAGES;
         const bool valid = src >= 0 && src < a.num_slots && dst >= 0 && dst < a.num_slots;
-        meta[stage] = make_int2(dst, valid ? 1 : 0);
+        // meta.y: 1 run, 0 out-of-range (reported), -1 padding (skipped silently)
+        meta[stage] = make_int2(dst, valid ? 1 : (src == GDN_SLOT_NONE ? -1 : 0));
         uint64_t* bar = &bars[stage];
         if (!valid) {
             mbar_arrive(bar);
@@ -586,7 +689,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_stream_kernel(StepArgs a) {
         float kr[RPT];
         float4 vr = make_float4(0.f, 0.f, 0.f, 0.f);
         float al = 0.f, be = 0.f;
-        if (m.y) {
+        if (m.y == 1) {
             float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
             float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -625,7 +728,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_stream_kernel(StepArgs a) {
         // The stage is consumed: refill it with the unit STAGES ahead.
         if (tid == 0 && p_next < n_local) issue();
 
-        if (m.y) {
+        if (m.y == 1) {
             float4 uu = red_u[cg];
             float4 ww = red_w[cg];
 #pragma unroll
@@ -657,7 +760,7 @@ __global__ void __launch_bounds__(NT, 1) gdn_stream_kernel(StepArgs a) {
                 s[r].w = fmaf(kr[r], c.w, al * s[r].w);
                 __stcs(D + (size_t)(r * RG + rg) * CG + cg, s[r]);
             }
-        } else if (tid == 0) {
+        } else if (m.y == 0 && tid == 0) {
             record_error(a.err, GDN_ERR_INDEX);
         }
         // No second barrier: the next unit writes the other reduction buffer,
@@ -686,35 +789,36 @@ __global__ void gdn_commit_kernel(const int32_t* __restrict__ accept_len, int32_
 
 constexpr int kMaxDk = 4096;
 
-// Column-block width of the single-token tile kernel (value columns per CTA)
-// and its per-thread register budget, which sets how many CTAs stay resident
-// per SM.  Compile-time tunables; the defaults are the measured best on B200.
-#ifndef GDN_TILE1_COLS
-#define GDN_TILE1_COLS 64
+// Column-block width of the register-tile kernel (value columns per CTA) and
+// its per-thread register budget, which sets how many CTAs stay resident per
+// SM.  Compile-time tunables; the defaults are the measured best on B200
+// (64 columns, 128 threads, 96 registers: 5 CTAs and 160 KiB in flight per SM).
+#ifndef GDN_TILE_COLS
+#define GDN_TILE_COLS 64
 #endif
-#ifndef GDN_TILE1_MAXREG
-#define GDN_TILE1_MAXREG 100
+#ifndef GDN_TILE_MAXREG
+#define GDN_TILE_MAXREG 100
 #endif
-constexpr int kTile1Cols = GDN_TILE1_COLS;
 
-template <int DK, int DV, int NT>
+template <int DK, int DV>
 gdn_status launch_tile(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
+    constexpr int DVC = DV < GDN_TILE_COLS ? DV : GDN_TILE_COLS;
+    constexpr int NT = (DVC / 4) * 8;  // 8 row groups
+    constexpr int MINB0 = 65536 / (NT * GDN_TILE_MAXREG);
+    constexpr int MINB = MINB0 < 1 ? 1 : (MINB0 > 16 ? 16 : MINB0);
+    const dim3 grid((unsigned)(a.B * a.Hv * (DV / DVC)));
+    const bool bf = dtype == GDN_BF16;
     if (a.T == 1) {
-        constexpr int DVC = DV < kTile1Cols ? DV : kTile1Cols;
-        constexpr int NT1 = (DVC / 4) * 8;               // 8 row groups
-        constexpr int MINB = (65536 / (NT1 * GDN_TILE1_MAXREG)) < 16 ? (65536 / (NT1 * GDN_TILE1_MAXREG)) : 16;
-        const dim3 grid((unsigned)(a.B * a.Hv * (DV / DVC)));
-        if (dtype == GDN_BF16)
-            gdn_tile1_kernel<DK, DV, DVC, NT1, MINB, __nv_bfloat16><<<grid, NT1, 0, stream>>>(a);
+        if (bf)
+            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16><<<grid, NT, 0, stream>>>(a);
         else
-            gdn_tile1_kernel<DK, DV, DVC, NT1, MINB, float><<<grid, NT1, 0, stream>>>(a);
-        return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float><<<grid, NT, 0, stream>>>(a);
+    } else {
+        if (bf)
+            gdn_tile_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, true><<<grid, NT, 0, stream>>>(a);
+        else
+            gdn_tile_kernel<DK, DV, DVC, NT, MINB, float, true><<<grid, NT, 0, stream>>>(a);
     }
-    const dim3 grid((unsigned)(a.B * a.Hv));
-    if (dtype == GDN_BF16)
-        gdn_tile_kernel<DK, DV, NT, __nv_bfloat16><<<grid, NT, 0, stream>>>(a);
-    else
-        gdn_tile_kernel<DK, DV, NT, float><<<grid, NT, 0, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -795,7 +899,7 @@ gdn_status launch(const StepArgs& a, int32_t dtype, int32_t variant, cudaStream_
             return bf ? launch_stream<256, __nv_bfloat16>(a, stream) : launch_stream<256, float>(a, stream);
         case GDN_VARIANT_TILE:
             if (!tile_ok(a)) return GDN_ERR_INVALID_ARG;
-            return a.dk == 128 ? launch_tile<128, 128, 256>(a, dtype, stream) : launch_tile<64, 64, 128>(a, dtype, stream);
+            return a.dk == 128 ? launch_tile<128, 128>(a, dtype, stream) : launch_tile<64, 64>(a, dtype, stream);
         case GDN_VARIANT_COLUMN:
             return launch_column(a, dtype, stream);
         default:

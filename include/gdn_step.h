@@ -68,6 +68,11 @@ typedef enum gdn_status {
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
+/* Padding sentinel for src_idx: a request whose source slot is GDN_SLOT_NONE is
+ * skipped without an error (nothing read or written, its dst entries ignored),
+ * so a batch can be padded to a fixed size, e.g. for a captured CUDA graph. */
+#define GDN_SLOT_NONE (-1)
+
 /* Kernel choice for gdn_decode_step_variant. */
 typedef enum gdn_variant {
     GDN_VARIANT_AUTO = 0,   /* what gdn_decode_step uses: the first of TILE, STREAM, COLUMN that applies */
@@ -112,9 +117,10 @@ typedef enum gdn_variant {
  * bounds either way): the B*T destination slots are pairwise distinct; no
  * destination equals another request's source; for T > 1 no destination equals
  * the request's own source.  Many requests may share one source slot.
- * Index check: a request whose src or any of its T dst entries lies outside
- * [0, num_slots) is skipped entirely (no state, no output) and GDN_ERR_INDEX is
- * recorded.
+ * Index check: a request whose src is GDN_SLOT_NONE is padding and is skipped
+ * silently.  Any other request whose src or any of its T dst entries lies
+ * outside [0, num_slots) is skipped entirely (no state, no output) and
+ * GDN_ERR_INDEX is recorded.
  */
 gdn_status gdn_decode_step(float* pool, int32_t num_slots, const int32_t* src_idx,
                            const int32_t* dst_idx, const void* q, const void* k, const void* v,

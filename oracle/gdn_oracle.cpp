@@ -31,8 +31,10 @@
 // every read sees the pool as it was before the call; the state is rounded to
 // fp32 after every token (that is the stored value) and carried forward from
 // the rounded value; o is computed in double from the fp32-rounded state and
-// rounded to fp32; a request whose source or any destination index lies
-// outside [0, num_slots) is skipped as a whole (no state, no output written).
+// rounded to fp32; a request whose source index is -1 is padding and is
+// skipped; any other request whose source or any destination index lies
+// outside [0, num_slots) is skipped as a whole (no state, no output written)
+// and counted.
 //
 // Commit: accept_len[b] draft tokens were accepted.  0 keeps the committed
 // slot; a >= 1 selects the state written after draft token a-1, i.e.
@@ -73,6 +75,9 @@ struct Problem {
     int64_t B, T, Hk, Hv, dk, dv;
     int32_t dtype;
 };
+
+// A source index of -1 marks a padding request: skipped, not an error.
+bool request_is_padding(const Problem& p, int64_t b) { return p.src_idx[b] == -1; }
 
 bool request_is_valid(const Problem& p, int64_t b) {
     const int64_t s = p.src_idx[b];
@@ -161,7 +166,8 @@ extern "C" {
 // out: [B][T][Hv][dv] fp32.  All buffers are host memory owned by the caller.
 // Every request is solved from the pre-call pool before anything is written;
 // writes then go out in (b, t) order.  nthreads <= 1 runs single-threaded.
-// Returns the number of skipped requests, or -1 for invalid sizes.
+// Returns the number of requests skipped for an out-of-range index (padding
+// requests are not counted), or -1 for invalid sizes.
 int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* src_idx,
                                const int32_t* dst_idx, const void* q, const void* k,
                                const void* v, const float* alpha, const float* beta, float* out,
@@ -180,8 +186,8 @@ int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* sr
 
     auto work = [&](int64_t b0, int64_t b1) {
         for (int64_t b = b0; b < b1; ++b) {
-            valid[b] = request_is_valid(p, b) ? 1 : 0;
-            if (valid[b]) solve_request(p, b, &states[b * state_elems], &outs[b * out_elems]);
+            valid[b] = request_is_padding(p, b) ? 2 : (request_is_valid(p, b) ? 1 : 0);
+            if (valid[b] == 1) solve_request(p, b, &states[b * state_elems], &outs[b * out_elems]);
         }
     };
     int64_t nt = nthreads < 1 ? 1 : nthreads;
@@ -198,8 +204,8 @@ int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* sr
     int64_t skipped = 0;
     const int64_t tile = dk * dv;
     for (int64_t b = 0; b < B; ++b) {
-        if (!valid[b]) {
-            ++skipped;
+        if (valid[b] != 1) {
+            if (valid[b] == 0) ++skipped;
             continue;
         }
         for (int64_t t = 0; t < T; ++t) {

@@ -177,7 +177,7 @@ def test_out_of_range_indices_skip_and_report(torch_cuda, dk, dv, T):
     num_slots, B = 12, 4
     pool = wl.init_pool(rng, num_slots, 2, dk, dv)
     q, k, v, a, b = wl.random_step_inputs(rng, B, T, 1, 2, dk, dv, wl.BF16)
-    src = np.array([0, num_slots, 2, -1], np.int32)
+    src = np.array([0, num_slots, 2, -3], np.int32)
     dst = np.array([[4, 5], [6, 7], [8, 99], [10, 11]], np.int32)[:, :T].copy()
     if T == 1:
         dst[2, 0] = 99
@@ -201,6 +201,37 @@ def test_out_of_range_indices_skip_and_report(torch_cuda, dk, dv, T):
     gdn.gdn_commit(accept, committed, cur, num_slots, err_word=err)
     assert committed.cpu().tolist() == [4, 1, 2, 3]
     assert gdn.gdn_get_error(err) == gdn.GDN_ERR_INDEX
+
+
+@pytest.mark.parametrize("variant", [None, "stream", "column"])
+@pytest.mark.parametrize("T", [1, 3])
+def test_padding_requests_are_silent(torch_cuda, variant, T):
+    """src = GDN_SLOT_NONE (-1) rows are skipped without an error, whatever their dst holds."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    if variant == "stream" and T != 1:
+        pytest.skip("the streaming kernel serves single-token calls")
+    rng = np.random.default_rng(70 + T)
+    B, num_slots, Hk, Hv = 8, 40, 2, 4
+    pool = wl.init_pool(rng, num_slots, Hv, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, T, Hk, Hv, 128, 128, wl.BF16)
+    perm = rng.permutation(num_slots).astype(np.int32)
+    src = perm[:B].copy()
+    dst = perm[B:B + B * T].reshape(B, T).copy()
+    src[[1, 4, 7]] = -1
+    dst[1, 0], dst[4, -1] = 10 ** 6, -9   # ignored for padding rows
+    s = wl.Step(q, k, v, a, b, src, dst)
+    dev = to_torch(pool)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_gpu(dev, s, err=err, variant=variant)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    ref_pool, ref_out, skipped = run_oracle(pool, s)
+    assert skipped == 0
+    live = np.array([0, 2, 3, 5, 6])
+    check_pool(dev.cpu().numpy(), ref_pool, pool, dst[live])
+    assert np.all(out[[1, 4, 7]] == -7.0)
+    assert rel_err(out[live], ref_out[live]) <= TOL_OUT_BF16
 
 
 def test_unaligned_pool_uses_column_path(torch_cuda):

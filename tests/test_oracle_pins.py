@@ -310,6 +310,21 @@ def test_out_of_range_index_skips_request():
     assert np.array_equal(out[0], out_good[0])
 
 
+def test_padding_requests_are_skipped_silently():
+    """src = -1 marks padding: nothing is read or written and it is not an error,
+    whatever its destination entries hold; other negative sources are errors."""
+    rng = np.random.default_rng(29)
+    pool = wl.init_pool(rng, 6, 1, 16, 16)
+    q, k, v, a, b = _inputs(rng, 3, 2, 1, 1, 16, 16)
+    src = np.array([0, -1, -2], np.int32)
+    dst = np.array([[2, 3], [99, -5], [4, 5]], np.int32)
+    new, out, skipped = _run(pool, src, dst, q, k, v, a, b)
+    assert skipped == 1  # only the -2 source counts
+    assert np.all(out[1:] == -7.0)
+    alone, out_alone, _ = _run(pool, src[:1], dst[:1], q[:1], k[:1], v[:1], a[:1], b[:1])
+    assert np.array_equal(new, alone) and np.array_equal(out[0], out_alone[0])
+
+
 def test_bf16_inputs_widen_exactly():
     """bf16 inputs give the same result as their exactly widened fp32 values."""
     rng = np.random.default_rng(27)
