@@ -787,6 +787,39 @@ __global__ void gdn_commit_kernel(const int32_t* __restrict__ accept_len, int32_
     committed[b] = s;
 }
 
+// ---------------------------------------------------------------------------
+// Precondition check of a decode call's slot indices (gdn_check_step).
+// owner[] (int32 per slot, filled with -1 beforehand) records which request
+// writes each slot: claiming a slot twice means two writes alias; a request
+// whose source slot is owned by another request (or, with T > 1, by itself)
+// would read a slot written in the same call.
+// ---------------------------------------------------------------------------
+__global__ void gdn_claim_dst_kernel(const int32_t* __restrict__ src_idx, const int32_t* __restrict__ dst_idx,
+                                     int B, int T, int num_slots, int32_t* __restrict__ owner, int32_t* err) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= (int64_t)B * T) return;
+    const int b = (int)(e / T);
+    const int src = src_idx[b];
+    if (src == GDN_SLOT_NONE) return;
+    const int d = dst_idx[e];
+    if (d < 0 || d >= num_slots || src < 0 || src >= num_slots) {
+        // An index error outranks an alias report, whichever thread gets there first.
+        if (atomicCAS(err, 0, GDN_ERR_INDEX) == GDN_ERR_ALIAS) atomicCAS(err, GDN_ERR_ALIAS, GDN_ERR_INDEX);
+        return;
+    }
+    if (atomicCAS(owner + d, -1, b) != -1) record_error(err, GDN_ERR_ALIAS);
+}
+
+__global__ void gdn_check_src_kernel(const int32_t* __restrict__ src_idx, int B, int T, int num_slots,
+                                     const int32_t* __restrict__ owner, int32_t* err) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    const int src = src_idx[b];
+    if (src == GDN_SLOT_NONE || src < 0 || src >= num_slots) return;  // range errors: reported by the claim pass
+    const int o = owner[src];
+    if (o != -1 && (o != b || T > 1)) record_error(err, GDN_ERR_ALIAS);
+}
+
 constexpr int kMaxDk = 4096;
 
 // Column-block width of the register-tile kernel (value columns per CTA) and
@@ -948,6 +981,24 @@ extern "C" gdn_status gdn_commit(const int32_t* accept_len, int32_t* committed, 
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+extern "C" gdn_status gdn_check_step(const int32_t* src_idx, const int32_t* dst_idx, int32_t B, int32_t T,
+                                     int32_t num_slots, int32_t* scratch, int32_t* err_word, cudaStream_t stream) {
+    if (B < 0 || T < 1 || num_slots < 1 || (int64_t)B * T >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!src_idx || !dst_idx || !scratch || !err_word) return GDN_ERR_INVALID_ARG;
+    // 0xFF bytes make every int32 owner entry -1 ("unclaimed").
+    if (cudaMemsetAsync(scratch, 0xFF, sizeof(int32_t) * (size_t)num_slots, stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int threads = 256;
+    const int64_t n = (int64_t)B * T;
+    gdn_claim_dst_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, stream>>>(src_idx, dst_idx, B, T,
+                                                                                         num_slots, scratch, err_word);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    gdn_check_src_kernel<<<(B + threads - 1) / threads, threads, 0, stream>>>(src_idx, B, T, num_slots, scratch,
+                                                                              err_word);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 extern "C" gdn_status gdn_get_error(int32_t* err_word, int32_t* host_code, cudaStream_t stream) {
     if (!err_word || !host_code) return GDN_ERR_INVALID_ARG;
     int32_t value = 0;
@@ -966,6 +1017,7 @@ extern "C" const char* gdn_status_string(int32_t status) {
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_INDEX: return "GDN_ERR_INDEX";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS";
         default: return "GDN_UNKNOWN_STATUS";
     }
 }

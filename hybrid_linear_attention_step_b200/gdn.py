@@ -20,6 +20,9 @@ GDN_ERR_INVALID_ARG = 1
 GDN_ERR_CUDA = 2
 GDN_ERR_INDEX = 3
 GDN_ERR_TIMEOUT = 4
+GDN_ERR_ALIAS = 5
+
+GDN_SLOT_NONE = -1
 
 GDN_F32 = 0
 GDN_BF16 = 1
@@ -60,6 +63,8 @@ def load_library() -> ctypes.CDLL:
                                             i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     lib.gdn_commit.restype = i32
     lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
+    lib.gdn_check_step.restype = i32
+    lib.gdn_check_step.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     lib.gdn_get_error.restype = i32
     lib.gdn_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -155,6 +160,25 @@ def gdn_commit(accept_len: torch.Tensor, committed: torch.Tensor, cur: torch.Ten
         _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_commit")
+    return status
+
+
+def gdn_check_step(src_idx: torch.Tensor, dst_idx: torch.Tensor, num_slots: int, scratch: torch.Tensor,
+                   err_word: torch.Tensor, stream=None, check: bool = True) -> int:
+    """Enqueue the device-side precondition check of a decode call's slot indices
+    (see gdn_check_step in include/gdn_step.h).  scratch: int32 [>= num_slots]."""
+    B = src_idx.shape[0]
+    T = dst_idx.shape[1] if dst_idx.dim() == 2 else 1
+    if dst_idx.numel() != B * T:
+        raise ValueError("dst_idx must hold B*T entries")
+    if scratch.numel() < num_slots:
+        raise ValueError("scratch must hold num_slots int32 entries")
+    status = load_library().gdn_check_step(
+        _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32), int(B), int(T),
+        int(num_slots), _dev(scratch, "scratch", torch.int32), _dev(err_word, "err_word", torch.int32),
+        _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_check_step")
     return status
 
 

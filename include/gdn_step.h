@@ -63,7 +63,8 @@ typedef enum gdn_status {
     GDN_ERR_INVALID_ARG = 1, /* sizes, null pointers, dtype: rejected before launch */
     GDN_ERR_CUDA = 2,        /* a CUDA runtime call or launch failed */
     GDN_ERR_INDEX = 3,       /* device-side: a slot index or accept length was out of range */
-    GDN_ERR_TIMEOUT = 4      /* device-side: a bounded wait gave up (reserved) */
+    GDN_ERR_TIMEOUT = 4,     /* device-side: a bounded wait gave up */
+    GDN_ERR_ALIAS = 5        /* device-side (gdn_check_step): the slot indices break a precondition */
 } gdn_status;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -167,6 +168,37 @@ gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t
  */
 gdn_status gdn_commit(const int32_t* accept_len, int32_t* committed, const int32_t* cur, int32_t B,
                       int32_t T, int32_t num_slots, int32_t* err_word, cudaStream_t stream);
+
+/*
+ * gdn_check_step -- verify on the device that a decode call's slot indices meet
+ * gdn_decode_step's preconditions, without touching the pool.
+ *
+ * Copy-on-write reuse of cached checkpoints (24-ai.news article, "Hybrid prefix
+ * caching for GDN/Mamba"; zubnet.ai article, second paragraph) is only sound if no
+ * call writes a slot that another request of the same call reads, and if no two
+ * writes land in one slot.  This call checks exactly that for the indices a
+ * gdn_decode_step(src_idx, dst_idx, B, T, num_slots) would receive:
+ *   1. every non-padding request's src and its T dst entries lie in [0, num_slots)
+ *      (otherwise GDN_ERR_INDEX is recorded);
+ *   2. the destinations of all non-padding requests are pairwise distinct;
+ *   3. no destination equals the source of a different request;
+ *   4. for T > 1, no destination equals the request's own source
+ *      (2-4 otherwise record GDN_ERR_ALIAS).
+ * Requests whose src is GDN_SLOT_NONE are ignored.  In-place updates (T == 1,
+ * dst == src of the same request) and shared sources are allowed.
+ *
+ *   src_idx    device int32 [B]; dst_idx device int32 [B*T]
+ *   scratch    device int32 [num_slots], caller-owned working memory; its contents
+ *              on entry do not matter and on return are unspecified
+ *   err_word   device int32, required: the first error found is recorded there
+ *              (GDN_ERR_INDEX or GDN_ERR_ALIAS; read it with gdn_get_error)
+ * Three operations are enqueued on `stream` (a fill of scratch and two kernels);
+ * nothing synchronises.  Calls sharing one scratch buffer must not overlap.
+ * B >= 0 (0 is a no-op), T >= 1, num_slots >= 1; null pointers or bad sizes return
+ * GDN_ERR_INVALID_ARG.
+ */
+gdn_status gdn_check_step(const int32_t* src_idx, const int32_t* dst_idx, int32_t B, int32_t T,
+                          int32_t num_slots, int32_t* scratch, int32_t* err_word, cudaStream_t stream);
 
 /*
  * gdn_get_error -- read and clear a device error word.

@@ -66,6 +66,8 @@ def _load():
         lib.oracle_gdn_decode_step.restype = i64
         lib.oracle_gdn_decode_step.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
                                                i64, i64, i64, i64, i64, i64, i32, i32]
+        lib.oracle_gdn_check_step.restype = i32
+        lib.oracle_gdn_check_step.argtypes = [vp, vp, i64, i64, i64]
         lib.oracle_gdn_commit.restype = i64
         lib.oracle_gdn_commit.argtypes = [vp, vp, vp, i64, i64, i64]
         _lib = lib
@@ -140,6 +142,21 @@ def commit(accept_len, committed, cur, num_slots: int) -> int:
     if committed.shape != (B,) or cur.shape != (B, T):
         raise ValueError("committed must be [B] and cur [B, T]")
     r = _load().oracle_gdn_commit(_ptr(accept_len), _ptr(committed), _ptr(cur), B, T, int(num_slots))
+    if r < 0:
+        raise ValueError("oracle rejected the sizes")
+    return int(r)
+
+
+def check_step(src_idx, dst_idx, num_slots: int) -> int:
+    """Precondition check of one call's slot indices: 0 ok, 3 index out of range,
+    5 aliasing slots (see oracle_gdn_check_step)."""
+    _need(src_idx, np.int32, "src_idx")
+    _need(dst_idx, np.int32, "dst_idx")
+    B = src_idx.shape[0]
+    T = dst_idx.shape[1] if dst_idx.ndim == 2 else 1
+    if dst_idx.size != B * T:
+        raise ValueError("dst_idx must hold B*T entries")
+    r = _load().oracle_gdn_check_step(_ptr(src_idx), _ptr(dst_idx), B, T, int(num_slots))
     if r < 0:
         raise ValueError("oracle rejected the sizes")
     return int(r)

@@ -220,6 +220,38 @@ int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* sr
     return skipped;
 }
 
+// Precondition check of one decode call's slot indices, by brute force over
+// all pairs.  Returns 0 when they hold, 3 when a non-padding request has a
+// source or destination outside [0, num_slots), 5 when two destinations
+// coincide, a destination equals another request's source, or (T > 1) a
+// destination equals the request's own source; an index error takes
+// precedence.  Requests whose source is -1 are ignored.  -1 for invalid sizes.
+int32_t oracle_gdn_check_step(const int32_t* src_idx, const int32_t* dst_idx, int64_t B, int64_t T,
+                              int64_t num_slots) {
+    if (B < 0 || T < 1 || num_slots < 1) return -1;
+    auto live = [&](int64_t b) { return src_idx[b] != -1; };
+    for (int64_t b = 0; b < B; ++b) {
+        if (!live(b)) continue;
+        if (src_idx[b] < 0 || src_idx[b] >= num_slots) return 3;
+        for (int64_t t = 0; t < T; ++t)
+            if (dst_idx[b * T + t] < 0 || dst_idx[b * T + t] >= num_slots) return 3;
+    }
+    for (int64_t e = 0; e < B * T; ++e) {
+        if (!live(e / T)) continue;
+        for (int64_t f = e + 1; f < B * T; ++f)
+            if (live(f / T) && dst_idx[e] == dst_idx[f]) return 5;
+    }
+    for (int64_t b = 0; b < B; ++b) {
+        if (!live(b)) continue;
+        for (int64_t e = 0; e < B * T; ++e) {
+            const int64_t w = e / T;
+            if (!live(w) || dst_idx[e] != src_idx[b]) continue;
+            if (w != b || T > 1) return 5;
+        }
+    }
+    return 0;
+}
+
 // Accept-length commit.  committed: [B] int32 (updated in place); cur: [B][T].
 // Returns the number of skipped requests, or -1 for invalid sizes.
 int64_t oracle_gdn_commit(const int32_t* accept_len, int32_t* committed, const int32_t* cur,

@@ -39,8 +39,8 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings(lib):
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_status_string.argtypes = [ctypes.c_int32]
-    assert [lib.gdn_status_string(i).decode() for i in range(5)] == [
-        "GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_CUDA", "GDN_ERR_INDEX", "GDN_ERR_TIMEOUT"]
+    assert [lib.gdn_status_string(i).decode() for i in range(6)] == [
+        "GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_CUDA", "GDN_ERR_INDEX", "GDN_ERR_TIMEOUT", "GDN_ERR_ALIAS"]
     assert lib.gdn_status_string(99).decode() == "GDN_UNKNOWN_STATUS"
 
 
@@ -73,6 +73,13 @@ def test_host_validation_before_any_cuda_call(lib):
     assert f(8, 8, 8, 1, 0, 4, None, None) == 1
     assert f(None, 8, 8, 1, 1, 4, None, None) == 1
     assert f(None, None, None, 0, 1, 4, None, None) == 0
+    h = lib.gdn_check_step
+    h.restype = ctypes.c_int32
+    h.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int32] * 3 + [ctypes.c_void_p] * 3
+    assert h(8, 8, -1, 1, 4, 8, 8, None) == 1
+    assert h(8, 8, 1, 1, 4, None, 8, None) == 1   # scratch required
+    assert h(8, 8, 1, 1, 4, 8, None, None) == 1   # err_word required
+    assert h(None, None, 0, 1, 4, None, None, None) == 0
     g = lib.gdn_get_error
     g.restype = ctypes.c_int32
     g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]

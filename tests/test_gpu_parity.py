@@ -312,3 +312,50 @@ def test_stream_kernel_partial_waves(torch_cuda, B):
     ref_pool, ref_out, _ = run_oracle(pool, s)
     check_pool(dev.cpu().numpy(), ref_pool, pool, s.dst_idx)
     assert rel_err(out, ref_out) <= TOL_OUT_BF16
+
+
+def test_check_step_matches_oracle(torch_cuda):
+    """The device precondition check returns exactly the oracle's verdict (integer work: bit-exact)."""
+    torch = torch_cuda
+    import oracle
+    from hybrid_linear_attention_step_b200 import gdn
+
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scratch = torch.empty(64, dtype=torch.int32, device="cuda")
+    rng = np.random.default_rng(80)
+    seen = set()
+    for trial in range(300):
+        T = int(rng.integers(1, 4))
+        num_slots = int(rng.integers(4, 48))
+        B = int(rng.integers(1, 9))
+        src = rng.integers(-2, num_slots + 1, size=B).astype(np.int32)
+        dst = rng.integers(-1, num_slots + 1, size=(B, T)).astype(np.int32)
+        if trial % 2 == 0:
+            perm = rng.permutation(num_slots + B * T + B)[: B + B * T] % num_slots
+            src, dst = perm[:B].astype(np.int32), perm[B:].reshape(B, T).astype(np.int32)
+            if trial % 4 == 0:
+                src[rng.integers(0, B)] = -1
+        want = oracle.check_step(src, dst, num_slots)
+        gdn.gdn_check_step(torch.from_numpy(src).cuda(), torch.from_numpy(dst).cuda(), num_slots, scratch, err)
+        got = gdn.gdn_get_error(err)
+        assert got == want, (src.tolist(), dst.tolist(), num_slots, got, want)
+        seen.add(want)
+    assert seen == {0, 3, 5}
+
+
+@pytest.mark.parametrize("name", ["decode_b16", "prefix_cow", "speculative"])
+def test_check_step_accepts_the_workloads(torch_cuda, name):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    w = wl.WORKLOADS[name]()
+    s = w.steps[0]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scratch = torch.empty(w.num_slots, dtype=torch.int32, device="cuda")
+    gdn.gdn_check_step(torch.from_numpy(s.src_idx).cuda(), torch.from_numpy(s.dst_idx).cuda(), w.num_slots,
+                       scratch, err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    bad = s.dst_idx.copy()
+    bad[-1, -1] = s.src_idx[0]  # the last request writes the first request's source
+    gdn.gdn_check_step(torch.from_numpy(s.src_idx).cuda(), torch.from_numpy(bad).cuda(), w.num_slots, scratch, err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_ERR_ALIAS

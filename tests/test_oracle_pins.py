@@ -399,3 +399,53 @@ def test_commit_matches_brute_force_and_is_idempotent():
     kept = committed0.copy()
     oracle.commit(zero, kept, cur, num_slots)
     assert np.array_equal(kept, committed0)
+
+
+# ------------------------------------------------------- precondition check
+
+def _check_brute(src, dst, num_slots):
+    """The preconditions restated over explicit sets."""
+    B, T = dst.shape
+    live = [b for b in range(B) if src[b] != -1]
+    if any(not 0 <= src[b] < num_slots or not all(0 <= d < num_slots for d in dst[b]) for b in live):
+        return 3
+    writes = [(int(d), b) for b in live for d in dst[b]]
+    if len({d for d, _ in writes}) != len(writes):
+        return 5
+    for b in live:
+        for d, w in writes:
+            if d == src[b] and (w != b or T > 1):
+                return 5
+    return 0
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_check_step_matches_brute_force(T):
+    rng = np.random.default_rng(31 + T)
+    seen = set()
+    for trial in range(400):
+        num_slots = int(rng.integers(4, 24))
+        B = int(rng.integers(0, 6))
+        src = rng.integers(-2, num_slots + 1, size=B).astype(np.int32)
+        dst = rng.integers(-1, num_slots + 1, size=(B, T)).astype(np.int32)
+        if trial % 3 == 0 and B:  # mostly-valid cases: distinct fresh destinations
+            perm = rng.permutation(num_slots + B * T + B)[: B + B * T] % num_slots
+            src = perm[:B].astype(np.int32)
+            dst = perm[B:].reshape(B, T).astype(np.int32)
+        want = _check_brute(src, dst, num_slots)
+        assert oracle.check_step(src, dst, num_slots) == want
+        seen.add(want)
+    assert seen == {0, 3, 5}
+
+
+def test_check_step_named_cases():
+    ok = lambda s, d, n=10: oracle.check_step(np.array(s, np.int32), np.array(d, np.int32).reshape(len(s), -1), n)
+    assert ok([1, 2], [[1], [2]]) == 0          # in place, T = 1
+    assert ok([1, 1], [[3], [4]]) == 0          # shared source (copy-on-write)
+    assert ok([1, 2], [[3], [3]]) == 5          # two writes to one slot
+    assert ok([1, 2], [[2], [4]]) == 5          # writes another request's source
+    assert ok([1, 2], [[1, 3], [4, 5]]) == 5    # T > 1 writes its own source
+    assert ok([1, 2], [[3, 3], [4, 5]]) == 5    # duplicate within one request
+    assert ok([-1, 2], [[2, 2], [4, 5]]) == 0   # padding rows are ignored
+    assert ok([1, 2], [[3], [10]]) == 3         # out of range
+    assert ok([1, 2], [[2], [10]]) == 3         # index error takes precedence over aliasing
