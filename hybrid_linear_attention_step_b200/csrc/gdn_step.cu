@@ -28,6 +28,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace {
 
 struct StepArgs {
@@ -995,6 +997,59 @@ extern "C" gdn_status gdn_check_step(const int32_t* src_idx, const int32_t* dst_
                                                                                          num_slots, scratch, err_word);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     gdn_check_src_kernel<<<(B + threads - 1) / threads, threads, 0, stream>>>(src_idx, B, T, num_slots, scratch,
+                                                                              err_word);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free precondition check.  The owner map lives in this file-scope
+// device array (1 MiB per GPU that loads the library).  Host code must not pass
+// `g_check_owner` itself to a kernel: on the host that name is only a stand-in
+// for the device symbol.  Its device address is looked up once per device with
+// cudaGetSymbolAddress and cached; the claim and source kernels above then run
+// on it exactly as they run on a caller's scratch buffer.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t g_check_owner[GDN_CHECK_NOALLOC_MAX_SLOTS];
+
+namespace {
+
+std::atomic<int32_t*> g_check_owner_addr[kMaxDevices];
+
+// Device address of g_check_owner on the current device (nullptr on failure).
+int32_t* check_owner_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+    if (dev < kMaxDevices) {
+        int32_t* cached = g_check_owner_addr[dev].load(std::memory_order_acquire);
+        if (cached != nullptr) return cached;
+    }
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_check_owner) != cudaSuccess || addr == nullptr) return nullptr;
+    int32_t* owner = static_cast<int32_t*>(addr);
+    if (dev < kMaxDevices) g_check_owner_addr[dev].store(owner, std::memory_order_release);
+    return owner;
+}
+
+}  // namespace
+
+extern "C" gdn_status gdn_check_step_noalloc(const int32_t* src_idx, const int32_t* dst_idx, int32_t B, int32_t T,
+                                             int32_t num_slots, int32_t* err_word, cudaStream_t stream) {
+    if (B < 0 || T < 1 || num_slots < 1 || (int64_t)B * T >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (num_slots > GDN_CHECK_NOALLOC_MAX_SLOTS) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!src_idx || !dst_idx || !err_word) return GDN_ERR_INVALID_ARG;
+    int32_t* owner = check_owner_address();
+    if (owner == nullptr) return GDN_ERR_CUDA;
+    // Reset the entries this call uses (0xFF bytes = -1, "unclaimed"): the array
+    // still holds whatever the previous call left there.
+    if (cudaMemsetAsync(owner, 0xFF, sizeof(int32_t) * (size_t)num_slots, stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int threads = 256;
+    const int64_t n = (int64_t)B * T;
+    gdn_claim_dst_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, stream>>>(src_idx, dst_idx, B, T,
+                                                                                         num_slots, owner, err_word);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    gdn_check_src_kernel<<<(B + threads - 1) / threads, threads, 0, stream>>>(src_idx, B, T, num_slots, owner,
                                                                               err_word);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

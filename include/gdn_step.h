@@ -201,6 +201,36 @@ gdn_status gdn_check_step(const int32_t* src_idx, const int32_t* dst_idx, int32_
                           int32_t num_slots, int32_t* scratch, int32_t* err_word, cudaStream_t stream);
 
 /*
+ * gdn_check_step_noalloc -- gdn_check_step for callers that cannot allocate.
+ *
+ * No counterpart on the source pages: this is a convenience of this library.
+ * gdn_check_step needs a caller-provided scratch buffer of num_slots int32.  Some
+ * callers cannot get one: a serving process whose device memory has been handed
+ * in full to its own allocator (a raw cudaMalloc then fails or waits on that
+ * allocator), or a latency-critical loop with a no-allocation rule because
+ * cudaMalloc and cudaFree may synchronise the whole device.  This entry point
+ * performs the same check with no scratch argument: it uses a fixed array of
+ * GDN_CHECK_NOALLOC_MAX_SLOTS int32 (1 MiB) that lives in the library's device
+ * memory on every GPU that loads the library, until the process exits.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   Arguments, checks and error codes are those of gdn_check_step without
+ *   `scratch`.  num_slots > GDN_CHECK_NOALLOC_MAX_SLOTS returns GDN_ERR_INVALID_ARG
+ *   before anything is enqueued.
+ *   Set-up: the first call on a device (with that device current) looks up the
+ *   array's device address with cudaGetSymbolAddress and keeps it for later calls;
+ *   make that first call before any stream capture begins.
+ *   Sharing: every call on a device uses the same array.  Each call resets the part
+ *   it uses before checking, but calls that overlap on the GPU (different streams,
+ *   or different host threads, without ordering between them) race on the array
+ *   and may report wrong results.  Order such calls, or use gdn_check_step with
+ *   separate scratch buffers.
+ */
+#define GDN_CHECK_NOALLOC_MAX_SLOTS (1 << 18)
+gdn_status gdn_check_step_noalloc(const int32_t* src_idx, const int32_t* dst_idx, int32_t B, int32_t T,
+                                  int32_t num_slots, int32_t* err_word, cudaStream_t stream);
+
+/*
  * gdn_get_error -- read and clear a device error word.
  *
  * Synchronises `stream`, copies *err_word (device) to *host_code (host) and
