@@ -359,3 +359,83 @@ def test_check_step_accepts_the_workloads(torch_cuda, name):
     bad[-1, -1] = s.src_idx[0]  # the last request writes the first request's source
     gdn.gdn_check_step(torch.from_numpy(s.src_idx).cuda(), torch.from_numpy(bad).cuda(), w.num_slots, scratch, err)
     assert gdn.gdn_get_error(err) == gdn.GDN_ERR_ALIAS
+
+
+def test_cuda_graph_replay_of_padded_batches(torch_cuda):
+    """Static-shape decode calls captured once in a CUDA graph and replayed: the batch is padded
+    to a fixed size with GDN_SLOT_NONE rows, the slot tables are rewritten between replays, and
+    every replay matches the oracle (single-token and speculative calls in one graph)."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(100)
+    Bmax, Hk, Hv, dk, dv, num_slots, T = 12, 2, 4, 128, 128, 96, 2
+    pool_np = wl.init_pool(rng, num_slots, Hv, dk, dv)
+    pool = to_torch(pool_np)
+    q1, k1, v1, a1, b1 = (to_torch(x) for x in wl.random_step_inputs(rng, Bmax, 1, Hk, Hv, dk, dv, wl.BF16))
+    q2, k2, v2, a2, b2 = (to_torch(x) for x in wl.random_step_inputs(rng, Bmax, T, Hk, Hv, dk, dv, wl.BF16))
+    src1 = torch.full((Bmax,), -1, dtype=torch.int32, device="cuda")
+    dst1 = torch.full((Bmax, 1), -1, dtype=torch.int32, device="cuda")
+    src2 = torch.full((Bmax,), -1, dtype=torch.int32, device="cuda")
+    cur2 = torch.full((Bmax, T), -1, dtype=torch.int32, device="cuda")
+    out1 = torch.zeros((Bmax, 1, Hv, dv), device="cuda")
+    out2 = torch.zeros((Bmax, T, Hv, dv), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def calls():
+        gdn.gdn_decode_step(pool, src1, dst1, q1, k1, v1, a1, b1, out1, err_word=err)
+        gdn.gdn_decode_step(pool, src2, cur2, q2, k2, v2, a2, b2, out2, err_word=err)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        calls()  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        calls()
+
+    def to_host(t):  # bf16 tensors come back as their uint16 bit patterns
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).cpu().numpy().view(np.uint16)
+        return t.cpu().numpy()
+
+    host = {n: to_host(t) for n, t in dict(q1=q1, k1=k1, v1=v1, a1=a1, b1=b1, q2=q2, k2=k2, v2=v2, a2=a2,
+                                            b2=b2).items()}
+    bits = lambda t: t
+    for replay in range(3):
+        n1, n2 = int(rng.integers(1, Bmax)), int(rng.integers(1, Bmax))
+        perm = rng.permutation(num_slots).astype(np.int32)
+        s1 = np.full(Bmax, -1, np.int32)
+        d1 = np.full((Bmax, 1), -1, np.int32)
+        s2 = np.full(Bmax, -1, np.int32)
+        c2 = np.full((Bmax, T), -1, np.int32)
+        rows1 = np.sort(rng.choice(Bmax, n1, replace=False))
+        rows2 = np.sort(rng.choice(Bmax, n2, replace=False))
+        s1[rows1] = perm[:n1]
+        d1[rows1, 0] = perm[:n1]                                   # in place
+        s2[rows2] = perm[n1:n1 + n2]
+        c2[rows2] = perm[n1 + n2:n1 + n2 + n2 * T].reshape(n2, T)  # fresh draft slots
+        for t_, a_ in ((src1, s1), (dst1, d1), (src2, s2), (cur2, c2)):
+            t_.copy_(torch.from_numpy(a_))
+        before = pool.cpu().numpy()
+        out1.fill_(-7.0)
+        out2.fill_(-7.0)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_error(err) == gdn.GDN_OK
+        ref = before
+        ref, ref_o1, sk1 = run_oracle(ref, wl.Step(bits(host["q1"]), bits(host["k1"]), bits(host["v1"]), host["a1"],
+                                                   host["b1"], s1, d1))
+        ref, ref_o2, sk2 = run_oracle(ref, wl.Step(bits(host["q2"]), bits(host["k2"]), bits(host["v2"]), host["a2"],
+                                                   host["b2"], s2, c2))
+        assert sk1 == sk2 == 0
+        written = np.concatenate([d1[rows1].ravel(), c2[rows2].ravel()])
+        check_pool(pool.cpu().numpy(), ref, before, written)
+        o1, o2 = out1.cpu().numpy(), out2.cpu().numpy()
+        assert rel_err(o1[rows1], ref_o1[rows1]) <= TOL_OUT_BF16
+        assert rel_err(o2[rows2], ref_o2[rows2]) <= TOL_OUT_BF16
+        pad1 = np.setdiff1d(np.arange(Bmax), rows1)
+        pad2 = np.setdiff1d(np.arange(Bmax), rows2)
+        assert np.all(o1[pad1] == -7.0) and np.all(o2[pad2] == -7.0)
