@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).  See profiles/.
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "4839168da5fe371a7512349ae486f777fb52b16b0fd84890dd76a88eed4244a9",
-               "bytes_per_launch": 541148928 + 483413504,
+               "source_sha256": "0f7ea8d477b60cefbdac3a835a678b5b8a8a89eea3d73729c64fab3e78ee1145",
+               "bytes_per_launch": 541223168 + 483794688,
                "profile": "profiles/gdn_tile1_kernel_large_decode.md"}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
@@ -175,7 +175,7 @@ class LargeDecode:
     """Device-resident large decode: ``layers`` pools, per-layer inputs, one step = ``layers`` calls."""
 
     def __init__(self, layers: int = 8, num_slots: int = 2048, B: int = 256, device: str = "cuda",
-                 seed: int = 4, variant: str = "auto"):
+                 seed: int = 4, variant: str = "auto", fused: bool = False):
         import numpy as np
         import torch
 
@@ -187,8 +187,9 @@ class LargeDecode:
         self.Hk, self.Hv, self.dk, self.dv = c["Hk"], c["Hv"], c["dk"], c["dv"]
         self.seed = seed
         self.variant = variant
+        self.fused = fused  # raw q, k and gate pre-activations through gdn_decode_step_fused
         self.device = torch.device(device)
-        self.host_steps = [wl.large_layer_step(l, seed, B, num_slots) for l in range(layers)]
+        self.host_steps = [wl.large_layer_step(l, seed, B, num_slots, raw=fused) for l in range(layers)]
         self.pools, self.inputs, self.outs = [], [], []
         for l in range(layers):
             pool = torch.empty((num_slots, self.Hv, self.dk, self.dv), dtype=torch.float32, device=self.device)
@@ -215,7 +216,10 @@ class LargeDecode:
     def launch(self, l: int, stream=None):
         x = self.inputs[l]
         args = (self.pools[l], x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], self.outs[l])
-        if self.variant == "auto":
+        if self.fused:
+            self.gdn.gdn_decode_step_fused(*args, self.gdn.GDN_FUSE_GATES | self.gdn.GDN_FUSE_QK_NORM,
+                                           err_word=self.err, stream=stream)
+        elif self.variant == "auto":
             self.gdn.gdn_decode_step(*args, err_word=self.err, stream=stream)
         else:
             self.gdn.gdn_decode_step_variant(*args, self.variant, err_word=self.err, stream=stream)
@@ -530,8 +534,11 @@ def run_ours(args):
     rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     hbm_peak, peak_kind = peaks()
-    wk = LargeDecode(layers=args.layers, num_slots=args.slots, B=args.batch, variant=args.variant)
+    wk = LargeDecode(layers=args.layers, num_slots=args.slots, B=args.batch, variant=args.variant,
+                     fused=args.fused)
     kernel = KERNEL_NAMES[args.variant]
+    if args.fused:
+        kernel = kernel.replace(",bf16>", ",bf16,fused>")
     stream = torch.cuda.current_stream()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
     smi_id = vis.split(",")[local].strip() if vis else str(local)
@@ -637,7 +644,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "variant": args.variant, "graph": bool(args.graph), "B": wk.B, "layers": L, "Hk": wk.Hk, "Hv": wk.Hv, "dk": wk.dk,
+        "config": {"workload": WORKLOAD, "variant": args.variant, "graph": bool(args.graph),
+                   "fused_prologue": bool(args.fused), "B": wk.B, "layers": L, "Hk": wk.Hk, "Hv": wk.Hv, "dk": wk.dk,
                    "dv": wk.dv, "qkv": "bf16", "state": "f32", "slots_per_layer": wk.num_slots,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (4 GiB of state touched per step), no flush"},
@@ -673,6 +681,8 @@ def main():
                     help="large = the headline 8-layer decode; the others time one call of that workload")
     ap.add_argument("--graph", action="store_true", help="replay the timed calls from a CUDA graph "
                     "(smaller workloads only)")
+    ap.add_argument("--fused", action="store_true", help="large workload through gdn_decode_step_fused: raw "
+                    "gate pre-activations and unnormalised q, k, folded into the kernel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -52,7 +52,17 @@ struct StepArgs {
     float* out;
     int32_t* err;
     int num_slots, B, T, Hk, Hv, dk, dv, G;
+    int flags;  // GDN_FUSE_* bits (gdn_decode_step_fused); 0 for plain calls
 };
+
+// Fused prologue (gdn_decode_step_fused).  alpha = exp(-softplus(x)) equals
+// 1 / (1 + e^x) exactly, and beta = sigmoid(y) = 1 / (1 + e^-y); both limits
+// (e^x overflowing to +inf, or underflowing to 0) give the right 0 and 1.
+constexpr float kQkNormEps = 1e-6f;  // q_hat = q / sqrt(sum q^2 + eps), same for k
+
+__device__ __forceinline__ float alpha_from_raw(float x) { return 1.0f / (1.0f + expf(x)); }
+__device__ __forceinline__ float beta_from_raw(float y) { return 1.0f / (1.0f + expf(-y)); }
+__device__ __forceinline__ float inv_norm(float sum_sq) { return 1.0f / sqrtf(sum_sq + kQkNormEps); }
 
 __device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
     if (err != nullptr) atomicCAS(err, 0, code);
@@ -139,7 +149,7 @@ __device__ __forceinline__ void add4(float4& acc, const float4& x) {
 // and the gates are staged in shared memory so that no register holds them
 // while the tile is in flight.
 // ---------------------------------------------------------------------------
-template <int DK, int DV, int DVC, int NT, int MINB, typename InT>
+template <int DK, int DV, int DVC, int NT, int MINB, typename InT, bool FUSE>
 __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     constexpr int CG = DVC / 4;
     static_assert(DV % DVC == 0 && DVC % 4 == 0 && NT % CG == 0 && NT >= 32, "tile shape");
@@ -156,6 +166,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     __shared__ float4 red_u[RG][CG];
     __shared__ float4 red_w[RG][CG];
     __shared__ float kq_s;
+    __shared__ float rk_s, rq_s;  // 1 / |k|, 1 / |q| (fused q/k normalisation)
 
     const int tid = threadIdx.x;
     const int cg = tid % CG;
@@ -194,8 +205,10 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     }
     for (int j = tid; j < DVC; j += NT) vs[j] = load_in<InT>(a.v, gh * DV + (size_t)chunk * DVC + j);
     if (tid == 0) {
-        gates[0] = __ldg(a.alpha + gh);
-        gates[1] = __ldg(a.beta + gh);
+        const float x = __ldg(a.alpha + gh), y = __ldg(a.beta + gh);
+        const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
+        gates[0] = raw ? alpha_from_raw(x) : x;
+        gates[1] = raw ? beta_from_raw(y) : y;
         dst_s = dst;
     }
     __syncthreads();
@@ -216,6 +229,27 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
         for (int i = tid; i < DK; i += 32) acc = fmaf(ks[i], qs[i], acc);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+        if (FUSE && (a.flags & GDN_FUSE_QK_NORM)) {
+            // |k|^2 and |q|^2 alongside k.q: with k_hat = k rk and q_hat = q rq the
+            // update needs only S k_hat = (S k) rk, S q_hat = (S q) rq, k_hat.q_hat = (k.q) rk rq.
+            float kk = 0.f, qq = 0.f;
+#pragma unroll
+            for (int i = tid; i < DK; i += 32) {
+                kk = fmaf(ks[i], ks[i], kk);
+                qq = fmaf(qs[i], qs[i], qq);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, kk, off));
+                qq = __fadd_rn(qq, __shfl_xor_sync(0xffffffffu, qq, off));
+            }
+            if (tid == 0) {
+                const float rk = inv_norm(kk), rq = inv_norm(qq);
+                rk_s = rk;
+                rq_s = rq;
+                acc = __fmul_rn(__fmul_rn(acc, rk), rq);
+            }
+        }
         if (tid == 0) kq_s = acc;
     }
     __syncthreads();
@@ -230,6 +264,13 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     const float al = gates[0];
     const float be = gates[1];
     const float4 vv = reinterpret_cast<const float4*>(vs)[cg];
+    float rk = 1.f;
+    if (FUSE && (a.flags & GDN_FUSE_QK_NORM)) {
+        rk = rk_s;
+        const float rq = rq_s;
+        u = make_float4(__fmul_rn(u.x, rk), __fmul_rn(u.y, rk), __fmul_rn(u.z, rk), __fmul_rn(u.w, rk));
+        w = make_float4(__fmul_rn(w.x, rq), __fmul_rn(w.y, rq), __fmul_rn(w.z, rq), __fmul_rn(w.w, rq));
+    }
     float4 c;
     c.x = __fmul_rn(be, fmaf(-al, u.x, vv.x));
     c.y = __fmul_rn(be, fmaf(-al, u.y, vv.y));
@@ -243,6 +284,10 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
         o.z = fmaf(c.z, kq, __fmul_rn(al, w.z));
         o.w = fmaf(c.w, kq, __fmul_rn(al, w.w));
         __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + col4, o);
+    }
+    if (FUSE && (a.flags & GDN_FUSE_QK_NORM)) {
+        // k_hat_i c_j = k_i (rk c_j): scale c once instead of every k_i
+        c = make_float4(__fmul_rn(c.x, rk), __fmul_rn(c.y, rk), __fmul_rn(c.z, rk), __fmul_rn(c.w, rk));
     }
     float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst_s * a.Hv + h) * (DK * DV)) + toff;
 #pragma unroll
@@ -282,7 +327,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
 // arithmetic in the same order, so T chained single-token calls and one
 // T-token call give identical bits.
 // ---------------------------------------------------------------------------
-template <int DK, int DV, int DVC, int NT, int MINB, typename InT, bool MULTI>
+template <int DK, int DV, int DVC, int NT, int MINB, typename InT, bool MULTI, bool FUSE>
 __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     constexpr int CG = DVC / 4;
     static_assert(DV % DVC == 0 && DVC % 4 == 0 && NT % CG == 0 && NT >= 32 && NT >= DVC, "tile shape");
@@ -300,6 +345,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     __shared__ float4 red_u[NB][RG][CG];
     __shared__ float4 red_w[NB][RG][CG];
     __shared__ float kq_s[NB];
+    __shared__ float rk_s[NB], rq_s[NB];  // 1 / |k|, 1 / |q| (fused q/k normalisation)
 
     const int tid = threadIdx.x;
     const int cg = tid % CG;
@@ -337,8 +383,10 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
         }
         if (tid < DVC) vx = load_in<InT>(a.v, (tok * a.Hv + h) * DV + (size_t)chunk * DVC + tid);
         if (tid == 0) {
-            ax = __ldg(a.alpha + tok * a.Hv + h);
-            bx = __ldg(a.beta + tok * a.Hv + h);
+            const float x = __ldg(a.alpha + tok * a.Hv + h), y = __ldg(a.beta + tok * a.Hv + h);
+            const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
+            ax = raw ? alpha_from_raw(x) : x;
+            bx = raw ? beta_from_raw(y) : y;
             dx = t == 0 ? dst0 : __ldg(a.dst_idx + tok);
         }
     };
@@ -399,6 +447,25 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             for (int i = tid; i < DK; i += 32) acc = fmaf(ks[cb][i], qs[cb][i], acc);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+            if (FUSE && (a.flags & GDN_FUSE_QK_NORM)) {
+                float kk = 0.f, qq = 0.f;
+#pragma unroll
+                for (int i = tid; i < DK; i += 32) {
+                    kk = fmaf(ks[cb][i], ks[cb][i], kk);
+                    qq = fmaf(qs[cb][i], qs[cb][i], qq);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, kk, off));
+                    qq = __fadd_rn(qq, __shfl_xor_sync(0xffffffffu, qq, off));
+                }
+                if (tid == 0) {
+                    const float rk = inv_norm(kk), rq = inv_norm(qq);
+                    rk_s[cb] = rk;
+                    rq_s[cb] = rq;
+                    acc = __fmul_rn(__fmul_rn(acc, rk), rq);
+                }
+            }
             if (tid == 0) kq_s[cb] = acc;
         }
         __syncthreads();
@@ -418,6 +485,13 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
         const float al = gates[cb][0];
         const float be = gates[cb][1];
         const float4 vv = reinterpret_cast<const float4*>(vs[cb])[cg];
+        float rk = 1.f;
+        if (FUSE && (a.flags & GDN_FUSE_QK_NORM)) {
+            rk = rk_s[cb];
+            const float rq = rq_s[cb];
+            u = make_float4(__fmul_rn(u.x, rk), __fmul_rn(u.y, rk), __fmul_rn(u.z, rk), __fmul_rn(u.w, rk));
+            w = make_float4(__fmul_rn(w.x, rq), __fmul_rn(w.y, rq), __fmul_rn(w.z, rq), __fmul_rn(w.w, rq));
+        }
         // Rounding is spelled out (fmaf / __fmul_rn) so that every form of this
         // kernel, and every compiler context, evaluates the same operations.
         float4 c;
@@ -435,6 +509,8 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             o.w = fmaf(c.w, kq, __fmul_rn(al, w.w));
             __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + col4, o);
         }
+        if (FUSE && (a.flags & GDN_FUSE_QK_NORM))
+            c = make_float4(__fmul_rn(c.x, rk), __fmul_rn(c.y, rk), __fmul_rn(c.z, rk), __fmul_rn(c.w, rk));
         const int dst = dst_s[cb];
         float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst * a.Hv + h) * (DK * DV)) + toff;
 #pragma unroll
@@ -495,18 +571,33 @@ __global__ void gdn_column_kernel(StepArgs a) {
         const int dst = __ldg(a.dst_idx + tok);
         float* D = a.pool + ((size_t)dst * a.Hv + h) * tile;
         if (active) {
-            float u = 0.f, w = 0.f, kq = 0.f;
+            float u = 0.f, w = 0.f, kq = 0.f, kk = 0.f, qq = 0.f;
             for (int i = 0; i < a.dk; ++i) {
                 const float m = S[(size_t)i * a.dv + j];
                 u = fmaf(m, ks[i], u);
                 w = fmaf(m, qs[i], w);
                 kq = fmaf(ks[i], qs[i], kq);
+                kk = fmaf(ks[i], ks[i], kk);
+                qq = fmaf(qs[i], qs[i], qq);
             }
             const size_t gh = tok * a.Hv + h;
-            const float al = __ldg(a.alpha + gh);
-            const float be = __ldg(a.beta + gh);
-            const float c = be * (load_in<InT>(a.v, gh * a.dv + j) - al * u);
+            float al = __ldg(a.alpha + gh);
+            float be = __ldg(a.beta + gh);
+            if (a.flags & GDN_FUSE_GATES) {
+                al = alpha_from_raw(al);
+                be = beta_from_raw(be);
+            }
+            float rk = 1.f;
+            if (a.flags & GDN_FUSE_QK_NORM) {  // see gdn_tile1_kernel: normalisation folded into u, w, k.q, c
+                rk = inv_norm(kk);
+                const float rq = inv_norm(qq);
+                u *= rk;
+                w *= rq;
+                kq = kq * rk * rq;
+            }
+            float c = be * (load_in<InT>(a.v, gh * a.dv + j) - al * u);
             a.out[gh * a.dv + j] = fmaf(c, kq, al * w);
+            c *= rk;
             for (int i = 0; i < a.dk; ++i) {
                 const float m = S[(size_t)i * a.dv + j];
                 D[(size_t)i * a.dv + j] = fmaf(ks[i], c, al * m);
@@ -863,8 +954,8 @@ constexpr int kMaxDk = 4096;
 #define GDN_TILE_MAXREG 100
 #endif
 
-template <int DK, int DV>
-gdn_status launch_tile(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
+template <int DK, int DV, bool FUSE>
+gdn_status launch_tile_impl(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
     constexpr int DVC = DV < GDN_TILE_COLS ? DV : GDN_TILE_COLS;
     constexpr int NT = (DVC / 4) * 8;  // 8 row groups
     constexpr int MINB0 = 65536 / (NT * GDN_TILE_MAXREG);
@@ -883,22 +974,30 @@ gdn_status launch_tile(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = bf ? cudaLaunchKernelEx(&cfg, gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16>, a)
-                                 : cudaLaunchKernelEx(&cfg, gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float>, a);
+        const cudaError_t e =
+            bf ? cudaLaunchKernelEx(&cfg, gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, FUSE>, a)
+               : cudaLaunchKernelEx(&cfg, gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float, FUSE>, a);
         if (e != cudaSuccess) return GDN_ERR_CUDA;
 #else
         if (bf)
-            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16><<<grid, NT, 0, stream>>>(a);
+            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, FUSE><<<grid, NT, 0, stream>>>(a);
         else
-            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float><<<grid, NT, 0, stream>>>(a);
+            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float, FUSE><<<grid, NT, 0, stream>>>(a);
 #endif
     } else {
+        // The fused multi-token form needs a few more registers than 5 CTAs/SM allow.
+        constexpr int MINB_T = (FUSE && MINB > 1) ? MINB - 1 : MINB;
         if (bf)
-            gdn_tile_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, true><<<grid, NT, 0, stream>>>(a);
+            gdn_tile_kernel<DK, DV, DVC, NT, MINB_T, __nv_bfloat16, true, FUSE><<<grid, NT, 0, stream>>>(a);
         else
-            gdn_tile_kernel<DK, DV, DVC, NT, MINB, float, true><<<grid, NT, 0, stream>>>(a);
+            gdn_tile_kernel<DK, DV, DVC, NT, MINB_T, float, true, FUSE><<<grid, NT, 0, stream>>>(a);
     }
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <int DK, int DV>
+gdn_status launch_tile(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
+    return a.flags ? launch_tile_impl<DK, DV, true>(a, dtype, stream) : launch_tile_impl<DK, DV, false>(a, dtype, stream);
 }
 
 gdn_status launch_column(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
@@ -950,7 +1049,7 @@ gdn_status launch_stream(const StepArgs& a, cudaStream_t stream) {
 // a compiled tile shape and 16-byte aligned pool/out; the column kernel takes
 // anything.
 bool stream_ok(const StepArgs& a) {
-    return a.T == 1 && a.dk == 128 && a.dv == 128 && ((int64_t)a.B * a.Hv) % 4 == 0 && aligned16(a.pool) &&
+    return a.flags == 0 && a.T == 1 && a.dk == 128 && a.dv == 128 && ((int64_t)a.B * a.Hv) % 4 == 0 && aligned16(a.pool) &&
            aligned16(a.out) && aligned16(a.q) && aligned16(a.k) && aligned16(a.v) && aligned16(a.alpha) &&
            aligned16(a.beta);
 }
@@ -1003,8 +1102,27 @@ extern "C" gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, co
     if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out) return GDN_ERR_INVALID_ARG;
 
     const StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word,
-                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk};
+                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk, 0};
     return launch(a, qkv_dtype, variant, stream);
+}
+
+extern "C" gdn_status gdn_decode_step_fused(float* pool, int32_t num_slots, const int32_t* src_idx,
+                                            const int32_t* dst_idx, const void* q, const void* k, const void* v,
+                                            const float* alpha_or_x, const float* beta_or_y, float* out, int32_t B,
+                                            int32_t T, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                                            int32_t qkv_dtype, int32_t flags, int32_t* err_word,
+                                            cudaStream_t stream) {
+    if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return GDN_ERR_INVALID_ARG;
+    if (Hv % Hk != 0 || dk > kMaxDk) return GDN_ERR_INVALID_ARG;
+    if (qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if ((flags & ~(GDN_FUSE_GATES | GDN_FUSE_QK_NORM)) != 0) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)B * Hv * 4 >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha_or_x || !beta_or_y || !out)
+        return GDN_ERR_INVALID_ARG;
+    const StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha_or_x, beta_or_y, out, err_word,
+                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk, flags};
+    return launch(a, qkv_dtype, GDN_VARIANT_AUTO, stream);
 }
 
 extern "C" gdn_status gdn_decode_step(float* pool, int32_t num_slots, const int32_t* src_idx,

@@ -24,6 +24,9 @@ GDN_ERR_ALIAS = 5
 
 GDN_SLOT_NONE = -1
 
+GDN_FUSE_GATES = 1
+GDN_FUSE_QK_NORM = 2
+
 GDN_F32 = 0
 GDN_BF16 = 1
 
@@ -61,6 +64,9 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_decode_step_variant.restype = i32
     lib.gdn_decode_step_variant.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                             i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    lib.gdn_decode_step_fused.restype = i32
+    lib.gdn_decode_step_fused.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                          i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.gdn_commit.restype = i32
     lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
     lib.gdn_check_step.restype = i32
@@ -142,6 +148,21 @@ def gdn_decode_step_variant(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: 
                                                     _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_decode_step_variant")
+    return status
+
+
+def gdn_decode_step_fused(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
+                          q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          alpha_or_x: torch.Tensor, beta_or_y: torch.Tensor, out: torch.Tensor, flags: int,
+                          err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """gdn_decode_step with the input prologue folded in (see gdn_decode_step_fused in
+    include/gdn_step.h): GDN_FUSE_GATES makes alpha_or_x / beta_or_y the raw x, y;
+    GDN_FUSE_QK_NORM L2-normalises q and k inside the kernel."""
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha_or_x, beta_or_y, out)
+    status = load_library().gdn_decode_step_fused(*args, int(flags), _ptr_or_null(err_word, "err_word"),
+                                                  _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_decode_step_fused")
     return status
 
 

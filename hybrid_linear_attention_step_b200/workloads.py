@@ -140,6 +140,22 @@ def random_step_inputs(rng: np.random.Generator, B: int, T: int, Hk: int, Hv: in
     return q, k, v, alpha, beta
 
 
+def random_raw_step_inputs(rng: np.random.Generator, B: int, T: int, Hk: int, Hv: int, dk: int, dv: int,
+                           dtype: str = BF16):
+    """Raw per-token projections for the fused prologue: q, k, v ~ N(0, 1) without
+    normalisation, and the gate pre-activations x, y ~ N(0, 1) (fp32)."""
+    q = rng.standard_normal((B, T, Hk, dk), dtype=np.float32)
+    k = rng.standard_normal((B, T, Hk, dk), dtype=np.float32)
+    v = rng.standard_normal((B, T, Hv, dv), dtype=np.float32)
+    x = rng.standard_normal((B, T, Hv)).astype(np.float32)
+    y = rng.standard_normal((B, T, Hv)).astype(np.float32)
+    if dtype == BF16:
+        q, k, v = f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(v)
+    elif dtype != F32:
+        raise ValueError(dtype)
+    return q, k, v, x, y
+
+
 def init_pool(rng: np.random.Generator, num_slots: int, Hv: int, dk: int, dv: int,
               std: float = STATE_STD) -> np.ndarray:
     """A host slot pool with every element ~ N(0, std), float32."""
@@ -225,12 +241,16 @@ def speculative(seed: int = 3) -> Workload:
 
 
 def large_layer_step(layer: int, seed: int = LARGE["seed"], B: int = LARGE["B"],
-                     num_slots: int = LARGE["num_slots"]) -> Step:
-    """Inputs of one layer of the large decode: in place on a random slot permutation."""
+                     num_slots: int = LARGE["num_slots"], raw: bool = False) -> Step:
+    """Inputs of one layer of the large decode: in place on a random slot permutation.
+
+    raw=True draws the fused prologue's inputs instead (unnormalised q, k and the gate
+    pre-activations x, y in the alpha/beta fields)."""
     c = LARGE
     rng = np.random.default_rng([seed, layer])
     slots = rng.permutation(num_slots)[:B].astype(np.int32)
-    q, k, v, a, b = random_step_inputs(rng, B, 1, c["Hk"], c["Hv"], c["dk"], c["dv"], c["dtype"])
+    draw = random_raw_step_inputs if raw else random_step_inputs
+    q, k, v, a, b = draw(rng, B, 1, c["Hk"], c["Hv"], c["dk"], c["dv"], c["dtype"])
     return Step(q, k, v, a, b, slots.copy(), slots.reshape(B, 1).copy())
 
 

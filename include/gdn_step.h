@@ -145,6 +145,33 @@ gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t
                                    int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int32_t qkv_dtype,
                                    int32_t* err_word, int32_t variant, cudaStream_t stream);
 
+/* Flags of gdn_decode_step_fused. */
+#define GDN_FUSE_GATES 1   /* alpha/beta arguments are raw x, y: alpha = exp(-softplus(x)), beta = sigmoid(y) */
+#define GDN_FUSE_QK_NORM 2 /* q and k are L2-normalised per (token, key head): x / sqrt(sum x^2 + 1e-6) */
+
+/*
+ * gdn_decode_step_fused -- gdn_decode_step with its input prologue folded in.
+ *
+ * The pages collapse multi-step prologues (norms, gate maps) into the kernel that
+ * consumes them, keeping intermediates in registers (zubnet.ai article, second
+ * paragraph: QK-RMSNorm + partial RoPE + gate split, 5 kernels to 1).  This entry
+ * does the same for the GDN step: the raw per-token projections enter directly.
+ *   flags & GDN_FUSE_GATES:   `alpha_or_x`, `beta_or_y` hold raw x, y [B][T][Hv]
+ *                             (fp32); the step uses alpha = exp(-softplus(x)) and
+ *                             beta = sigmoid(y).  A model's own scale or bias on x,
+ *                             if it has one, is applied by the caller.
+ *   flags & GDN_FUSE_QK_NORM: q and k are used as q / sqrt(|q|^2 + 1e-6) and
+ *                             k / sqrt(|k|^2 + 1e-6), per (token, key head).
+ * Without flags the call is gdn_decode_step.  Same layouts, preconditions, errors
+ * and bytes moved as gdn_decode_step; unknown flag bits return GDN_ERR_INVALID_ARG.
+ * Served by the register-tile kernels (column kernel for other shapes/alignments).
+ */
+gdn_status gdn_decode_step_fused(float* pool, int32_t num_slots, const int32_t* src_idx,
+                                 const int32_t* dst_idx, const void* q, const void* k, const void* v,
+                                 const float* alpha_or_x, const float* beta_or_y, float* out, int32_t B,
+                                 int32_t T, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int32_t qkv_dtype,
+                                 int32_t flags, int32_t* err_word, cudaStream_t stream);
+
 /*
  * gdn_commit -- accept speculative draft tokens by rewriting an int32 index table.
  *

@@ -66,6 +66,9 @@ def _load():
         lib.oracle_gdn_decode_step.restype = i64
         lib.oracle_gdn_decode_step.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
                                                i64, i64, i64, i64, i64, i64, i32, i32]
+        lib.oracle_gdn_decode_step_fused.restype = i64
+        lib.oracle_gdn_decode_step_fused.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                     i64, i64, i64, i64, i64, i64, i32, i32, i32]
         lib.oracle_gdn_check_step.restype = i32
         lib.oracle_gdn_check_step.argtypes = [vp, vp, i64, i64, i64]
         lib.oracle_gdn_commit.restype = i64
@@ -83,13 +86,18 @@ def _need(a: np.ndarray, dtype, name: str) -> None:
         raise TypeError(f"{name} must be a C-contiguous numpy array of {np.dtype(dtype)}")
 
 
-def decode_step(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, *, nthreads: int = 1) -> int:
+FUSE_GATES = 1
+FUSE_QK_NORM = 2
+
+
+def decode_step(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, *, nthreads: int = 1, flags: int = 0) -> int:
     """One decode call on host arrays; ``pool`` and ``out`` are updated in place.
 
     pool  [num_slots, Hv, dk, dv] float32
     src_idx [B] int32, dst_idx [B, T] (or [B] for T = 1) int32
     q, k  [B, T, Hk, dk] and v [B, T, Hv, dv]: float32, or uint16 bfloat16 bit patterns
-    alpha, beta [B, T, Hv] float32; out [B, T, Hv, dv] float32
+    alpha, beta [B, T, Hv] float32 (raw x, y when flags & FUSE_GATES); out [B, T, Hv, dv] float32
+    flags: FUSE_GATES (alpha = exp(-softplus(x)), beta = sigmoid(y)) | FUSE_QK_NORM
     Returns the number of requests skipped for an out-of-range index.
     """
     _need(pool, np.float32, "pool")
@@ -120,9 +128,14 @@ def decode_step(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, *, nthreads: 
     _need(out, np.float32, "out")
     if out.shape != (B, T, Hv, dv):
         raise ValueError("out must be [B, T, Hv, dv]")
-    r = _load().oracle_gdn_decode_step(
-        _ptr(pool), num_slots, _ptr(src_idx), _ptr(dst_idx), _ptr(q), _ptr(k), _ptr(v),
-        _ptr(alpha), _ptr(beta), _ptr(out), B, T, Hk, Hv, dk, dv, dtype, int(nthreads))
+    if flags:
+        r = _load().oracle_gdn_decode_step_fused(
+            _ptr(pool), num_slots, _ptr(src_idx), _ptr(dst_idx), _ptr(q), _ptr(k), _ptr(v),
+            _ptr(alpha), _ptr(beta), _ptr(out), B, T, Hk, Hv, dk, dv, dtype, int(flags), int(nthreads))
+    else:
+        r = _load().oracle_gdn_decode_step(
+            _ptr(pool), num_slots, _ptr(src_idx), _ptr(dst_idx), _ptr(q), _ptr(k), _ptr(v),
+            _ptr(alpha), _ptr(beta), _ptr(out), B, T, Hk, Hv, dk, dv, dtype, int(nthreads))
     if r < 0:
         raise ValueError("oracle rejected the sizes")
     return int(r)

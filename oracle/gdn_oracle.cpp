@@ -74,7 +74,22 @@ struct Problem {
     const float* beta;
     int64_t B, T, Hk, Hv, dk, dv;
     int32_t dtype;
+    int32_t flags;  // 1: alpha/beta are raw x, y; 2: L2-normalise q and k
 };
+
+// Fused prologue, from its definition: alpha = exp(-softplus(x)) with
+// softplus(x) = log(1 + e^x) (written so that e^x never overflows), beta =
+// sigmoid(y) = 1 / (1 + e^-y), and x_hat = x / sqrt(sum x^2 + 1e-6).
+double softplus(double x) { return x > 0.0 ? x + std::log1p(std::exp(-x)) : std::log1p(std::exp(x)); }
+double alpha_of(double x) { return std::exp(-softplus(x)); }
+double beta_of(double y) { return 1.0 / (1.0 + std::exp(-y)); }
+
+void l2_normalise(std::vector<double>& x) {
+    double ss = 0.0;
+    for (double e : x) ss += e * e;
+    const double n = std::sqrt(ss + 1e-6);
+    for (double& e : x) e /= n;
+}
 
 // A source index of -1 marks a padding request: skipped, not an error.
 bool request_is_padding(const Problem& p, int64_t b) { return p.src_idx[b] == -1; }
@@ -116,8 +131,16 @@ void solve_request(const Problem& p, int64_t b, float* states, float* outs) {
                 qv[i] = input_at(p.q, p.dtype, (tok * p.Hk + hk) * dk + i);
             }
             for (int64_t j = 0; j < dv; ++j) vv[j] = input_at(p.v, p.dtype, (tok * p.Hv + h) * dv + j);
-            const double a = p.alpha[tok * p.Hv + h];
-            const double be = p.beta[tok * p.Hv + h];
+            double a = p.alpha[tok * p.Hv + h];
+            double be = p.beta[tok * p.Hv + h];
+            if (p.flags & 1) {
+                a = alpha_of(a);
+                be = beta_of(be);
+            }
+            if (p.flags & 2) {
+                l2_normalise(kv);
+                l2_normalise(qv);
+            }
 
             // P = I - beta k k^T
             for (int64_t r = 0; r < dk; ++r)
@@ -160,7 +183,9 @@ void solve_request(const Problem& p, int64_t b, float* states, float* outs) {
 
 extern "C" {
 
-// One decode call.  pool: [num_slots][Hv][dk][dv] fp32, updated in place.
+// One decode call, with the optional fused prologue (flags: 1 = alpha/beta hold
+// raw x, y; 2 = L2-normalise q and k).  pool: [num_slots][Hv][dk][dv] fp32,
+// updated in place.
 // src_idx: [B]; dst_idx: [B][T]; q, k: [B][T][Hk][dk]; v: [B][T][Hv][dv]
 // (dtype 0 = fp32, 1 = bf16 bit patterns); alpha, beta: [B][T][Hv] fp32;
 // out: [B][T][Hv][dv] fp32.  All buffers are host memory owned by the caller.
@@ -168,16 +193,16 @@ extern "C" {
 // writes then go out in (b, t) order.  nthreads <= 1 runs single-threaded.
 // Returns the number of requests skipped for an out-of-range index (padding
 // requests are not counted), or -1 for invalid sizes.
-int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* src_idx,
-                               const int32_t* dst_idx, const void* q, const void* k,
-                               const void* v, const float* alpha, const float* beta, float* out,
-                               int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
-                               int64_t dv, int32_t dtype, int32_t nthreads) {
+int64_t oracle_gdn_decode_step_fused(float* pool, int64_t num_slots, const int32_t* src_idx,
+                                     const int32_t* dst_idx, const void* q, const void* k,
+                                     const void* v, const float* alpha, const float* beta, float* out,
+                                     int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
+                                     int64_t dv, int32_t dtype, int32_t flags, int32_t nthreads) {
     if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return -1;
-    if (Hv % Hk != 0 || (dtype != 0 && dtype != 1)) return -1;
+    if (Hv % Hk != 0 || (dtype != 0 && dtype != 1) || (flags & ~3) != 0) return -1;
     if (B == 0) return 0;
 
-    Problem p{pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, B, T, Hk, Hv, dk, dv, dtype};
+    Problem p{pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, B, T, Hk, Hv, dk, dv, dtype, flags};
     const int64_t state_elems = T * Hv * dk * dv;
     const int64_t out_elems = T * Hv * dv;
     std::vector<float> states(static_cast<size_t>(B * state_elems));
@@ -218,6 +243,16 @@ int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* sr
         }
     }
     return skipped;
+}
+
+// The plain call: alpha and beta given, q and k used as they are.
+int64_t oracle_gdn_decode_step(float* pool, int64_t num_slots, const int32_t* src_idx,
+                               const int32_t* dst_idx, const void* q, const void* k,
+                               const void* v, const float* alpha, const float* beta, float* out,
+                               int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
+                               int64_t dv, int32_t dtype, int32_t nthreads) {
+    return oracle_gdn_decode_step_fused(pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, out,
+                                        B, T, Hk, Hv, dk, dv, dtype, 0, nthreads);
 }
 
 // Precondition check of one decode call's slot indices, by brute force over

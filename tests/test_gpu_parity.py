@@ -439,3 +439,66 @@ def test_cuda_graph_replay_of_padded_batches(torch_cuda):
         pad1 = np.setdiff1d(np.arange(Bmax), rows1)
         pad2 = np.setdiff1d(np.arange(Bmax), rows2)
         assert np.all(o1[pad1] == -7.0) and np.all(o2[pad2] == -7.0)
+
+
+FUSED_SHAPES = [
+    # (B, T, Hk, Hv, dk, dv, dtype)
+    (16, 1, 16, 32, 128, 128, wl.BF16),   # single-token register tiles
+    (6, 3, 2, 4, 128, 128, wl.BF16),      # multi-token register tiles
+    (5, 1, 2, 2, 64, 64, wl.F32),
+    (3, 2, 1, 2, 33, 72, wl.BF16),        # column kernel
+]
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3], ids=["gates", "qknorm", "both"])
+@pytest.mark.parametrize("shape", FUSED_SHAPES, ids=lambda s: "B{}T{}Hk{}Hv{}dk{}dv{}{}".format(*s))
+def test_fused_prologue_matches_oracle(torch_cuda, shape, flags):
+    """gdn_decode_step_fused: raw gate pre-activations and/or unnormalised q, k enter the kernel."""
+    torch = torch_cuda
+    import oracle
+    from hybrid_linear_attention_step_b200 import gdn
+
+    B, T, Hk, Hv, dk, dv, dtype = shape
+    rng = np.random.default_rng(zlib.crc32(repr((shape, flags)).encode()))
+    num_slots = B * (T + 1) + 2
+    pool = wl.init_pool(rng, num_slots, Hv, dk, dv)
+    qr, kr, v, x, y = wl.random_raw_step_inputs(rng, B, T, Hk, Hv, dk, dv, dtype)
+    qn, kn, _, alpha, beta = wl.random_step_inputs(rng, B, T, Hk, Hv, dk, dv, dtype)
+    q, k = (qr, kr) if flags & gdn.GDN_FUSE_QK_NORM else (qn, kn)
+    g1, g2 = (x, y) if flags & gdn.GDN_FUSE_GATES else (alpha, beta)
+    perm = rng.permutation(num_slots).astype(np.int32)
+    src = perm[:B].copy()
+    dst = perm[B:B + B * T].reshape(B, T).copy()
+    s = wl.Step(q, k, v, g1, g2, src, dst)
+    dev = to_torch(pool)
+    xd = step_to_device(s)
+    out = torch.full((B, T, Hv, dv), -7.0, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gdn.gdn_decode_step_fused(dev, xd["src"], xd["dst"], xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out,
+                              flags, err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    ref_pool, ref_out = pool.copy(), np.zeros((B, T, Hv, dv), np.float32)
+    oracle.decode_step(ref_pool, src, dst, q, k, v, g1, g2, ref_out, flags=flags, nthreads=8)
+    check_pool(dev.cpu().numpy(), ref_pool, pool, dst)
+    assert rel_err(out.cpu().numpy(), ref_out) <= _tol_out(s)
+
+
+def test_fused_without_flags_equals_plain_bitwise(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    w = wl.decode_b16()
+    s = w.steps[0]
+    xd = step_to_device(s)
+    outs, pools = [], []
+    for fused in (False, True):
+        dev = to_torch(w.pool)
+        out = torch.zeros((s.B, 1, s.Hv, s.dv), device="cuda")
+        args = (dev, xd["src"], xd["dst"], xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out)
+        gdn.gdn_decode_step_fused(*args, 0) if fused else gdn.gdn_decode_step(*args)
+        torch.cuda.synchronize()
+        outs.append(out.cpu().numpy())
+        pools.append(dev.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(pools[0].view(np.uint32), pools[1].view(np.uint32))
+    with pytest.raises(gdn.GdnError):
+        gdn.gdn_decode_step_fused(*args, 4)

@@ -24,6 +24,11 @@ MUTANTS = {
     "carry_unrounded": ("S[j * dk + i] = static_cast<double>(Sf[j * dk + i]);", "S[j * dk + i] = s_new;"),
     "commit_first_token": ("cur[b * T + (a - 1)]", "cur[b * T]"),
     "skip_check_dropped": ("if (d < 0 || d >= p.num_slots) return false;", "(void)d;"),
+    "fused_beta_sign": ("double beta_of(double y) { return 1.0 / (1.0 + std::exp(-y)); }",
+                        "double beta_of(double y) { return 1.0 / (1.0 + std::exp(y)); }"),
+    "fused_alpha_softplus_sign": ("double alpha_of(double x) { return std::exp(-softplus(x)); }",
+                                  "double alpha_of(double x) { return std::exp(-softplus(-x)); }"),
+    "fused_norm_without_sqrt": ("const double n = std::sqrt(ss + 1e-6);", "const double n = ss + 1e-6;"),
     "check_in_place_for_all_T": ("if (w != b || T > 1) return 5;", "if (w != b) return 5;"),
     "check_ignores_padding_flag": ("auto live = [&](int64_t b) { return src_idx[b] != -1; };",
                                    "auto live = [&](int64_t b) { return b >= 0; };"),

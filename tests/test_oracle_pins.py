@@ -449,3 +449,62 @@ def test_check_step_named_cases():
     assert ok([-1, 2], [[2, 2], [4, 5]]) == 0   # padding rows are ignored
     assert ok([1, 2], [[3], [10]]) == 3         # out of range
     assert ok([1, 2], [[2], [10]]) == 3         # index error takes precedence over aliasing
+
+
+# ------------------------------------------------------- fused prologue
+
+def _run_fused(pool, src, dst, q, k, v, x, y, flags):
+    pool = pool.copy()
+    B, T = q.shape[0], q.shape[1]
+    out = np.zeros((B, T, v.shape[2], v.shape[3]), np.float32)
+    oracle.decode_step(pool, np.asarray(src, np.int32), np.asarray(dst, np.int32).reshape(B, T), q, k, v,
+                       x, y, out, flags=flags)
+    return pool, out
+
+
+@pytest.mark.parametrize("x,alpha", [(0.0, 0.5), (np.log(3.0), 0.25), (-50.0, 1.0), (50.0, 0.0)])
+@pytest.mark.parametrize("y,beta", [(0.0, 0.5), (np.log(3.0), 0.75), (50.0, 1.0), (-50.0, 0.0)])
+def test_fused_gates_closed_forms(x, alpha, y, beta):
+    """exp(-softplus(0)) = 1/2, exp(-softplus(ln 3)) = 1/4, sigmoid(ln 3) = 3/4, and the saturated ends."""
+    rng = np.random.default_rng(40)
+    pool = wl.init_pool(rng, 3, 2, 16, 16)
+    q, k, v, _, _ = _inputs(rng, 1, 2, 1, 2, 16, 16)
+    fused, of = _run_fused(pool, [0], [[1, 2]], q, k, v, _full((1, 2, 2), x), _full((1, 2, 2), y), oracle.FUSE_GATES)
+    plain, op, _ = _run(pool, [0], [[1, 2]], q, k, v, _full((1, 2, 2), alpha), _full((1, 2, 2), beta))
+    np.testing.assert_allclose(fused, plain, rtol=2e-6, atol=1e-9)
+    np.testing.assert_allclose(of, op, rtol=2e-6, atol=1e-7)
+
+
+def test_fused_norm_is_scale_invariant():
+    """Normalising inside the step makes the result independent of the scale of q and k, and
+    leaves already-unit q and k unchanged (to the 1e-6 epsilon)."""
+    rng = np.random.default_rng(41)
+    pool = wl.init_pool(rng, 4, 4, 16, 16)
+    q, k, v, x, y = wl.random_raw_step_inputs(rng, 2, 1, 2, 4, 16, 16, wl.F32)
+    src, dst = [0, 1], [[2], [3]]
+    a_, oa = _run_fused(pool, src, dst, q, k, v, x, y, oracle.FUSE_GATES | oracle.FUSE_QK_NORM)
+    b_, ob = _run_fused(pool, src, dst, (q * 7.0).astype(np.float32), (k * 0.3).astype(np.float32), v, x, y,
+                        oracle.FUSE_GATES | oracle.FUSE_QK_NORM)
+    np.testing.assert_allclose(a_, b_, rtol=2e-5, atol=1e-8)
+    np.testing.assert_allclose(oa, ob, rtol=2e-5, atol=1e-6)
+    # unit q and k (normalised in double, rounded to fp32), gates given directly
+    qn = (q / np.linalg.norm(q.astype(np.float64), axis=-1, keepdims=True)).astype(np.float32)
+    kn = (k / np.linalg.norm(k.astype(np.float64), axis=-1, keepdims=True)).astype(np.float32)
+    alpha, beta = _full((2, 1, 4), 0.75), _full((2, 1, 4), 0.5)
+    c_, oc = _run_fused(pool, src, dst, qn, kn, v, alpha, beta, oracle.FUSE_QK_NORM)
+    d_, od, _ = _run(pool, src, dst, qn, kn, v, alpha, beta)
+    np.testing.assert_allclose(c_, d_, rtol=1e-5, atol=1e-6 * float(np.abs(d_).max()))
+    np.testing.assert_allclose(oc, od, rtol=1e-5, atol=1e-7)
+
+
+def test_fused_norm_retrieval_of_unnormalised_key():
+    """Raw k = (3, 4, 0, ...), saturated gates (alpha = 1, beta = 1): S' (k / 5) = v."""
+    rng = np.random.default_rng(42)
+    dk, dv = 16, 16
+    pool = wl.init_pool(rng, 2, 1, dk, dv)
+    q, _, v, _, _ = _inputs(rng, 1, 1, 1, 1, dk, dv)
+    k = np.zeros((1, 1, 1, dk), np.float32)
+    k[0, 0, 0, :2] = (3.0, 4.0)
+    new, _ = _run_fused(pool, [0], [[1]], q, k, v, _full((1, 1, 1), -60.0), _full((1, 1, 1), 60.0), 3)
+    got = new[1, 0].astype(np.float64).T @ (k[0, 0, 0].astype(np.float64) / 5.0)
+    np.testing.assert_allclose(got, v[0, 0, 0].astype(np.float64), rtol=0, atol=2e-6 * np.abs(v).max())
