@@ -1235,6 +1235,7 @@ extern "C" const char* gdn_status_string(int32_t status) {
         case GDN_ERR_INDEX: return "GDN_ERR_INDEX";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
         case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS";
+        case GDN_ERR_CAPACITY: return "GDN_ERR_CAPACITY";
         default: return "GDN_UNKNOWN_STATUS";
     }
 }

@@ -64,7 +64,8 @@ typedef enum gdn_status {
     GDN_ERR_CUDA = 2,        /* a CUDA runtime call or launch failed */
     GDN_ERR_INDEX = 3,       /* device-side: a slot index or accept length was out of range */
     GDN_ERR_TIMEOUT = 4,     /* device-side: a bounded wait gave up */
-    GDN_ERR_ALIAS = 5        /* device-side (gdn_check_step): the slot indices break a precondition */
+    GDN_ERR_ALIAS = 5,       /* device-side (gdn_check_step): the slot indices break a precondition */
+    GDN_ERR_CAPACITY = 6     /* host-side (gdn_slot_cache_*): no free slot and nothing evictable, or out of memory */
 } gdn_status;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;

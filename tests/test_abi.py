@@ -21,7 +21,8 @@ def declared_functions():
     names = []
     for h in sorted((ROOT / "include").glob("*.h")):
         text = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
-        names += re.findall(r"^\s*(?:gdn_status|const\s+char\s*\*)\s*(gdn_\w+)\s*\(", text, flags=re.M)
+        names += re.findall(r"^\s*(?:gdn_status|const\s+char\s*\*|void|int32_t)\s*(gdn_\w+)\s*\(", text,
+                            flags=re.M)
     return names
 
 
@@ -39,8 +40,9 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings(lib):
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_status_string.argtypes = [ctypes.c_int32]
-    assert [lib.gdn_status_string(i).decode() for i in range(6)] == [
-        "GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_CUDA", "GDN_ERR_INDEX", "GDN_ERR_TIMEOUT", "GDN_ERR_ALIAS"]
+    assert [lib.gdn_status_string(i).decode() for i in range(7)] == [
+        "GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_CUDA", "GDN_ERR_INDEX", "GDN_ERR_TIMEOUT", "GDN_ERR_ALIAS",
+        "GDN_ERR_CAPACITY"]
     assert lib.gdn_status_string(99).decode() == "GDN_UNKNOWN_STATUS"
 
 
