@@ -28,3 +28,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Build the CUDA library and the CPU oracle when missing or older than their sources
+    (nvcc cross-compiles without a GPU).  Nothing falls back if a build fails: the build
+    error ends the session."""
+    from hybrid_linear_attention_step_b200 import build
+
+    import oracle
+
+    build.build()
+    oracle.build()
+    yield
