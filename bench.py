@@ -526,6 +526,59 @@ def run_workload(args):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args):
+    """Times gdn_prefill on a long-prompt batch: B requests x L tokens, Hk=16, Hv=32,
+    dk=dv=128, bf16 inputs; only the final states are stored (checkpoints)."""
+    import numpy as np
+    import torch
+
+    from hybrid_linear_attention_step_b200 import gdn, workloads as wl
+
+    torch.cuda.set_device(0)
+    B, L, Hk, Hv, dk, dv = args.prefill_batch, args.prefill_len, 16, 32, 128, 128
+    rng = np.random.default_rng(6)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, dk, dv, wl.BF16)
+    bf = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    xq, xk, xv = bf(q), bf(k), bf(v)
+    xa, xb = torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()
+    pool = torch.empty((2 * B, Hv, dk, dv), dtype=torch.float32, device="cuda")
+    wl.fill_pool_device(pool, 6, 0)
+    src = torch.arange(B, dtype=torch.int32, device="cuda")
+    dst = torch.arange(B, 2 * B, dtype=torch.int32, device="cuda")
+    out = torch.empty((B, L, Hv, dv), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    call = lambda: gdn.gdn_prefill(pool, src, dst, xq, xk, xv, xa, xb, out, err_word=err)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0")
+    sampler.start()
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark(w0, time.time())
+    clocks = sampler.stop()
+    if gdn.gdn_get_error(err) != 0:
+        raise RuntimeError("device error word set during the prefill benchmark")
+    us = 1e3 * e0.elapsed_time(e1) / args.steps
+    units = B * L * Hv
+    flops = 7.0 * dk * dv * units  # per element: 2 FMA (u, w) + 1 FMA + 1 multiply (update)
+    sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # fp32 FMA lanes x 2 flop x median clock
+    line = {"metric": METRIC, "workload": f"prefill B={B} L={L} Hk={Hk} Hv={Hv} dk=dv={dk}", "unit": UNIT,
+            "value": units / (us / 1e6), "us_per_call": us, "steps": args.steps, "warmup": args.warmup,
+            "roofline": {"bound": "alu", "achieved": flops / us / 1e6, "peak": peak_tflops, "unit": "TFLOP/s",
+                         "frac": flops / us / 1e6 / peak_tflops,
+                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 flop x median SM clock"},
+            "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def run_ours(args):
@@ -677,8 +730,11 @@ def main():
     ap.add_argument("--batch", type=int, default=256)
     ap.add_argument("--variant", choices=["auto", "stream", "tile", "column"], default="auto",
                     help="kernel for the decode calls (auto = what gdn_decode_step picks)")
-    ap.add_argument("--workload", choices=["large", "decode_b16", "prefix_cow", "speculative"], default="large",
+    ap.add_argument("--workload", choices=["large", "decode_b16", "prefix_cow", "speculative", "prefill"],
+                    default="large",
                     help="large = the headline 8-layer decode; the others time one call of that workload")
+    ap.add_argument("--prefill-batch", type=int, default=4)
+    ap.add_argument("--prefill-len", type=int, default=2048)
     ap.add_argument("--graph", action="store_true", help="replay the timed calls from a CUDA graph "
                     "(smaller workloads only)")
     ap.add_argument("--fused", action="store_true", help="large workload through gdn_decode_step_fused: raw "
@@ -690,6 +746,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "prefill":
+        run_prefill(args)
     elif args.workload != "large":
         run_workload(args)
     else:

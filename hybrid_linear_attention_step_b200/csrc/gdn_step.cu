@@ -52,7 +52,8 @@ struct StepArgs {
     float* out;
     int32_t* err;
     int num_slots, B, T, Hk, Hv, dk, dv, G;
-    int flags;  // GDN_FUSE_* bits (gdn_decode_step_fused); 0 for plain calls
+    int flags;    // GDN_FUSE_* bits (gdn_decode_step_fused); 0 for plain calls
+    int prefill;  // 1 (gdn_prefill): dst_idx is [B], only the state after the last token is stored
 };
 
 // Fused prologue (gdn_decode_step_fused).  alpha = exp(-softplus(x)) equals
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     const int T = MULTI ? a.T : 1;
 
     int src, dst0 = 0;
-    const int status = request_status(a, b, T, src, dst0);
+    const int status = request_status(a, b, a.prefill ? 1 : T, src, dst0);
     if (status != kRun) {
         if (status == kBad && tid == 0) record_error(a.err, GDN_ERR_INDEX);
         return;
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
             ax = raw ? alpha_from_raw(x) : x;
             bx = raw ? beta_from_raw(y) : y;
-            dx = t == 0 ? dst0 : __ldg(a.dst_idx + tok);
+            dx = (t == 0 || a.prefill) ? dst0 : __ldg(a.dst_idx + tok);
         }
     };
     // The destination slot goes through shared memory as well: re-reading it
@@ -513,6 +514,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             c = make_float4(__fmul_rn(c.x, rk), __fmul_rn(c.y, rk), __fmul_rn(c.z, rk), __fmul_rn(c.w, rk));
         const int dst = dst_s[cb];
         float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst * a.Hv + h) * (DK * DV)) + toff;
+        const bool store = !a.prefill || t == T - 1;  // prefill keeps intermediate states on chip
 #pragma unroll
         for (int m = 0; m < RPT; ++m) {
             const float ki = ks[cb][m * RG + rg];
@@ -520,7 +522,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             s[m].y = fmaf(ki, c.y, __fmul_rn(al, s[m].y));
             s[m].z = fmaf(ki, c.z, __fmul_rn(al, s[m].z));
             s[m].w = fmaf(ki, c.w, __fmul_rn(al, s[m].w));
-            __stcs(D + m * kRowStep, s[m]);
+            if (store) __stcs(D + m * kRowStep, s[m]);
         }
         if (MULTI && t + 1 < T) {
             // The other buffer was last read during token t-1, before this token's barrier.
@@ -551,7 +553,7 @@ __global__ void gdn_column_kernel(StepArgs a) {
     const size_t tile = (size_t)a.dk * a.dv;
 
     int src, dst0 = 0;
-    const int status = request_status(a, b, a.T, src, dst0);
+    const int status = request_status(a, b, a.prefill ? 1 : a.T, src, dst0);
     if (status != kRun) {
         if (status == kBad && threadIdx.x == 0) record_error(a.err, GDN_ERR_INDEX);
         return;
@@ -568,7 +570,9 @@ __global__ void gdn_column_kernel(StepArgs a) {
         }
         __syncthreads();
 
-        const int dst = __ldg(a.dst_idx + tok);
+        // Prefill works in its destination slot: token 0 reads the source and
+        // every token writes the destination, which the next token reads back.
+        const int dst = a.prefill ? dst0 : __ldg(a.dst_idx + tok);
         float* D = a.pool + ((size_t)dst * a.Hv + h) * tile;
         if (active) {
             float u = 0.f, w = 0.f, kq = 0.f, kk = 0.f, qq = 0.f;
@@ -1102,7 +1106,7 @@ extern "C" gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, co
     if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out) return GDN_ERR_INVALID_ARG;
 
     const StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word,
-                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk, 0};
+                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk, 0, 0};
     return launch(a, qkv_dtype, variant, stream);
 }
 
@@ -1121,7 +1125,7 @@ extern "C" gdn_status gdn_decode_step_fused(float* pool, int32_t num_slots, cons
     if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha_or_x || !beta_or_y || !out)
         return GDN_ERR_INVALID_ARG;
     const StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha_or_x, beta_or_y, out, err_word,
-                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk, flags};
+                     num_slots, B, T, Hk, Hv, dk, dv, Hv / Hk, flags, 0};
     return launch(a, qkv_dtype, GDN_VARIANT_AUTO, stream);
 }
 
@@ -1132,6 +1136,21 @@ extern "C" gdn_status gdn_decode_step(float* pool, int32_t num_slots, const int3
                                       int32_t* err_word, cudaStream_t stream) {
     return gdn_decode_step_variant(pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, out, B, T, Hk, Hv, dk,
                                    dv, qkv_dtype, err_word, GDN_VARIANT_AUTO, stream);
+}
+
+extern "C" gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, const int32_t* dst_idx,
+                                  const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                                  float* out, int32_t B, int32_t L, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                                  int32_t qkv_dtype, int32_t* err_word, cudaStream_t stream) {
+    if (B < 0 || L < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return GDN_ERR_INVALID_ARG;
+    if (Hv % Hk != 0 || dk > kMaxDk) return GDN_ERR_INVALID_ARG;
+    if (qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)B * Hv * 4 >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out) return GDN_ERR_INVALID_ARG;
+    const StepArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word,
+                     num_slots, B, L, Hk, Hv, dk, dv, Hv / Hk, 0, 1};
+    return launch(a, qkv_dtype, GDN_VARIANT_AUTO, stream);
 }
 
 extern "C" gdn_status gdn_commit(const int32_t* accept_len, int32_t* committed, const int32_t* cur, int32_t B,

@@ -67,6 +67,8 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_decode_step_fused.restype = i32
     lib.gdn_decode_step_fused.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                           i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    lib.gdn_prefill.restype = i32
+    lib.gdn_prefill.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.gdn_commit.restype = i32
     lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
     lib.gdn_check_step.restype = i32
@@ -163,6 +165,22 @@ def gdn_decode_step_fused(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: to
                                                   _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_decode_step_fused")
+    return status
+
+
+def gdn_prefill(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
+                q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
+                err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """Enqueue a prefill (see gdn_prefill in include/gdn_step.h): q, k [B, L, Hk, dk],
+    v [B, L, Hv, dv], alpha/beta [B, L, Hv], out [B, L, Hv, dv]; only the state after the
+    last token is stored, to pool[dst_idx[b]] (dst_idx [B])."""
+    if dst_idx.numel() != src_idx.numel():
+        raise ValueError("dst_idx must hold one slot per request")
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+    status = load_library().gdn_prefill(*args, _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_prefill")
     return status
 
 

@@ -174,6 +174,29 @@ gdn_status gdn_decode_step_fused(float* pool, int32_t num_slots, const int32_t* 
                                  int32_t flags, int32_t* err_word, cudaStream_t stream);
 
 /*
+ * gdn_prefill -- feed L tokens per request and store only the final state: the
+ * checkpoint of the prefix.
+ *
+ * The pages checkpoint the recurrent state of a prefix next to its KV pages so that
+ * later requests reuse it (zubnet.ai article, second paragraph; 24-ai.news article,
+ * "Hybrid prefix caching for GDN/Mamba").  This call produces such a checkpoint:
+ * for each request b it applies the same per-token update as gdn_decode_step with
+ * T = L, starting from pool[src_idx[b]], writes o for every token to
+ * out[b][t][h][:], and stores only the state after token L-1, to
+ * pool[dst_idx[b]][h].  The intermediate states stay on chip (or, in the column
+ * kernel, in the destination slot).  dst may equal src (continue a sequence in place).
+ *
+ *   Same arguments and layouts as gdn_decode_step with T = L, except dst_idx: int32 [B].
+ *   Preconditions: destinations distinct; no destination equals another request's
+ *   source.  Padding (src GDN_SLOT_NONE), index errors and the error word behave as in
+ *   gdn_decode_step.  A fresh sequence starts from a slot the caller zero-filled.
+ */
+gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, const int32_t* dst_idx,
+                       const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                       float* out, int32_t B, int32_t L, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                       int32_t qkv_dtype, int32_t* err_word, cudaStream_t stream);
+
+/*
  * gdn_commit -- accept speculative draft tokens by rewriting an int32 index table.
  *
  * Defined by the O(1) index update that replaces an O(L*D) state copy (24-ai.news

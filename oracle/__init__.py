@@ -69,6 +69,9 @@ def _load():
         lib.oracle_gdn_decode_step_fused.restype = i64
         lib.oracle_gdn_decode_step_fused.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
                                                      i64, i64, i64, i64, i64, i64, i32, i32, i32]
+        lib.oracle_gdn_prefill.restype = i64
+        lib.oracle_gdn_prefill.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           i64, i64, i64, i64, i64, i64, i32, i32]
         lib.oracle_gdn_check_step.restype = i32
         lib.oracle_gdn_check_step.argtypes = [vp, vp, i64, i64, i64]
         lib.oracle_gdn_commit.restype = i64
@@ -170,6 +173,31 @@ def check_step(src_idx, dst_idx, num_slots: int) -> int:
     if dst_idx.size != B * T:
         raise ValueError("dst_idx must hold B*T entries")
     r = _load().oracle_gdn_check_step(_ptr(src_idx), _ptr(dst_idx), B, T, int(num_slots))
+    if r < 0:
+        raise ValueError("oracle rejected the sizes")
+    return int(r)
+
+
+def prefill(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, *, nthreads: int = 1) -> int:
+    """Prefill on host arrays: L tokens per request (q [B, L, Hk, dk] ...), only the final
+    state stored, to dst_idx[b] (dst_idx [B]); ``out`` [B, L, Hv, dv] gets every token."""
+    _need(pool, np.float32, "pool")
+    num_slots, Hv, dk, dv = pool.shape
+    _need(src_idx, np.int32, "src_idx")
+    _need(dst_idx, np.int32, "dst_idx")
+    B, L, Hk = q.shape[0], q.shape[1], q.shape[2]
+    if src_idx.shape != (B,) or dst_idx.size != B:
+        raise ValueError("src_idx and dst_idx must hold B entries")
+    dtype = BF16 if q.dtype == np.uint16 else F32
+    for name, a in (("q", q), ("k", k), ("v", v)):
+        _need(a, q.dtype, name)
+    for name, a in (("alpha", alpha), ("beta", beta), ("out", out)):
+        _need(a, np.float32, name)
+    if k.shape != (B, L, Hk, dk) or v.shape != (B, L, Hv, dv) or alpha.shape != (B, L, Hv) or \
+            beta.shape != (B, L, Hv) or out.shape != (B, L, Hv, dv):
+        raise ValueError("shapes must follow q [B, L, Hk, dk]")
+    r = _load().oracle_gdn_prefill(_ptr(pool), num_slots, _ptr(src_idx), _ptr(dst_idx), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(alpha), _ptr(beta), _ptr(out), B, L, Hk, Hv, dk, dv, dtype, int(nthreads))
     if r < 0:
         raise ValueError("oracle rejected the sizes")
     return int(r)

@@ -75,6 +75,7 @@ struct Problem {
     int64_t B, T, Hk, Hv, dk, dv;
     int32_t dtype;
     int32_t flags;  // 1: alpha/beta are raw x, y; 2: L2-normalise q and k
+    bool last_only; // prefill: dst_idx is [B]; only the state after the last token is kept
 };
 
 // Fused prologue, from its definition: alpha = exp(-softplus(x)) with
@@ -97,8 +98,9 @@ bool request_is_padding(const Problem& p, int64_t b) { return p.src_idx[b] == -1
 bool request_is_valid(const Problem& p, int64_t b) {
     const int64_t s = p.src_idx[b];
     if (s < 0 || s >= p.num_slots) return false;
-    for (int64_t t = 0; t < p.T; ++t) {
-        const int64_t d = p.dst_idx[b * p.T + t];
+    const int64_t nd = p.last_only ? 1 : p.T;
+    for (int64_t t = 0; t < nd; ++t) {
+        const int64_t d = p.dst_idx[b * nd + t];
         if (d < 0 || d >= p.num_slots) return false;
     }
     return true;
@@ -163,10 +165,12 @@ void solve_request(const Problem& p, int64_t b, float* states, float* outs) {
                     S[j * dk + i] = static_cast<double>(Sf[j * dk + i]);
                 }
 
-            // Stored layout of token t, head h: [dk][dv].
-            float* St = states + ((t * p.Hv + h) * dk) * dv;
-            for (int64_t i = 0; i < dk; ++i)
-                for (int64_t j = 0; j < dv; ++j) St[i * dv + j] = Sf[j * dk + i];
+            // Stored layout of token t, head h: [dk][dv] (prefill keeps the last token only).
+            if (!p.last_only || t == p.T - 1) {
+                float* St = states + (((p.last_only ? 0 : t) * p.Hv + h) * dk) * dv;
+                for (int64_t i = 0; i < dk; ++i)
+                    for (int64_t j = 0; j < dv; ++j) St[i * dv + j] = Sf[j * dk + i];
+            }
 
             // o = S' q from the fp32-rounded S'.
             float* ot = outs + (t * p.Hv + h) * dv;
@@ -193,17 +197,22 @@ extern "C" {
 // writes then go out in (b, t) order.  nthreads <= 1 runs single-threaded.
 // Returns the number of requests skipped for an out-of-range index (padding
 // requests are not counted), or -1 for invalid sizes.
-int64_t oracle_gdn_decode_step_fused(float* pool, int64_t num_slots, const int32_t* src_idx,
-                                     const int32_t* dst_idx, const void* q, const void* k,
-                                     const void* v, const float* alpha, const float* beta, float* out,
-                                     int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
-                                     int64_t dv, int32_t dtype, int32_t flags, int32_t nthreads) {
+}  // extern "C"
+
+namespace {
+
+int64_t run_calls(float* pool, int64_t num_slots, const int32_t* src_idx, const int32_t* dst_idx, const void* q,
+                  const void* k, const void* v, const float* alpha, const float* beta, float* out, int64_t B,
+                  int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv, int32_t dtype, int32_t flags,
+                  bool last_only, int32_t nthreads) {
     if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return -1;
     if (Hv % Hk != 0 || (dtype != 0 && dtype != 1) || (flags & ~3) != 0) return -1;
     if (B == 0) return 0;
 
-    Problem p{pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, B, T, Hk, Hv, dk, dv, dtype, flags};
-    const int64_t state_elems = T * Hv * dk * dv;
+    Problem p{pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, B, T, Hk, Hv, dk, dv, dtype, flags,
+              last_only};
+    const int64_t kept = last_only ? 1 : T;  // states kept per request
+    const int64_t state_elems = kept * Hv * dk * dv;
     const int64_t out_elems = T * Hv * dv;
     std::vector<float> states(static_cast<size_t>(B * state_elems));
     std::vector<float> outs(static_cast<size_t>(B * out_elems));
@@ -234,15 +243,42 @@ int64_t oracle_gdn_decode_step_fused(float* pool, int64_t num_slots, const int32
             continue;
         }
         for (int64_t t = 0; t < T; ++t) {
-            const int64_t d = dst_idx[b * T + t];
-            for (int64_t h = 0; h < Hv; ++h)
-                std::memcpy(pool + (d * Hv + h) * tile, &states[b * state_elems + (t * Hv + h) * tile],
-                            sizeof(float) * tile);
+            if (!last_only || t == T - 1) {
+                const int64_t d = last_only ? dst_idx[b] : dst_idx[b * T + t];
+                const int64_t ts = last_only ? 0 : t;
+                for (int64_t h = 0; h < Hv; ++h)
+                    std::memcpy(pool + (d * Hv + h) * tile, &states[b * state_elems + (ts * Hv + h) * tile],
+                                sizeof(float) * tile);
+            }
             std::memcpy(out + (b * T + t) * Hv * dv, &outs[b * out_elems + t * Hv * dv],
                         sizeof(float) * Hv * dv);
         }
     }
     return skipped;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t oracle_gdn_decode_step_fused(float* pool, int64_t num_slots, const int32_t* src_idx,
+                                     const int32_t* dst_idx, const void* q, const void* k,
+                                     const void* v, const float* alpha, const float* beta, float* out,
+                                     int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk,
+                                     int64_t dv, int32_t dtype, int32_t flags, int32_t nthreads) {
+    return run_calls(pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, out, B, T, Hk, Hv, dk, dv, dtype,
+                     flags, false, nthreads);
+}
+
+// Prefill: the same per-token update over T = L tokens, keeping only the state
+// after the last token (written to dst_idx[b], dst_idx is [B]); every token's
+// output is written.  Returns skipped requests as above.
+int64_t oracle_gdn_prefill(float* pool, int64_t num_slots, const int32_t* src_idx, const int32_t* dst_idx,
+                           const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                           float* out, int64_t B, int64_t L, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                           int32_t dtype, int32_t nthreads) {
+    return run_calls(pool, num_slots, src_idx, dst_idx, q, k, v, alpha, beta, out, B, L, Hk, Hv, dk, dv, dtype, 0,
+                     true, nthreads);
 }
 
 // The plain call: alpha and beta given, q and k used as they are.

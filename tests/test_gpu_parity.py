@@ -502,3 +502,88 @@ def test_fused_without_flags_equals_plain_bitwise(torch_cuda):
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(pools[0].view(np.uint32), pools[1].view(np.uint32))
     with pytest.raises(gdn.GdnError):
         gdn.gdn_decode_step_fused(*args, 4)
+
+
+PREFILL_SHAPES = [
+    # (B, L, Hk, Hv, dk, dv, dtype, in_place)
+    (4, 1, 2, 4, 128, 128, wl.BF16, False),
+    (3, 7, 2, 4, 128, 128, wl.BF16, True),
+    (2, 96, 1, 2, 128, 128, wl.BF16, False),
+    (3, 33, 2, 2, 64, 64, wl.F32, True),
+    (2, 9, 1, 2, 40, 24, wl.BF16, False),   # column kernel
+]
+
+
+@pytest.mark.parametrize("shape", PREFILL_SHAPES, ids=lambda s: "B{}L{}Hk{}Hv{}dk{}dv{}{}{}".format(*s[:7], "ip" if s[7] else ""))
+def test_prefill_matches_oracle(torch_cuda, shape):
+    torch = torch_cuda
+    import oracle
+    from hybrid_linear_attention_step_b200 import gdn
+
+    B, L, Hk, Hv, dk, dv, dtype, in_place = shape
+    rng = np.random.default_rng(zlib.crc32(repr(shape).encode()))
+    num_slots = 2 * B + 3
+    pool = wl.init_pool(rng, num_slots, Hv, dk, dv)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, dk, dv, dtype)
+    perm = rng.permutation(num_slots).astype(np.int32)
+    src = perm[:B].copy()
+    dst = src.copy() if in_place else perm[B:2 * B].copy()
+    s = wl.Step(q, k, v, a, b, src, dst.reshape(B, 1))
+    xd = step_to_device(s)
+    dev = to_torch(pool)
+    out = torch.full((B, L, Hv, dv), -7.0, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gdn.gdn_prefill(dev, xd["src"], to_torch(dst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out,
+                    err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    ref_pool, ref_out = pool.copy(), np.zeros((B, L, Hv, dv), np.float32)
+    assert oracle.prefill(ref_pool, src, dst, q, k, v, a, b, ref_out, nthreads=8) == 0
+    check_pool(dev.cpu().numpy(), ref_pool, pool, dst)
+    assert rel_err(out.cpu().numpy(), ref_out) <= _tol_out(s)
+
+
+def test_prefill_equals_decode_last_state_bitwise(torch_cuda):
+    """On the GPU the prefill's final state is the bits a T = L decode call stores for its last token."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(44)
+    B, L, Hk, Hv = 3, 12, 2, 4
+    pool = wl.init_pool(rng, 3 * B + B * L, Hv, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, 128, 128, wl.BF16)
+    src = np.arange(B, dtype=np.int32)
+    pdst = np.arange(B, 2 * B, dtype=np.int32)
+    cur = (3 * B + np.arange(B * L, dtype=np.int32)).reshape(B, L)
+    xd = step_to_device(wl.Step(q, k, v, a, b, src, cur))
+    dev = to_torch(pool)
+    o1 = torch.zeros((B, L, Hv, 128), device="cuda")
+    o2 = torch.zeros_like(o1)
+    gdn.gdn_prefill(dev, xd["src"], to_torch(pdst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o1)
+    gdn.gdn_decode_step(dev, xd["src"], xd["dst"], xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], o2)
+    torch.cuda.synchronize()
+    got = dev.cpu().numpy()
+    assert np.array_equal(got[pdst].view(np.uint32), got[cur[:, -1]].view(np.uint32))
+    assert torch.equal(o1, o2)
+
+
+def test_prefill_padding_rows_are_silent(torch_cuda):
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(45)
+    B, L = 4, 5
+    pool = wl.init_pool(rng, 10, 4, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, 2, 4, 128, 128, wl.BF16)
+    src = np.array([0, -1, 2, -1], np.int32)
+    dst = np.array([4, 99, 5, -3], np.int32)  # padding rows' destinations are ignored
+    xd = step_to_device(wl.Step(q, k, v, a, b, src, dst.reshape(B, 1)))
+    dev = to_torch(pool)
+    out = torch.full((B, L, 4, 128), -7.0, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gdn.gdn_prefill(dev, xd["src"], to_torch(dst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out,
+                    err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    o = out.cpu().numpy()
+    assert np.all(o[[1, 3]] == -7.0) and not np.any(o[[0, 2]] == -7.0)
+    untouched = [0, 1, 2, 3, 6, 7, 8, 9]
+    assert np.array_equal(dev.cpu().numpy()[untouched].view(np.uint32), pool[untouched].view(np.uint32))

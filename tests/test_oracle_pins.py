@@ -508,3 +508,31 @@ def test_fused_norm_retrieval_of_unnormalised_key():
     new, _ = _run_fused(pool, [0], [[1]], q, k, v, _full((1, 1, 1), -60.0), _full((1, 1, 1), 60.0), 3)
     got = new[1, 0].astype(np.float64).T @ (k[0, 0, 0].astype(np.float64) / 5.0)
     np.testing.assert_allclose(got, v[0, 0, 0].astype(np.float64), rtol=0, atol=2e-6 * np.abs(v).max())
+
+
+# ------------------------------------------------------------------ prefill
+
+def test_prefill_equals_chained_single_token_calls():
+    """A prefill over L tokens ends in the state, bit for bit, that L chained single-token calls
+    reach, emits the same outputs, and writes nothing but its destination slot."""
+    rng = np.random.default_rng(43)
+    B, L, Hk, Hv, dk, dv = 2, 5, 1, 2, 16, 8
+    pool = wl.init_pool(rng, 6, Hv, dk, dv)
+    q, k, v, a, b = _inputs(rng, B, L, Hk, Hv, dk, dv, wl.BF16)
+    src = np.array([0, 1], np.int32)
+    dst = np.array([2, 1], np.int32)            # request 1 continues in place
+    pre = pool.copy()
+    out = np.zeros((B, L, Hv, dv), np.float32)
+    assert oracle.prefill(pre, src, dst, q, k, v, a, b, out) == 0
+    chain = pool.copy()
+    for bi in range(B):
+        cur = int(src[bi])
+        for t in range(L):
+            nxt = [4, 5][t % 2]                 # scratch slots
+            sl = lambda x: np.ascontiguousarray(x[bi:bi + 1, t:t + 1])
+            chain, o, _ = _run(chain, [cur], [[nxt]], sl(q), sl(k), sl(v), sl(a), sl(b))
+            assert np.array_equal(o[0, 0], out[bi, t])
+            cur = nxt
+        assert np.array_equal(pre[dst[bi]].view(np.uint32), chain[cur].view(np.uint32))
+    untouched = [0, 3, 4, 5]
+    assert np.array_equal(pre[untouched].view(np.uint32), pool[untouched].view(np.uint32))
