@@ -547,7 +547,11 @@ def run_prefill(args):
     dst = torch.arange(B, 2 * B, dtype=torch.int32, device="cuda")
     out = torch.empty((B, L, Hv, dv), dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    call = lambda: gdn.gdn_prefill(pool, src, dst, xq, xk, xv, xa, xb, out, err_word=err)
+    if args.chunked:
+        ws = torch.empty(gdn.gdn_prefill_workspace_bytes(B, L, Hv, dk, dv), dtype=torch.uint8, device="cuda")
+        call = lambda: gdn.gdn_prefill_chunked(pool, src, dst, xq, xk, xv, xa, xb, out, ws, err_word=err)
+    else:
+        call = lambda: gdn.gdn_prefill(pool, src, dst, xq, xk, xv, xa, xb, out, err_word=err)
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()
@@ -570,7 +574,8 @@ def run_prefill(args):
     flops = 7.0 * dk * dv * units  # per element: 2 FMA (u, w) + 1 FMA + 1 multiply (update)
     sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
     peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # fp32 FMA lanes x 2 flop x median clock
-    line = {"metric": METRIC, "workload": f"prefill B={B} L={L} Hk={Hk} Hv={Hv} dk=dv={dk}", "unit": UNIT,
+    line = {"metric": METRIC, "workload": f"prefill B={B} L={L} Hk={Hk} Hv={Hv} dk=dv={dk}",
+            "kernel": "chunked (gdn_prefill_chunked)" if args.chunked else "token steps (gdn_prefill)", "unit": UNIT,
             "value": units / (us / 1e6), "us_per_call": us, "steps": args.steps, "warmup": args.warmup,
             "roofline": {"bound": "alu", "achieved": flops / us / 1e6, "peak": peak_tflops, "unit": "TFLOP/s",
                          "frac": flops / us / 1e6 / peak_tflops,
@@ -735,6 +740,7 @@ def main():
                     help="large = the headline 8-layer decode; the others time one call of that workload")
     ap.add_argument("--prefill-batch", type=int, default=4)
     ap.add_argument("--prefill-len", type=int, default=2048)
+    ap.add_argument("--chunked", action="store_true", help="prefill workload through gdn_prefill_chunked")
     ap.add_argument("--graph", action="store_true", help="replay the timed calls from a CUDA graph "
                     "(smaller workloads only)")
     ap.add_argument("--fused", action="store_true", help="large workload through gdn_decode_step_fused: raw "

@@ -15,7 +15,7 @@ import subprocess
 
 PKG = pathlib.Path(__file__).resolve().parent
 ROOT = PKG.parent
-SOURCES = [PKG / "csrc" / "gdn_step.cu", PKG / "csrc" / "slot_cache.cpp"]
+SOURCES = [PKG / "csrc" / "gdn_step.cu", PKG / "csrc" / "gdn_prefill_chunked.cu", PKG / "csrc" / "slot_cache.cpp"]
 HEADERS = [ROOT / "include" / "gdn_step.h", ROOT / "include" / "gdn_slot_cache.h"]
 LIB_PATH = PKG / "libgdn_b200.so"
 

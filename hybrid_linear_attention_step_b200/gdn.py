@@ -69,6 +69,11 @@ def load_library() -> ctypes.CDLL:
                                           i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.gdn_prefill.restype = i32
     lib.gdn_prefill.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    lib.gdn_prefill_chunked.restype = i32
+    lib.gdn_prefill_chunked.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                        vp, ctypes.c_size_t, vp, vp]
+    lib.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_prefill_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     lib.gdn_commit.restype = i32
     lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
     lib.gdn_check_step.restype = i32
@@ -181,6 +186,27 @@ def gdn_prefill(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor
     status = load_library().gdn_prefill(*args, _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_prefill")
+    return status
+
+
+def gdn_prefill_workspace_bytes(B: int, L: int, Hv: int, dk: int, dv: int) -> int:
+    return int(load_library().gdn_prefill_workspace_bytes(int(B), int(L), int(Hv), int(dk), int(dv)))
+
+
+def gdn_prefill_chunked(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
+                        q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                        err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+    """gdn_prefill computed chunk by chunk (see gdn_prefill_chunked in include/gdn_step.h);
+    ``workspace`` is a CUDA tensor of at least gdn_prefill_workspace_bytes(...) bytes."""
+    if dst_idx.numel() != src_idx.numel():
+        raise ValueError("dst_idx must hold one slot per request")
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+    nbytes = workspace.numel() * workspace.element_size()
+    status = load_library().gdn_prefill_chunked(*args, _dev(workspace, "workspace"), nbytes,
+                                                _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_prefill_chunked")
     return status
 
 

@@ -51,6 +51,7 @@
 #ifndef GDN_STEP_H
 #define GDN_STEP_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -195,6 +196,32 @@ gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, c
                        const void* q, const void* k, const void* v, const float* alpha, const float* beta,
                        float* out, int32_t B, int32_t L, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
                        int32_t qkv_dtype, int32_t* err_word, cudaStream_t stream);
+
+/*
+ * gdn_prefill_chunked -- gdn_prefill computed chunk by chunk (64 tokens) with dense
+ * per-chunk contractions instead of one token step at a time.
+ *
+ * Same operation, arguments, preconditions and errors as gdn_prefill (the result
+ * equals it within fp32 rounding, not bit for bit).  Within a chunk the token
+ * dependencies reduce to a unit lower-triangular system (I + A) E = R whose inverse
+ * depends only on the chunk's keys and gates; a first kernel builds it for all
+ * chunks in parallel, a second walks each sequence's chunks in order carrying the
+ * state.  Supports dk = dv = 128.
+ *
+ *   workspace        device memory of at least gdn_prefill_workspace_bytes(B, L, Hv,
+ *                    dk, dv) bytes, 16-byte aligned, caller-owned; contents on entry
+ *                    do not matter and on return are unspecified.  Calls sharing one
+ *                    workspace must not overlap.
+ * Unsupported shapes, a missing or short workspace return GDN_ERR_INVALID_ARG.
+ */
+gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const int32_t* src_idx, const int32_t* dst_idx,
+                               const void* q, const void* k, const void* v, const float* alpha,
+                               const float* beta, float* out, int32_t B, int32_t L, int32_t Hk, int32_t Hv,
+                               int32_t dk, int32_t dv, int32_t qkv_dtype, void* workspace,
+                               size_t workspace_bytes, int32_t* err_word, cudaStream_t stream);
+
+/* Workspace bytes gdn_prefill_chunked needs for these sizes; 0 if it does not support them. */
+size_t gdn_prefill_workspace_bytes(int32_t B, int32_t L, int32_t Hv, int32_t dk, int32_t dv);
 
 /*
  * gdn_commit -- accept speculative draft tokens by rewriting an int32 index table.

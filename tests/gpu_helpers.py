@@ -44,7 +44,8 @@ def to_torch(a: np.ndarray, device="cuda"):
 def step_to_device(s: wl.Step, device="cuda"):
     return dict(q=to_torch(s.q, device), k=to_torch(s.k, device), v=to_torch(s.v, device),
                 alpha=to_torch(s.alpha, device), beta=to_torch(s.beta, device),
-                src=to_torch(s.src_idx, device), dst=to_torch(np.ascontiguousarray(s.dst_idx.reshape(s.B, s.T)), device))
+                src=to_torch(s.src_idx, device),
+                dst=to_torch(np.ascontiguousarray(s.dst_idx.reshape(s.B, -1)), device))
 
 
 def run_gpu(pool_dev, s: wl.Step, out_fill=-7.0, err=None, stream=None, variant=None):

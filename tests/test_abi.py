@@ -21,7 +21,7 @@ def declared_functions():
     names = []
     for h in sorted((ROOT / "include").glob("*.h")):
         text = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
-        names += re.findall(r"^\s*(?:gdn_status|const\s+char\s*\*|void|int32_t)\s*(gdn_\w+)\s*\(", text,
+        names += re.findall(r"^\s*(?:gdn_status|const\s+char\s*\*|void|int32_t|size_t)\s*(gdn_\w+)\s*\(", text,
                             flags=re.M)
     return names
 

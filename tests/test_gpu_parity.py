@@ -587,3 +587,76 @@ def test_prefill_padding_rows_are_silent(torch_cuda):
     assert np.all(o[[1, 3]] == -7.0) and not np.any(o[[0, 2]] == -7.0)
     untouched = [0, 1, 2, 3, 6, 7, 8, 9]
     assert np.array_equal(dev.cpu().numpy()[untouched].view(np.uint32), pool[untouched].view(np.uint32))
+
+
+CHUNKED_SHAPES = [
+    # (B, L, Hk, Hv, dtype, in_place)
+    (2, 1, 1, 2, wl.BF16, False),
+    (3, 64, 2, 4, wl.BF16, True),
+    (2, 65, 1, 2, wl.BF16, False),
+    (2, 200, 2, 2, wl.F32, False),
+    (1, 1000, 1, 2, wl.BF16, True),
+]
+
+
+@pytest.mark.parametrize("shape", CHUNKED_SHAPES, ids=lambda s: "B{}L{}Hk{}Hv{}{}{}".format(*s[:5], "ip" if s[5] else ""))
+def test_prefill_chunked_matches_oracle(torch_cuda, shape):
+    """The chunked prefill (per-chunk triangular solve + dense contractions) against the
+    token-by-token oracle, for chunk-aligned, ragged and multi-chunk lengths."""
+    torch = torch_cuda
+    import oracle
+    from hybrid_linear_attention_step_b200 import gdn
+
+    B, L, Hk, Hv, dtype, in_place = shape
+    rng = np.random.default_rng(zlib.crc32(repr(shape).encode()))
+    num_slots = 2 * B + 3
+    pool = wl.init_pool(rng, num_slots, Hv, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, 128, 128, dtype)
+    perm = rng.permutation(num_slots).astype(np.int32)
+    src = perm[:B].copy()
+    dst = src.copy() if in_place else perm[B:2 * B].copy()
+    xd = step_to_device(wl.Step(q, k, v, a, b, src, dst.reshape(B, 1)))
+    dev = to_torch(pool)
+    out = torch.full((B, L, Hv, 128), -7.0, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(gdn.gdn_prefill_workspace_bytes(B, L, Hv, 128, 128), dtype=torch.uint8, device="cuda")
+    gdn.gdn_prefill_chunked(dev, xd["src"], to_torch(dst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out,
+                            ws, err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    ref_pool, ref_out = pool.copy(), np.zeros((B, L, Hv, 128), np.float32)
+    assert oracle.prefill(ref_pool, src, dst, q, k, v, a, b, ref_out, nthreads=8) == 0
+    check_pool(dev.cpu().numpy(), ref_pool, pool, dst)
+    assert rel_err(out.cpu().numpy(), ref_out) <= TOL_OUT_BF16
+
+
+def test_prefill_chunked_edge_cases(torch_cuda):
+    """Padding rows, an out-of-range slot, a full reset (alpha = 0) and a short workspace."""
+    torch = torch_cuda
+    import oracle
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(46)
+    B, L, Hv = 4, 130, 2
+    pool = wl.init_pool(rng, 12, Hv, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, 1, Hv, 128, 128, wl.BF16)
+    a[2, 70, :] = 0.0  # request 2 forgets its history at token 70
+    src = np.array([0, -1, 2, 3], np.int32)
+    dst = np.array([4, 99, 6, 12], np.int32)  # request 3: destination out of range
+    xd = step_to_device(wl.Step(q, k, v, a, b, src, dst.reshape(B, 1)))
+    dev = to_torch(pool)
+    out = torch.full((B, L, Hv, 128), -7.0, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nbytes = gdn.gdn_prefill_workspace_bytes(B, L, Hv, 128, 128)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    with pytest.raises(gdn.GdnError):
+        gdn.gdn_prefill_chunked(dev, xd["src"], to_torch(dst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"],
+                                out, ws[: nbytes - 16], err_word=err)
+    gdn.gdn_prefill_chunked(dev, xd["src"], to_torch(dst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out,
+                            ws, err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_ERR_INDEX
+    ref_pool, ref_out = pool.copy(), np.full((B, L, Hv, 128), -7.0, np.float32)
+    assert oracle.prefill(ref_pool, src, dst, q, k, v, a, b, ref_out, nthreads=8) == 1
+    check_pool(dev.cpu().numpy(), ref_pool, pool, np.array([4, 6]))
+    o = out.cpu().numpy()
+    assert np.all(o[[1, 3]] == -7.0)
+    assert rel_err(o[[0, 2]], ref_out[[0, 2]]) <= TOL_OUT_BF16
