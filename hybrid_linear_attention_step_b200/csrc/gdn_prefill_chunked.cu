@@ -28,6 +28,15 @@
 // Ratios g_t / g_i are formed as exp(log g_t - log g_i) <= 1, so nothing
 // overflows; g_t itself may underflow to zero, which is its true value to fp32
 // precision.
+//
+// Workspace record of one (request, head, chunk), bytes, laid out as the
+// shared-memory image kernel 2 copies in (bulk copies, 16-byte granules):
+//   A1  [K; Q] as bf16, 128 rows x 128 (dk) in the no-swizzle K-major core
+//       layout of the tensor-core operand (bf16 inputs only)
+//   A2  K^T as bf16, 128 (dk) rows x 64 tokens, same layout (bf16 inputs only)
+//   U   four column slabs [4][64][36] fp32 (32 columns + 4 padding each)
+//   TP  [64][65] fp32: Tb on and below the diagonal, P^T strictly above it
+//   G   log g [64], then the diagonal of P [64]
 
 #include "gdn_step.h"
 
@@ -37,11 +46,32 @@
 
 namespace {
 
-constexpr int kC = 64;     // tokens per chunk
-constexpr int kD = 128;    // dk = dv supported here
-constexpr int kDVC = 32;   // value columns per CTA in the sequential kernel
-constexpr int kNT = 256;   // threads per CTA (both kernels)
-constexpr int kPad = 4;    // row padding of [C][D] shared arrays (bank spread)
+constexpr int kC = 64;          // tokens per chunk
+constexpr int kD = 128;         // dk = dv supported here
+constexpr int kDVC = 32;        // value columns per CTA in the sequential kernel
+constexpr int kNCB = kD / kDVC; // column blocks per (request, head)
+constexpr int kNT = 256;        // threads per CTA (both kernels)
+constexpr int kUS = kDVC + 4;   // row stride of the 64 x 32 fp32 tiles (16-byte rows, bank spread)
+constexpr int kTS = kC + 1;     // row stride of TP
+constexpr int kPad = 4;         // row padding of [C][D] shared arrays in the fp32 scan kernel
+
+// Workspace record (bytes).
+constexpr size_t kRecA1 = 0;
+constexpr size_t kRecA2 = kRecA1 + (size_t)2 * kC * kD * 2;
+constexpr size_t kRecU = kRecA2 + (size_t)kD * kC * 2;
+constexpr size_t kUSlab = (size_t)kC * kUS * 4;
+constexpr size_t kRecTP = kRecU + kNCB * kUSlab;
+constexpr size_t kRecG = kRecTP + (size_t)kC * kTS * 4;
+constexpr size_t kRecBytes = kRecG + (size_t)2 * kC * 4;
+// One CTA's image of a chunk in shared memory: A1 A2 | its U slab | TP G.
+constexpr uint32_t kBufA2 = (uint32_t)kRecA2;
+constexpr uint32_t kBufU = (uint32_t)kRecU;
+constexpr uint32_t kBufTP = kBufU + (uint32_t)kUSlab;
+constexpr uint32_t kBufG = kBufTP + (uint32_t)((size_t)kC * kTS * 4);
+constexpr uint32_t kBufBytes = kBufG + 2 * kC * 4;
+static_assert(kRecU % 16 == 0 && kRecTP % 16 == 0 && kRecG % 16 == 0 && kRecBytes % 16 == 0, "16-byte records");
+static_assert(kUSlab % 16 == 0 && kBufTP % 16 == 0 && kBufBytes % 16 == 0, "16-byte bulk copies");
+static_assert(kRecG - kRecTP == kBufG - kBufTP, "TP and G are copied together");
 
 struct ChunkArgs {
     float* pool;
@@ -53,17 +83,34 @@ struct ChunkArgs {
     const float* alpha;
     const float* beta;
     float* out;
-    float* ws;  // workspace: per (b, h, chunk) a ChunkWs record
+    unsigned char* ws;  // workspace: per (b, h, chunk) one record of kRecBytes
     int32_t* err;
     int num_slots, B, L, Hk, Hv, G, nchunks;
 };
 
-// Workspace record of one (request, head, chunk), floats.
-constexpr size_t kWsU = 0;                        // U = T diag(beta) V    [C][D]
-constexpr size_t kWsT = kWsU + (size_t)kC * kD;   // Tb = T diag(beta g)   [C][C]
-constexpr size_t kWsP = kWsT + (size_t)kC * kC;   // P                     [C][C]
-constexpr size_t kWsG = kWsP + (size_t)kC * kC;   // log g                 [C]
-constexpr size_t kWsFloats = kWsG + kC;
+__device__ __forceinline__ unsigned char* record_of(const ChunkArgs& a, int bh, int c) {
+    return a.ws + ((size_t)bh * a.nchunks + c) * kRecBytes;
+}
+
+// 8 consecutive input elements (a 16-byte aligned group for bf16, 32 bytes for fp32) as fp32.
+template <typename InT>
+__device__ __forceinline__ void ld8(const void* base, size_t idx, float (&x)[8]);
+template <>
+__device__ __forceinline__ void ld8<float>(const void* base, size_t idx, float (&x)[8]) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void ld8<__nv_bfloat16>(const void* base, size_t idx, float (&x)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        x[2 * j] = __uint_as_float(w[j] << 16);
+        x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+}
 
 template <typename InT>
 __device__ __forceinline__ float ld_in(const void* base, size_t idx);
@@ -71,13 +118,21 @@ template <>
 __device__ __forceinline__ float ld_in<float>(const void* base, size_t idx) {
     return __ldg(static_cast<const float*>(base) + idx);
 }
-template <>
-__device__ __forceinline__ float ld_in<__nv_bfloat16>(const void* base, size_t idx) {
-    return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(base) + idx));
-}
 
 __device__ __forceinline__ void record(int32_t* err, int32_t code) {
     if (err != nullptr) atomicCAS(err, 0, code);
+}
+
+// Byte offset of element (row r, column k) of a K-major bf16 tensor-core operand
+// with Kdim columns: 8 x 8 core matrices of 128 contiguous bytes (8 rows of 16
+// bytes), K-adjacent core matrices 128 bytes apart, 8-row groups Kdim*16 apart.
+__host__ __device__ constexpr uint32_t core_off(int r, int k, int Kdim) {
+    return (uint32_t)((r >> 3) * (Kdim >> 3) * 128 + (k >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // ---------------------------------------------------------------------------
@@ -105,18 +160,24 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
     const int hk = h / a.G;
     const int t0 = c * kC;
     const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
+    unsigned char* rec = record_of(a, bh, c);
+    float* TP = reinterpret_cast<float*>(rec + kRecTP);
+    float* Gs = reinterpret_cast<float*>(rec + kRecG);
 
-    // Load K, Q (fp32) and the gates.
-    for (int e = tid; e < kC * kD; e += kNT) {
-        const int t = e / kD, d = e % kD;
-        float kv = 0.f, qv = 0.f;
+    // Load K, Q (fp32) in groups of 8 and the gates.
+    for (int e = tid; e < kC * (kD / 8); e += kNT) {
+        const int t = e / (kD / 8), d0 = (e % (kD / 8)) * 8;
+        float kv[8] = {}, qv[8] = {};
         if (t < n) {
-            const size_t row = (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD;
-            kv = ld_in<InT>(a.k, row + d);
-            qv = ld_in<InT>(a.q, row + d);
+            const size_t row = (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD + d0;
+            ld8<InT>(a.k, row, kv);
+            ld8<InT>(a.q, row, qv);
         }
-        sm.K[t][d] = kv;
-        sm.X[t][d] = qv;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            sm.K[t][d0 + j] = kv[j];
+            sm.X[t][d0 + j] = qv[j];
+        }
     }
     if (tid < 32) {
         // log g_t = sum_{i<=t} log alpha_i by a warp scan over two 32-token halves.
@@ -139,6 +200,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
             }
             sm.lg[t] = carry + x;
             sm.bt[t] = be;
+            Gs[t] = carry + x;
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
     }
@@ -146,7 +208,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
 
     // KK (strictly lower, scaled into A) and QK (lower, scaled into P), 4x4 per thread:
     // rows ty*4 + r (broadcast within a half-warp), columns tx + 16 s (16 consecutive
-    // rows of K, conflict-free with the odd row stride).
+    // rows of K, conflict-free with the odd row stride).  P goes to the workspace:
+    // strictly below the diagonal transposed into TP's upper triangle, the diagonal to G.
     {
         const int ty = tid / 16, tx = tid % 16;
         float kk[4][4] = {}, qk[4][4] = {};
@@ -166,7 +229,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
                     qk[r][s] = fmaf(qr[r], kc[s], qk[r][s]);
                 }
         }
-        float* P = a.ws + ((size_t)bh * a.nchunks + c) * kWsFloats + kWsP;
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -174,8 +236,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
                 const int t = ty * 4 + r, i = tx + 16 * s;
                 const float ratio = i <= t ? expf(sm.lg[t] - sm.lg[i]) : 0.f;
                 sm.A[t][i] = i < t ? sm.bt[t] * ratio * kk[r][s] : 0.f;
-                P[t * kC + i] = i <= t ? ratio * qk[r][s] : 0.f;
+                if (i < t)
+                    TP[i * kTS + t] = ratio * qk[r][s];
+                else if (i == t)
+                    Gs[kC + t] = qk[r][s];
             }
+    }
+    // The tensor-core operands of kernel 2: [K; Q] and K^T as bf16 (exact: the
+    // inputs are bf16) in the K-major core layout, one 16-byte granule per store;
+    // consecutive threads write consecutive granules.
+    if constexpr (sizeof(InT) == 2) {
+        for (int e = tid; e < 2 * kC * (kD / 8); e += kNT) {
+            const int r = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;  // row, k-group
+            const float* src = r < kC ? &sm.K[r][8 * g] : &sm.X[r - kC][8 * g];
+            uint4 w;
+            w.x = pack_bf16x2(src[0], src[1]);
+            w.y = pack_bf16x2(src[2], src[3]);
+            w.z = pack_bf16x2(src[4], src[5]);
+            w.w = pack_bf16x2(src[6], src[7]);
+            *reinterpret_cast<uint4*>(rec + kRecA1 + core_off(r, 8 * g, kD)) = w;
+        }
+        for (int e = tid; e < kD * (kC / 8); e += kNT) {
+            const int d = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // dk row, token group
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = sm.K[8 * g + j][d];
+            uint4 w;
+            w.x = pack_bf16x2(x[0], x[1]);
+            w.y = pack_bf16x2(x[2], x[3]);
+            w.z = pack_bf16x2(x[4], x[5]);
+            w.w = pack_bf16x2(x[6], x[7]);
+            *reinterpret_cast<uint4*>(rec + kRecA2 + core_off(d, 8 * g, kC)) = w;
+        }
     }
     __syncthreads();
 
@@ -226,16 +318,17 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
     }
 
     // V (scaled by beta) replaces Q in X; U = T diag(beta) V, and Tb = T diag(beta g).
-    for (int e = tid; e < kC * kD; e += kNT) {
-        const int t = e / kD, d = e % kD;
-        float vv = 0.f;
-        if (t < n) vv = ld_in<InT>(a.v, (((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + d);
-        sm.X[t][d] = vv * sm.bt[t];
+    for (int e = tid; e < kC * (kD / 8); e += kNT) {
+        const int t = e / (kD / 8), d0 = (e % (kD / 8)) * 8;
+        float vv[8] = {};
+        if (t < n) ld8<InT>(a.v, (((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + d0, vv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sm.X[t][d0 + j] = vv[j] * sm.bt[t];
     }
     __syncthreads();
     {
-        float* rec = a.ws + ((size_t)bh * a.nchunks + c) * kWsFloats;
         // 64 x 128 outputs; thread: 4 rows x 8 columns (columns strided by 16 for bank spread)
+        float* U = reinterpret_cast<float*>(rec + kRecU);
         const int ty = tid / 16, tx = tid % 16;
         float u[4][8] = {};
         for (int i = 0; i < kC; ++i) {
@@ -252,21 +345,19 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int s = 0; s < 8; ++s) rec[kWsU + (ty * 4 + r) * kD + tx + 16 * s] = u[r][s];
+            for (int s = 0; s < 8; ++s) {
+                const int col = tx + 16 * s;
+                U[(col / kDVC) * (kC * kUS) + (ty * 4 + r) * kUS + col % kDVC] = u[r][s];
+            }
         for (int e = tid; e < kC * kC; e += kNT) {
             const int t = e / kC, i = e % kC;
-            rec[kWsT + e] = sm.T[t][i] * (sm.bt[i] * expf(sm.lg[i]));
+            if (i <= t) TP[t * kTS + i] = sm.T[t][i] * (sm.bt[i] * expf(sm.lg[i]));
         }
-        if (tid < kC) rec[kWsG + tid] = sm.lg[tid];
     }
 }
 
-// ---------------------------------------------------------------------------
-// Kernel 2 pieces shared by its two forms.
-// ---------------------------------------------------------------------------
-
-// Reads (src, dst) of request b into shared memory and classifies it: 0 run,
-// 1 padding (skipped silently), 2 bad index (skipped, reported).
+// Reads (src, dst) of request b and classifies it: 0 run, 1 padding (skipped
+// silently), 2 bad index (skipped, reported).
 __device__ __forceinline__ void scan_prologue(const ChunkArgs& a, int b, int& src, int& dst, int& status) {
     const int s = __ldg(a.src_idx + b), d = __ldg(a.dst_idx + b);
     int st = 0;
@@ -280,64 +371,9 @@ __device__ __forceinline__ void scan_prologue(const ChunkArgs& a, int b, int& sr
     if (st == 2) record(a.err, GDN_ERR_INDEX);
 }
 
-// E = U - Tb KM (stored over U), then O = QM + P E for the chunk's valid rows.
-// 64 x kDVC tiles: thread rows ty*2 + r, columns tx + 8 q.  QM already holds g Q M.
-__device__ __forceinline__ void scan_tail(const ChunkArgs& a, float (*U)[kDVC + 1], const float (*Tb)[kC + 1],
-                                          const float (*P)[kC + 1], const float (*KM)[kDVC + 1],
-                                          const float (*QM)[kDVC + 1], int b, int h, int t0, int n, int col0,
-                                          int tid) {
-    const int ty = tid / 8, tx = tid % 8;
-    float e[2][4];
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) e[r][q] = U[ty * 2 + r][tx + 8 * q];
-    for (int i = 0; i < kC; ++i) {
-        float km[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) km[q] = KM[i][tx + 8 * q];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const float tb = Tb[ty * 2 + r][i];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) e[r][q] = fmaf(-tb, km[q], e[r][q]);
-        }
-    }
-    // Each thread has read only its own U entries; E replaces them.
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) U[ty * 2 + r][tx + 8 * q] = e[r][q];
-    __syncthreads();
-    float o[2][4];
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) o[r][q] = QM[ty * 2 + r][tx + 8 * q];
-    for (int i = 0; i < kC; ++i) {
-        float ev[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) ev[q] = U[i][tx + 8 * q];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const float pr = P[ty * 2 + r][i];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) o[r][q] = fmaf(pr, ev[q], o[r][q]);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int t = ty * 2 + r;
-        if (t < n) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                a.out[(((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + col0 + tx + 8 * q] = o[r][q];
-        }
-    }
-}
-
 // ---------------------------------------------------------------------------
-// Kernel 2, CUDA-core form: per (b, h, column block of kDVC), the chunks in order.
+// Kernel 2, CUDA-core form (fp32 inputs): per (b, h, column block of kDVC), the
+// chunks in order.
 // ---------------------------------------------------------------------------
 struct Smem2 {
     float M[kD][kDVC + 1];      // state block, [dk][dv cols]
@@ -359,9 +395,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem2& sm = *reinterpret_cast<Smem2*>(smem_raw);
     const int tid = threadIdx.x;
-    constexpr int NCB = kD / kDVC;
-    const int cb = blockIdx.x % NCB;
-    const int bh = blockIdx.x / NCB;
+    const int cb = blockIdx.x % kNCB;
+    const int bh = blockIdx.x / kNCB;
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
     const int hk = h / a.G;
@@ -381,9 +416,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
     for (int c = 0; c < a.nchunks; ++c) {
         const int t0 = c * kC;
         const int n = min(kC, a.L - t0);
-        const float* rec = a.ws + ((size_t)bh * a.nchunks + c) * kWsFloats;
+        const unsigned char* rec = record_of(a, bh, c);
+        const float* Ur = reinterpret_cast<const float*>(rec + kRecU + cb * kUSlab);
+        const float* TP = reinterpret_cast<const float*>(rec + kRecTP);
+        const float* Gs = reinterpret_cast<const float*>(rec + kRecG);
         if (tid < kC) {
-            const float lgt = rec[kWsG + tid], lgC_ = rec[kWsG + kC - 1];
+            const float lgt = Gs[tid], lgC_ = Gs[kC - 1];
             sm.lg[tid] = lgt;
             sm.gq[tid] = expf(lgt);
             sm.gk[tid] = expf(lgC_ - lgt);
@@ -403,11 +441,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
         }
         for (int e = tid; e < kC * kDVC; e += kNT) {
             const int t = e / kDVC, jj = e % kDVC;
-            sm.U[t][jj] = rec[kWsU + (size_t)t * kD + col0 + jj];
+            sm.U[t][jj] = Ur[t * kUS + jj];
         }
         for (int e = tid; e < kC * kC; e += kNT) {
-            sm.Tb[e / kC][e % kC] = rec[kWsT + e];
-            sm.P[e / kC][e % kC] = rec[kWsP + e];
+            const int t = e / kC, i = e % kC;
+            sm.Tb[t][i] = i <= t ? TP[t * kTS + i] : 0.f;
+            sm.P[t][i] = i < t ? TP[i * kTS + t] : (i == t ? Gs[kC + t] : 0.f);
         }
         __syncthreads();
 
@@ -437,8 +476,59 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
                 }
         }
         __syncthreads();
-        scan_tail(a, sm.U, sm.Tb, sm.P, sm.KM, sm.QM, b, h, t0, n, col0, tid);
-        // M is updated from K^T E on the CUDA cores
+        // E = U - Tb KM (over U); each thread reads and writes only its own entries.
+        {
+            float e[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) e[r][q] = sm.U[ty * 2 + r][tx + 8 * q];
+            for (int i = 0; i < kC; ++i) {
+                float km[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) km[q] = sm.KM[i][tx + 8 * q];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const float tb = sm.Tb[ty * 2 + r][i];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) e[r][q] = fmaf(-tb, km[q], e[r][q]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sm.U[ty * 2 + r][tx + 8 * q] = e[r][q];
+        }
+        __syncthreads();
+        // O = QM + P E for the chunk's valid rows
+        {
+            float o[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) o[r][q] = sm.QM[ty * 2 + r][tx + 8 * q];
+            for (int i = 0; i < kC; ++i) {
+                float ev[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) ev[q] = sm.U[i][tx + 8 * q];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const float pr = sm.P[ty * 2 + r][i];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) o[r][q] = fmaf(pr, ev[q], o[r][q]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int t = ty * 2 + r;
+                if (t < n) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        a.out[(((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + col0 + tx + 8 * q] = o[r][q];
+                }
+            }
+        }
+        // M = g_C M + K^T diag(g_C / g) E; each thread reads and writes only its own rows of M.
         {
             const float gC = expf(lgC);
             const int ry = tid / 8;  // rows ry*4 .. +3
@@ -453,7 +543,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) acc[q] = fmaf(kv, sm.U[t][tx + 8 * q], acc[q]);
                 }
-                // Each thread reads and writes only its own rows of M in this phase.
 #pragma unroll
                 for (int q = 0; q < 4; ++q) sm.M[i][tx + 8 * q] = acc[q];
             }
@@ -474,19 +563,17 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 //                       K = dk in 8 steps; M split into 3 bf16 parts -> 24 MMAs)
 //   D2 = K^T E'        (M=128 rows of dk, N = kDVC, K = 64 tokens in 4 steps,
 //                       E' = diag(g_C / g) E split into 3 bf16 parts -> 12 MMAs)
-// Operands sit in shared memory in the no-swizzle K-major canonical layout
-// (8 x 8 bf16 core matrices of 128 contiguous bytes); accumulators live in
-// 64 TMEM columns (D1 at column 0, D2 at column 32) allocated by warp 0.
-// Thread 0 issues the MMAs and commits them to an mbarrier; every wait is
-// bounded.  The triangular products (Tb KM, P E) run on the CUDA cores.
+// Operands sit in shared memory in the no-swizzle K-major core layout;
+// accumulators live in 64 TMEM columns (D1 at column 0, D2 at column 32)
+// allocated by warp 0.  Thread 0 issues the MMAs and commits them to an
+// mbarrier, and streams the chunk images: the image of chunk c + 2 is copied
+// (cp.async.bulk, two buffers) while chunk c + 1's waits and chunk c computes.
+// The triangular products (Tb KM, P E) run on the CUDA cores, each thread on a
+// row pair (p, 63 - p) so that every thread does the same 65 row-steps.  Every
+// wait is bounded (2 s); a timeout is recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Byte offset of element (row r, column k) of a K-major bf16 tile with Kdim columns.
-__device__ __forceinline__ uint32_t core_off(int r, int k, int Kdim) {
-    return (uint32_t)((r >> 3) * (Kdim >> 3) * 128 + (k >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2);
 }
 
 // Shared-memory matrix descriptor: no swizzle, K-adjacent core matrices 128 B apart
@@ -517,6 +604,23 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(1) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 
 __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
     uint32_t done = 0;
@@ -549,29 +653,35 @@ __device__ __forceinline__ void tmem_ld16(uint32_t addr, float (&v)[16]) {
     for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
 
-// x = hi + mid + lo with each part in bf16 (24 significant bits in total).
-__device__ __forceinline__ void split3(float x, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
-    hi = __float2bfloat16_rn(x);
-    const float r1 = x - __bfloat162float(hi);
-    mid = __float2bfloat16_rn(r1);
-    lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+// Eight fp32 values as three 16-byte granules of bf16 parts: x = hi + mid + lo.
+__device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& mid, uint4& lo) {
+    uint32_t h[4], m[4], l[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a0 = x[2 * j], a1 = x[2 * j + 1];
+        h[j] = pack_bf16x2(a0, a1);
+        a0 -= __uint_as_float(h[j] << 16);
+        a1 -= __uint_as_float(h[j] & 0xffff0000u);
+        m[j] = pack_bf16x2(a0, a1);
+        a0 -= __uint_as_float(m[j] << 16);
+        a1 -= __uint_as_float(m[j] & 0xffff0000u);
+        l[j] = pack_bf16x2(a0, a1);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    mid = make_uint4(m[0], m[1], m[2], m[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;  // one bf16 part of M^T (32 x 128)
+
 struct SmemTC {
-    unsigned char A1[128 * kD * 2];        // [K; Q] rows x dk, K-major core tiles
-    unsigned char A2[kD * kC * 2];         // K^T: dk rows x 64 tokens
-    unsigned char B1[3][kDVC * kD * 2];    // M^T parts: kDVC rows x dk
-    unsigned char B2[3][kDVC * kC * 2];    // E'^T parts: kDVC rows x 64 tokens
-    float M[kD][kDVC + 1];
-    float U[kC][kDVC + 1];                 // U, then E
-    float Tb[kC][kC + 1];
-    float P[kC][kC + 1];
-    float KM[kC][kDVC + 1];
-    float QM[kC][kDVC + 1];
-    float lg[kC];
-    float gq[kC];
-    float gk[kC];
-    uint64_t bar;
+    unsigned char buf[2][kBufBytes];  // chunk images (A1 A2 U TP G), double-buffered
+    unsigned char bop[3][kBopPart];   // B operand parts: M^T, later E'^T (32 x 64, same slots)
+    float M[kD][kUS];                 // state block [dk][32 columns]
+    float KM[kC][kUS];
+    float QM[kC][kUS];                // g Q M
+    uint64_t full[2];
+    uint64_t mma;
     uint32_t tmem;
     int src, dst, status;
 };
@@ -581,19 +691,35 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     SmemTC& sm = *reinterpret_cast<SmemTC*>(smem_tc);
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
-    constexpr int NCB = kD / kDVC;
-    const int cb = blockIdx.x % NCB;
-    const int bh = blockIdx.x / NCB;
+    const int cb = blockIdx.x % kNCB;
+    const int bh = blockIdx.x / kNCB;
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
-    const int hk = h / a.G;
     const int col0 = cb * kDVC;
     constexpr uint32_t kIdesc = umma_idesc(128, kDVC);
+    const int nch = a.nchunks;
+
+    // Thread 0 copies chunk c's image into buffer c & 1.
+    auto issue = [&](int c) {
+        const unsigned char* rec = record_of(a, bh, c);
+        unsigned char* dst = sm.buf[c & 1];
+        uint64_t* bar = &sm.full[c & 1];
+        mbar_expect_tx(bar, kBufBytes);
+        bulk_g2s(dst, rec, (uint32_t)kRecU, bar);
+        bulk_g2s(dst + kBufU, rec + kRecU + cb * kUSlab, (uint32_t)kUSlab, bar);
+        bulk_g2s(dst + kBufTP, rec + kRecTP, (uint32_t)(kRecBytes - kRecTP), bar);
+    };
 
     if (tid == 0) {
         scan_prologue(a, b, sm.src, sm.dst, sm.status);
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&sm.bar)), "r"(1) : "memory");
+        mbar_init(&sm.full[0]);
+        mbar_init(&sm.full[1]);
+        mbar_init(&sm.mma);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (sm.status == 0) {
+            issue(0);
+            if (nch > 1) issue(1);
+        }
     }
     __syncthreads();
     if (sm.status != 0) return;
@@ -603,156 +729,208 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-
-    const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD);
-    for (int e = tid; e < kD * kDVC; e += kNT) {
-        const int i = e / kDVC, j = e % kDVC;
-        sm.M[i][j] = M0[(size_t)i * kD + col0 + j];
+    {
+        const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) + col0;
+        for (int e = tid; e < kD * (kDVC / 4); e += kNT) {
+            const int i = e / (kDVC / 4), j4 = e % (kDVC / 4);
+            *reinterpret_cast<float4*>(&sm.M[i][4 * j4]) = *reinterpret_cast<const float4*>(M0 + (size_t)i * kD + 4 * j4);
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;  // TMEM columns half*16 .. +15
-    const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(a.k);
-    const __nv_bfloat16* qin = static_cast<const __nv_bfloat16*>(a.q);
-    uint32_t phase = 0;
+    const int half = warp / 4;          // TMEM columns half*16 .. +15
+    const int tx = tid % 8, p = tid / 8; // triangular phases: columns 4tx..4tx+3, rows p and 63-p
+    const int rlo = p, rhi = kC - 1 - p;
     bool ok = true;
+    int c = 0;
 
-    for (int c = 0; c < a.nchunks && ok; ++c) {
+    for (; c < nch; ++c) {
+        const int s = c & 1;
         const int t0 = c * kC;
         const int n = min(kC, a.L - t0);
-        const float* rec = a.ws + ((size_t)bh * a.nchunks + c) * kWsFloats;
-        if (tid < kC) {
-            const float lgt = rec[kWsG + tid], lgC_ = rec[kWsG + kC - 1];
-            sm.lg[tid] = lgt;
-            sm.gq[tid] = expf(lgt);
-            sm.gk[tid] = expf(lgC_ - lgt);
+        if (__syncthreads_or(wait_parity(&sm.full[s], (uint32_t)(c >> 1) & 1u) ? 0 : 1)) {
+            ok = false;
+            break;
         }
-        // Operands of D1 and D2's A: K and Q rows as they are (exact bf16).
-        for (int e = tid; e < kC * kD; e += kNT) {
-            const int t = e / kD, d = e % kD;
-            __nv_bfloat16 kv = __float2bfloat16_rn(0.f), qv = kv;
-            if (t < n) {
-                const size_t row = (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD;
-                kv = kin[row + d];
-                qv = qin[row + d];
-            }
-            *reinterpret_cast<__nv_bfloat16*>(sm.A1 + core_off(t, d, kD)) = kv;
-            *reinterpret_cast<__nv_bfloat16*>(sm.A1 + core_off(kC + t, d, kD)) = qv;
-            *reinterpret_cast<__nv_bfloat16*>(sm.A2 + core_off(d, t, kC)) = kv;
-        }
-        for (int e = tid; e < kC * kDVC; e += kNT) {
-            const int t = e / kDVC, jj = e % kDVC;
-            sm.U[t][jj] = rec[kWsU + (size_t)t * kD + col0 + jj];
-        }
-        for (int e = tid; e < kC * kC; e += kNT) {
-            sm.Tb[e / kC][e % kC] = rec[kWsT + e];
-            sm.P[e / kC][e % kC] = rec[kWsP + e];
-        }
-        // B of D1: M^T in three bf16 parts.
-        for (int e = tid; e < kD * kDVC; e += kNT) {
-            const int i = e / kDVC, jj = e % kDVC;
-            __nv_bfloat16 p0, p1, p2;
-            split3(sm.M[i][jj], p0, p1, p2);
-            const uint32_t off = core_off(jj, i, kD);
-            *reinterpret_cast<__nv_bfloat16*>(sm.B1[0] + off) = p0;
-            *reinterpret_cast<__nv_bfloat16*>(sm.B1[1] + off) = p1;
-            *reinterpret_cast<__nv_bfloat16*>(sm.B1[2] + off) = p2;
+        unsigned char* img = sm.buf[s];
+        float* U = reinterpret_cast<float*>(img + kBufU);          // [64][kUS]: U, then E
+        const float* TP = reinterpret_cast<const float*>(img + kBufTP);
+        const float* lg = reinterpret_cast<const float*>(img + kBufG);
+        const float* pd = lg + kC;
+
+        // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.
+        for (int e = tid; e < kDVC * (kD / 8); e += kNT) {
+            const int jj = e % kDVC, g = e / kDVC;
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = sm.M[8 * g + j][jj];
+            uint4 p0, p1, p2;
+            split3x8(x, p0, p1, p2);
+            const uint32_t off = core_off(jj, 8 * g, kD);
+            *reinterpret_cast<uint4*>(sm.bop[0] + off) = p0;
+            *reinterpret_cast<uint4*>(sm.bop[1] + off) = p1;
+            *reinterpret_cast<uint4*>(sm.bop[2] + off) = p2;
         }
         async_proxy_fence();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
+            const uint32_t a1 = smem_u32(img);
             for (int part = 0; part < 3; ++part)
-                for (int s = 0; s < kD / 16; ++s)
-                    umma_bf16(tmem, umma_desc(smem_u32(sm.A1) + 256 * s, (kD / 8) * 128),
-                              umma_desc(smem_u32(sm.B1[part]) + 256 * s, (kD / 8) * 128), kIdesc,
-                              (part | s) != 0 ? 1u : 0u);
-            umma_commit(&sm.bar);
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    umma_bf16(tmem, umma_desc(a1 + 256 * ks, (kD / 8) * 128),
+                              umma_desc(smem_u32(sm.bop[part]) + 256 * ks, (kD / 8) * 128), kIdesc,
+                              (part | ks) != 0 ? 1u : 0u);
+            umma_commit(&sm.mma);
         }
         // The decision to read TMEM is block-uniform (tcgen05.ld is warp-collective).
-        if (__syncthreads_or(wait_parity(&sm.bar, phase) ? 0 : 1)) {
+        if (__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1)) {
             ok = false;
             break;
         }
-        phase ^= 1u;
         tc_fence_after();
         {
             float v[16];
             tmem_ld16(tmem + lane_base + (uint32_t)(half * 16), v);
             const int row = (warp % 4) * 32 + lane;
+            float* dstrow;
+            float g = 1.f;
             if (row < kC) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) sm.KM[row][half * 16 + j] = v[j];
+                dstrow = &sm.KM[row][half * 16];
             } else {
-                const float g = sm.gq[row - kC];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) sm.QM[row - kC][half * 16 + j] = v[j] * g;
+                dstrow = &sm.QM[row - kC][half * 16];
+                g = expf(lg[row - kC]);
             }
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(dstrow + j) = make_float4(v[j] * g, v[j + 1] * g, v[j + 2] * g, v[j + 3] * g);
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        scan_tail(a, sm.U, sm.Tb, sm.P, sm.KM, sm.QM, b, h, t0, n, col0, tid);
+        // E = U - Tb KM over U: Tb[t][i] = TP[t][i] for i <= t.
+        {
+            float4 elo = *reinterpret_cast<const float4*>(&U[rlo * kUS + 4 * tx]);
+            float4 ehi = *reinterpret_cast<const float4*>(&U[rhi * kUS + 4 * tx]);
+            for (int i = 0; i <= rhi; ++i) {
+                const float4 km = *reinterpret_cast<const float4*>(&sm.KM[i][4 * tx]);
+                const float th = TP[rhi * kTS + i];
+                ehi.x = fmaf(-th, km.x, ehi.x), ehi.y = fmaf(-th, km.y, ehi.y);
+                ehi.z = fmaf(-th, km.z, ehi.z), ehi.w = fmaf(-th, km.w, ehi.w);
+                if (i <= rlo) {
+                    const float tl = TP[rlo * kTS + i];
+                    elo.x = fmaf(-tl, km.x, elo.x), elo.y = fmaf(-tl, km.y, elo.y);
+                    elo.z = fmaf(-tl, km.z, elo.z), elo.w = fmaf(-tl, km.w, elo.w);
+                }
+            }
+            *reinterpret_cast<float4*>(&U[rlo * kUS + 4 * tx]) = elo;
+            *reinterpret_cast<float4*>(&U[rhi * kUS + 4 * tx]) = ehi;
+        }
+        __syncthreads();
 
-        // B of D2: E' = diag(g_C / g) E, transposed, in three bf16 parts.
-        for (int e = tid; e < kC * kDVC; e += kNT) {
-            const int t = e / kDVC, jj = e % kDVC;
-            __nv_bfloat16 p0, p1, p2;
-            split3(sm.U[t][jj] * sm.gk[t], p0, p1, p2);
-            const uint32_t off = core_off(jj, t, kC);
-            *reinterpret_cast<__nv_bfloat16*>(sm.B2[0] + off) = p0;
-            *reinterpret_cast<__nv_bfloat16*>(sm.B2[1] + off) = p1;
-            *reinterpret_cast<__nv_bfloat16*>(sm.B2[2] + off) = p2;
+        // B of D2: E' = diag(g_C / g) E, transposed (32 rows x 64 tokens), three bf16 parts.
+        {
+            const int jj = tid % kDVC, g = tid / kDVC;  // 32 x 8 granules, one per thread
+            const float lgC = lg[kC - 1];
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = U[(8 * g + j) * kUS + jj] * expf(lgC - lg[8 * g + j]);
+            uint4 p0, p1, p2;
+            split3x8(x, p0, p1, p2);
+            const uint32_t off = core_off(jj, 8 * g, kC);
+            *reinterpret_cast<uint4*>(sm.bop[0] + off) = p0;
+            *reinterpret_cast<uint4*>(sm.bop[1] + off) = p1;
+            *reinterpret_cast<uint4*>(sm.bop[2] + off) = p2;
         }
         async_proxy_fence();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
+            const uint32_t a2 = smem_u32(img + kBufA2);
             for (int part = 0; part < 3; ++part)
-                for (int s = 0; s < kC / 16; ++s)
-                    umma_bf16(tmem + 32, umma_desc(smem_u32(sm.A2) + 256 * s, (kC / 8) * 128),
-                              umma_desc(smem_u32(sm.B2[part]) + 256 * s, (kC / 8) * 128), kIdesc,
-                              (part | s) != 0 ? 1u : 0u);
-            umma_commit(&sm.bar);
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    umma_bf16(tmem + 32, umma_desc(a2 + 256 * ks, (kC / 8) * 128),
+                              umma_desc(smem_u32(sm.bop[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
+                              (part | ks) != 0 ? 1u : 0u);
+            umma_commit(&sm.mma);
         }
-        if (__syncthreads_or(wait_parity(&sm.bar, phase) ? 0 : 1)) {
+
+        // O = QM + P E while the tensor core works; P[t][i] = TP[i][t] for i < t, P[t][t] = pd[t].
+        {
+            float4 olo = *reinterpret_cast<const float4*>(&sm.QM[rlo][4 * tx]);
+            float4 ohi = *reinterpret_cast<const float4*>(&sm.QM[rhi][4 * tx]);
+            for (int i = 0; i < rhi; ++i) {
+                const float4 ev = *reinterpret_cast<const float4*>(&U[i * kUS + 4 * tx]);
+                const float ph = TP[i * kTS + rhi];
+                ohi.x = fmaf(ph, ev.x, ohi.x), ohi.y = fmaf(ph, ev.y, ohi.y);
+                ohi.z = fmaf(ph, ev.z, ohi.z), ohi.w = fmaf(ph, ev.w, ohi.w);
+                if (i < rlo) {
+                    const float pl = TP[i * kTS + rlo];
+                    olo.x = fmaf(pl, ev.x, olo.x), olo.y = fmaf(pl, ev.y, olo.y);
+                    olo.z = fmaf(pl, ev.z, olo.z), olo.w = fmaf(pl, ev.w, olo.w);
+                }
+            }
+            {
+                const float4 eh = *reinterpret_cast<const float4*>(&U[rhi * kUS + 4 * tx]);
+                const float4 el = *reinterpret_cast<const float4*>(&U[rlo * kUS + 4 * tx]);
+                const float dh = pd[rhi], dl = pd[rlo];
+                ohi.x = fmaf(dh, eh.x, ohi.x), ohi.y = fmaf(dh, eh.y, ohi.y);
+                ohi.z = fmaf(dh, eh.z, ohi.z), ohi.w = fmaf(dh, eh.w, ohi.w);
+                olo.x = fmaf(dl, el.x, olo.x), olo.y = fmaf(dl, el.y, olo.y);
+                olo.z = fmaf(dl, el.z, olo.z), olo.w = fmaf(dl, el.w, olo.w);
+            }
+            float* ob = a.out + (((size_t)b * a.L + t0) * a.Hv + h) * kD + col0 + 4 * tx;
+            const size_t row_stride = (size_t)a.Hv * kD;
+            if (rlo < n) *reinterpret_cast<float4*>(ob + rlo * row_stride) = olo;
+            if (rhi < n) *reinterpret_cast<float4*>(ob + rhi * row_stride) = ohi;
+        }
+
+        if (__syncthreads_or(wait_parity(&sm.mma, 1) ? 0 : 1)) {
             ok = false;
             break;
         }
-        phase ^= 1u;
         tc_fence_after();
         {
             float v[16];
             tmem_ld16(tmem + lane_base + 32u + (uint32_t)(half * 16), v);
             const int i = (warp % 4) * 32 + lane;  // dk row
-            const float gC = expf(sm.lg[kC - 1]);
+            const float gC = expf(lg[kC - 1]);
+            float* mrow = &sm.M[i][half * 16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) sm.M[i][half * 16 + j] = fmaf(gC, sm.M[i][half * 16 + j], v[j]);
+            for (int j = 0; j < 16; j += 4) {
+                float4 m = *reinterpret_cast<float4*>(mrow + j);
+                m.x = fmaf(gC, m.x, v[j]), m.y = fmaf(gC, m.y, v[j + 1]);
+                m.z = fmaf(gC, m.z, v[j + 2]), m.w = fmaf(gC, m.w, v[j + 3]);
+                *reinterpret_cast<float4*>(mrow + j) = m;
+            }
         }
+        // Buffer s (E was written into it) is refilled next by the async proxy.
+        async_proxy_fence();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0 && c + 2 < nch) issue(c + 2);
     }
 
     if (ok) {
-        float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD);
-        for (int e = tid; e < kD * kDVC; e += kNT) {
-            const int i = e / kDVC, jj = e % kDVC;
-            MD[(size_t)i * kD + col0 + jj] = sm.M[i][jj];
+        float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + col0;
+        for (int e = tid; e < kD * (kDVC / 4); e += kNT) {
+            const int i = e / (kDVC / 4), j4 = e % (kDVC / 4);
+            *reinterpret_cast<float4*>(MD + (size_t)i * kD + 4 * j4) = *reinterpret_cast<const float4*>(&sm.M[i][4 * j4]);
         }
-    } else {
-        // A commit that never arrived: give the tensor core one more bounded wait
-        // to finish with this CTA's TMEM before it is freed.
-        if (tid == 0) {
-            record(a.err, GDN_ERR_TIMEOUT);
-            wait_parity(&sm.bar, phase);
-        }
+    } else if (tid == 0) {
+        // Something never arrived: record it, then give the copies and MMAs still
+        // in flight one more bounded wait each before the shared memory and TMEM go.
+        record(a.err, GDN_ERR_TIMEOUT);
+        for (int cc = c; cc < min(c + 2, nch); ++cc) wait_parity(&sm.full[cc & 1], (uint32_t)(cc >> 1) & 1u);
+        wait_parity(&sm.mma, 0);
+        wait_parity(&sm.mma, 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -766,7 +944,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
 extern "C" size_t gdn_prefill_workspace_bytes(int32_t B, int32_t L, int32_t Hv, int32_t dk, int32_t dv) {
     if (B < 0 || L < 1 || Hv < 1 || dk != kD || dv != kD) return 0;
     const size_t nchunks = ((size_t)L + kC - 1) / kC;
-    return (size_t)B * Hv * nchunks * kWsFloats * sizeof(float);
+    return (size_t)B * Hv * nchunks * kRecBytes;
 }
 
 extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const int32_t* src_idx,
@@ -784,10 +962,14 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     const int nchunks = (L + kC - 1) / kC;
     if (workspace_bytes < gdn_prefill_workspace_bytes(B, L, Hv, dk, dv)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)B * Hv * nchunks >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return GDN_ERR_INVALID_ARG;
+    // 16-byte vector accesses: workspace, pool, out, q, k, v (rows of 128 elements keep the alignment).
+    const uintptr_t align = reinterpret_cast<uintptr_t>(workspace) | reinterpret_cast<uintptr_t>(pool) |
+                            reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(q) |
+                            reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v);
+    if ((align & 15u) != 0) return GDN_ERR_INVALID_ARG;
 
-    const ChunkArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, static_cast<float*>(workspace), err_word,
-                      num_slots, B, L, Hk, Hv, Hv / Hk, nchunks};
+    const ChunkArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, static_cast<unsigned char*>(workspace),
+                      err_word, num_slots, B, L, Hk, Hv, Hv / Hk, nchunks};
     const bool bf = qkv_dtype == GDN_BF16;
     const int s1 = (int)sizeof(Smem1), s2 = bf ? (int)sizeof(SmemTC) : (int)sizeof(Smem2);
     cudaError_t e = bf ? cudaFuncSetAttribute(gdn_chunk_prepare_kernel<__nv_bfloat16>,
@@ -798,7 +980,7 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     e = bf ? cudaFuncSetAttribute(gdn_chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s2)
            : cudaFuncSetAttribute(gdn_chunk_scan_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    const unsigned g1 = (unsigned)(B * Hv * nchunks), g2 = (unsigned)(B * Hv * (kD / kDVC));
+    const unsigned g1 = (unsigned)(B * Hv * nchunks), g2 = (unsigned)(B * Hv * kNCB);
     if (bf) {
         gdn_chunk_prepare_kernel<__nv_bfloat16><<<g1, kNT, s1, stream>>>(a);
         gdn_chunk_scan_tc_kernel<<<g2, kNT, s2, stream>>>(a);

@@ -212,7 +212,8 @@ gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, c
  *                    dk, dv) bytes, 16-byte aligned, caller-owned; contents on entry
  *                    do not matter and on return are unspecified.  Calls sharing one
  *                    workspace must not overlap.
- * Unsupported shapes, a missing or short workspace return GDN_ERR_INVALID_ARG.
+ * Unsupported shapes, a missing or short workspace, or a workspace, pool, out, q, k
+ * or v that is not 16-byte aligned return GDN_ERR_INVALID_ARG.
  */
 gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const int32_t* src_idx, const int32_t* dst_idx,
                                const void* q, const void* k, const void* v, const float* alpha,
