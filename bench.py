@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).  See profiles/.
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "0f7ea8d477b60cefbdac3a835a678b5b8a8a89eea3d73729c64fab3e78ee1145",
-               "bytes_per_launch": 541223168 + 483794688,
+               "source_sha256": "2749ceb8bdba484ccb2c638bc20fa1bd165c2b17abd6d9fd3899c0caa34bbfaa",
+               "bytes_per_launch": 541164544 + 483485952,
                "profile": "profiles/gdn_tile1_kernel_large_decode.md"}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
