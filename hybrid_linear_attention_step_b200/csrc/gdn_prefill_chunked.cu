@@ -30,13 +30,14 @@
 // precision.
 //
 // Workspace record of one (request, head, chunk), bytes, laid out as the
-// shared-memory image kernel 2 copies in (bulk copies, 16-byte granules):
+// shared-memory images kernel 2 copies in (bulk copies, 16-byte granules):
 //   A1  [K; Q] as bf16, 128 rows x 128 (dk) in the no-swizzle K-major core
 //       layout of the tensor-core operand (bf16 inputs only)
 //   A2  K^T as bf16, 128 (dk) rows x 64 tokens, same layout (bf16 inputs only)
 //   U   four column slabs [4][64][36] fp32 (32 columns + 4 padding each)
-//   TP  [64][65] fp32: Tb on and below the diagonal, P^T strictly above it
-//   G   log g [64], then the diagonal of P [64]
+//   TbT [64][64] fp32: Tb transposed, TbT[i][t] = Tb[t][i], zero for t < i
+//   PT  [64][64] fp32: P transposed, PT[i][t] = P[t][i], zero for t < i
+//   G   log g [64]
 
 #include "gdn_step.h"
 
@@ -52,7 +53,6 @@ constexpr int kDVC = 32;        // value columns per CTA in the sequential kerne
 constexpr int kNCB = kD / kDVC; // column blocks per (request, head)
 constexpr int kNT = 256;        // threads per CTA (both kernels)
 constexpr int kUS = kDVC + 4;   // row stride of the 64 x 32 fp32 tiles (16-byte rows, bank spread)
-constexpr int kTS = kC + 1;     // row stride of TP
 constexpr int kPad = 4;         // row padding of [C][D] shared arrays in the fp32 scan kernel
 
 // Workspace record (bytes).
@@ -60,18 +60,17 @@ constexpr size_t kRecA1 = 0;
 constexpr size_t kRecA2 = kRecA1 + (size_t)2 * kC * kD * 2;
 constexpr size_t kRecU = kRecA2 + (size_t)kD * kC * 2;
 constexpr size_t kUSlab = (size_t)kC * kUS * 4;
-constexpr size_t kRecTP = kRecU + kNCB * kUSlab;
-constexpr size_t kRecG = kRecTP + (size_t)kC * kTS * 4;
-constexpr size_t kRecBytes = kRecG + (size_t)2 * kC * 4;
-// One CTA's image of a chunk in shared memory: A1 A2 | its U slab | TP G.
-constexpr uint32_t kBufA2 = (uint32_t)kRecA2;
-constexpr uint32_t kBufU = (uint32_t)kRecU;
-constexpr uint32_t kBufTP = kBufU + (uint32_t)kUSlab;
-constexpr uint32_t kBufG = kBufTP + (uint32_t)((size_t)kC * kTS * 4);
-constexpr uint32_t kBufBytes = kBufG + 2 * kC * 4;
-static_assert(kRecU % 16 == 0 && kRecTP % 16 == 0 && kRecG % 16 == 0 && kRecBytes % 16 == 0, "16-byte records");
-static_assert(kUSlab % 16 == 0 && kBufTP % 16 == 0 && kBufBytes % 16 == 0, "16-byte bulk copies");
-static_assert(kRecG - kRecTP == kBufG - kBufTP, "TP and G are copied together");
+constexpr size_t kRecTb = kRecU + kNCB * kUSlab;
+constexpr size_t kRecP = kRecTb + (size_t)kC * kC * 4;
+constexpr size_t kRecG = kRecP + (size_t)kC * kC * 4;
+constexpr size_t kRecBytes = kRecG + (size_t)kC * 4;
+// One CTA's small image of a chunk in shared memory: its U slab | TbT PT G.
+constexpr uint32_t kImgTb = (uint32_t)kUSlab;
+constexpr uint32_t kImgP = kImgTb + (uint32_t)(kRecP - kRecTb);
+constexpr uint32_t kImgG = kImgP + (uint32_t)(kRecG - kRecP);
+constexpr uint32_t kImgBytes = kImgG + (uint32_t)(kRecBytes - kRecG);
+static_assert(kRecA2 % 16 == 0 && kRecU % 16 == 0 && kRecTb % 16 == 0 && kRecBytes % 16 == 0, "16-byte records");
+static_assert(kUSlab % 16 == 0 && kImgBytes % 16 == 0, "16-byte bulk copies");
 
 struct ChunkArgs {
     float* pool;
@@ -92,7 +91,7 @@ __device__ __forceinline__ unsigned char* record_of(const ChunkArgs& a, int bh, 
     return a.ws + ((size_t)bh * a.nchunks + c) * kRecBytes;
 }
 
-// 8 consecutive input elements (a 16-byte aligned group for bf16, 32 bytes for fp32) as fp32.
+// 8 consecutive fp32 input elements (32 bytes, 16-byte aligned).
 template <typename InT>
 __device__ __forceinline__ void ld8(const void* base, size_t idx, float (&x)[8]);
 template <>
@@ -101,17 +100,6 @@ __device__ __forceinline__ void ld8<float>(const void* base, size_t idx, float (
     const float4 a = __ldg(p), b = __ldg(p + 1);
     x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
 }
-template <>
-__device__ __forceinline__ void ld8<__nv_bfloat16>(const void* base, size_t idx, float (&x)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        x[2 * j] = __uint_as_float(w[j] << 16);
-        x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-    }
-}
-
 template <typename InT>
 __device__ __forceinline__ float ld_in(const void* base, size_t idx);
 template <>
@@ -136,7 +124,191 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 1: per (b, h, chunk), independent of the state.
+// tcgen05 / bulk-copy helpers (sm_100a PTX).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor: no swizzle, K-adjacent core matrices 128 B apart
+// (leading byte offset), 8-row groups `sbo` bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) |
+           (1ull << 46);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(1) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
+    uint32_t done = 0;
+    uint64_t t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    while (true) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+        uint64_t t1;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+        if (t1 - t0 > 2000000000ull) return false;  // 2 s
+    }
+}
+
+// 16 consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(addr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Eight fp32 values as three 16-byte granules of bf16 parts: x = hi + mid + lo.
+__device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& mid, uint4& lo) {
+    uint32_t h[4], m[4], l[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a0 = x[2 * j], a1 = x[2 * j + 1];
+        h[j] = pack_bf16x2(a0, a1);
+        a0 -= __uint_as_float(h[j] << 16);
+        a1 -= __uint_as_float(h[j] & 0xffff0000u);
+        m[j] = pack_bf16x2(a0, a1);
+        a0 -= __uint_as_float(m[j] << 16);
+        a1 -= __uint_as_float(m[j] & 0xffff0000u);
+        l[j] = pack_bf16x2(a0, a1);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    mid = make_uint4(m[0], m[1], m[2], m[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1 pieces shared by its two forms.
+// ---------------------------------------------------------------------------
+
+// Warp 0: log g_t = sum_{i<=t} log alpha_i by a warp scan over two 32-token
+// halves, beta_t, and log g into the record.
+__device__ __forceinline__ void gate_scan(const ChunkArgs& a, int b, int h, int t0, int n, int lane, float* lg,
+                                          float* bt, float* Gs) {
+    float carry = 0.f;
+    for (int half = 0; half < 2; ++half) {
+        const int t = half * 32 + lane;
+        const size_t gi = (((size_t)b * a.L + t0 + t) * a.Hv + h);
+        float la = 0.f, be = 0.f;
+        if (t < n) {
+            // alpha = 0 (a full reset) would make log g = -inf and the ratios
+            // -inf - -inf; e^-80 ~ 2e-35 is zero at fp32 precision instead.
+            la = fmaxf(logf(__ldg(a.alpha + gi)), -80.f);
+            be = __ldg(a.beta + gi);
+        }
+        float x = la;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        lg[t] = carry + x;
+        bt[t] = be;
+        Gs[t] = carry + x;
+        carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+}
+
+// T = (I + A)^-1 for strictly lower-triangular A (all threads; A complete on
+// entry, T complete on return).  Blocked in 16 x 16: diagonal blocks by forward
+// substitution (one warp each), then block rows I = 1..3:
+// T_IJ = -T_II sum_{J<=K<I} A_IK T_KJ.
+__device__ __forceinline__ void invert_unit_lower(const float (*A)[kC + 1], float (*T)[kC + 1], float (*Y)[48],
+                                                  int tid) {
+    const int w = tid / 32, lane = tid % 32;
+    if (w < 4) {
+        const int o = w * 16;
+        for (int r = 0; r < 16; ++r) {
+            if (lane < 16) {
+                const int j = lane;
+                float val = (r == j) ? 1.f : 0.f;
+                if (j < r) {
+                    float acc = 0.f;
+                    for (int m = j; m < r; ++m) acc = fmaf(A[o + r][o + m], T[o + m][o + j], acc);
+                    val = -acc;
+                }
+                T[o + r][o + j] = val;
+            }
+            __syncwarp();
+        }
+    }
+    // zero the strictly upper blocks
+    for (int e = tid; e < kC * kC; e += kNT) {
+        const int r = e / kC, j = e % kC;
+        if (j / 16 > r / 16) T[r][j] = 0.f;
+    }
+    __syncthreads();
+    for (int I = 1; I < 4; ++I) {
+        // Y[r][J*16 + j] = sum_{K=J}^{I-1} sum_m A[16I + r][16K + m] T[16K + m][16J + j]
+        for (int e = tid; e < 16 * 16 * I; e += kNT) {
+            const int r = e / (16 * I), col = e % (16 * I);
+            const int J = col / 16, j = col % 16;
+            float acc = 0.f;
+            for (int kk2 = 16 * J; kk2 < 16 * I; ++kk2) acc = fmaf(A[16 * I + r][kk2], T[kk2][16 * J + j], acc);
+            Y[r][col] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < 16 * 16 * I; e += kNT) {
+            const int r = e / (16 * I), col = e % (16 * I);
+            float acc = 0.f;
+            for (int m = 0; m <= r; ++m) acc = fmaf(T[16 * I + r][16 * I + m], Y[m][col], acc);
+            T[16 * I + r][col] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1, CUDA-core form (fp32 inputs): per (b, h, chunk), independent of the state.
 // ---------------------------------------------------------------------------
 struct Smem1 {
     float K[kC][kD + 1];     // odd row stride: rows r and r+1 sit in different banks
@@ -161,7 +333,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
     const int t0 = c * kC;
     const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
     unsigned char* rec = record_of(a, bh, c);
-    float* TP = reinterpret_cast<float*>(rec + kRecTP);
+    float* TbT = reinterpret_cast<float*>(rec + kRecTb);
+    float* PT = reinterpret_cast<float*>(rec + kRecP);
     float* Gs = reinterpret_cast<float*>(rec + kRecG);
 
     // Load K, Q (fp32) in groups of 8 and the gates.
@@ -179,37 +352,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
             sm.X[t][d0 + j] = qv[j];
         }
     }
-    if (tid < 32) {
-        // log g_t = sum_{i<=t} log alpha_i by a warp scan over two 32-token halves.
-        float carry = 0.f;
-        for (int half = 0; half < 2; ++half) {
-            const int t = half * 32 + tid;
-            const size_t gi = (((size_t)b * a.L + t0 + t) * a.Hv + h);
-            float la = 0.f, be = 0.f;
-            if (t < n) {
-                // alpha = 0 (a full reset) would make log g = -inf and the ratios
-                // -inf - -inf; e^-80 ~ 2e-35 is zero at fp32 precision instead.
-                la = fmaxf(logf(__ldg(a.alpha + gi)), -80.f);
-                be = __ldg(a.beta + gi);
-            }
-            float x = la;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (tid >= off) x += y;
-            }
-            sm.lg[t] = carry + x;
-            sm.bt[t] = be;
-            Gs[t] = carry + x;
-            carry += __shfl_sync(0xffffffffu, x, 31);
-        }
-    }
+    if (tid < 32) gate_scan(a, b, h, t0, n, tid, sm.lg, sm.bt, Gs);
     __syncthreads();
 
     // KK (strictly lower, scaled into A) and QK (lower, scaled into P), 4x4 per thread:
     // rows ty*4 + r (broadcast within a half-warp), columns tx + 16 s (16 consecutive
-    // rows of K, conflict-free with the odd row stride).  P goes to the workspace:
-    // strictly below the diagonal transposed into TP's upper triangle, the diagonal to G.
+    // rows of K, conflict-free with the odd row stride).  P goes to the workspace, transposed.
     {
         const int ty = tid / 16, tx = tid % 16;
         float kk[4][4] = {}, qk[4][4] = {};
@@ -236,86 +384,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
                 const int t = ty * 4 + r, i = tx + 16 * s;
                 const float ratio = i <= t ? expf(sm.lg[t] - sm.lg[i]) : 0.f;
                 sm.A[t][i] = i < t ? sm.bt[t] * ratio * kk[r][s] : 0.f;
-                if (i < t)
-                    TP[i * kTS + t] = ratio * qk[r][s];
-                else if (i == t)
-                    Gs[kC + t] = qk[r][s];
+                PT[i * kC + t] = ratio * qk[r][s];
             }
-    }
-    // The tensor-core operands of kernel 2: [K; Q] and K^T as bf16 (exact: the
-    // inputs are bf16) in the K-major core layout, one 16-byte granule per store;
-    // consecutive threads write consecutive granules.
-    if constexpr (sizeof(InT) == 2) {
-        for (int e = tid; e < 2 * kC * (kD / 8); e += kNT) {
-            const int r = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;  // row, k-group
-            const float* src = r < kC ? &sm.K[r][8 * g] : &sm.X[r - kC][8 * g];
-            uint4 w;
-            w.x = pack_bf16x2(src[0], src[1]);
-            w.y = pack_bf16x2(src[2], src[3]);
-            w.z = pack_bf16x2(src[4], src[5]);
-            w.w = pack_bf16x2(src[6], src[7]);
-            *reinterpret_cast<uint4*>(rec + kRecA1 + core_off(r, 8 * g, kD)) = w;
-        }
-        for (int e = tid; e < kD * (kC / 8); e += kNT) {
-            const int d = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // dk row, token group
-            float x[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = sm.K[8 * g + j][d];
-            uint4 w;
-            w.x = pack_bf16x2(x[0], x[1]);
-            w.y = pack_bf16x2(x[2], x[3]);
-            w.z = pack_bf16x2(x[4], x[5]);
-            w.w = pack_bf16x2(x[6], x[7]);
-            *reinterpret_cast<uint4*>(rec + kRecA2 + core_off(d, 8 * g, kC)) = w;
-        }
     }
     __syncthreads();
 
-    // T = (I + A)^-1, blocked in 16 x 16: diagonal blocks by forward substitution
-    // (one warp each), then block rows I = 1..3: T_IJ = -T_II sum_{J<=K<I} A_IK T_KJ.
-    {
-        const int w = tid / 32, lane = tid % 32;
-        if (w < 4) {
-            const int o = w * 16;
-            for (int r = 0; r < 16; ++r) {
-                if (lane < 16) {
-                    const int j = lane;
-                    float val = (r == j) ? 1.f : 0.f;
-                    if (j < r) {
-                        float acc = 0.f;
-                        for (int m = j; m < r; ++m) acc = fmaf(sm.A[o + r][o + m], sm.T[o + m][o + j], acc);
-                        val = -acc;
-                    }
-                    sm.T[o + r][o + j] = val;
-                }
-                __syncwarp();
-            }
-        }
-        // zero the strictly upper blocks
-        for (int e = tid; e < kC * kC; e += kNT) {
-            const int r = e / kC, j = e % kC;
-            if (j / 16 > r / 16) sm.T[r][j] = 0.f;
-        }
-        __syncthreads();
-        for (int I = 1; I < 4; ++I) {
-            // Y[r][J*16 + j] = sum_{K=J}^{I-1} sum_m A[16I + r][16K + m] T[16K + m][16J + j]
-            for (int e = tid; e < 16 * 16 * I; e += kNT) {
-                const int r = e / (16 * I), col = e % (16 * I);
-                const int J = col / 16, j = col % 16;
-                float acc = 0.f;
-                for (int kk2 = 16 * J; kk2 < 16 * I; ++kk2) acc = fmaf(sm.A[16 * I + r][kk2], sm.T[kk2][16 * J + j], acc);
-                sm.Y[r][col] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < 16 * 16 * I; e += kNT) {
-                const int r = e / (16 * I), col = e % (16 * I);
-                float acc = 0.f;
-                for (int m = 0; m <= r; ++m) acc = fmaf(sm.T[16 * I + r][16 * I + m], sm.Y[m][col], acc);
-                sm.T[16 * I + r][col] = -acc;
-            }
-            __syncthreads();
-        }
-    }
+    invert_unit_lower(sm.A, sm.T, sm.Y, tid);
 
     // V (scaled by beta) replaces Q in X; U = T diag(beta) V, and Tb = T diag(beta g).
     for (int e = tid; e < kC * (kD / 8); e += kNT) {
@@ -350,10 +424,232 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
                 U[(col / kDVC) * (kC * kUS) + (ty * 4 + r) * kUS + col % kDVC] = u[r][s];
             }
         for (int e = tid; e < kC * kC; e += kNT) {
-            const int t = e / kC, i = e % kC;
-            if (i <= t) TP[t * kTS + i] = sm.T[t][i] * (sm.bt[i] * expf(sm.lg[i]));
+            const int i = e / kC, t = e % kC;
+            TbT[e] = i <= t ? sm.T[t][i] * (sm.bt[i] * expf(sm.lg[i])) : 0.f;
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1, tensor-core form (bf16 inputs).  The products whose operands are the
+// chunk's bf16 inputs run as tcgen05 MMAs with fp32 accumulation in TMEM:
+//   D0 = [K; Q] K^T                 (M = 128, N = 64, K = dk: 8 MMAs, exact products)
+//   D1 = V^T (T diag(beta))^T = U^T (M = 128 = dv, N = 64, K = 64 tokens; the fp32
+//                                    factor in three bf16 parts: 12 MMAs)
+// The inverse T and the elementwise gate scalings stay on the CUDA cores.
+// ---------------------------------------------------------------------------
+struct SmemP {
+    union {
+        unsigned char A1[2 * kC * kD * 2];     // [K; Q] operand (also B = K of D0)
+        float Y[16][48];                       // scratch of the inverse (after D0)
+        struct {
+            unsigned char VT[kD * kC * 2];     // V^T operand of D1
+            unsigned char Bp[3][kC * kC * 2];  // (T diag(beta)) parts, B of D1
+        } d1;
+    } op;
+    union {
+        float A[kC][kC + 1];
+        __nv_bfloat16 Vb[kC][kD + 2];  // V rows after the inverse (odd word stride for the column gathers)
+    } av;
+    float T[kC][kC + 1];
+    float lg[kC];
+    float bt[kC];
+    uint64_t mma;
+    uint32_t tmem;
+};
+static_assert(sizeof(SmemP) <= 74 * 1024 + 1024, "three prepare CTAs per SM");
+
+__global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem_p[];
+    SmemP& sm = *reinterpret_cast<SmemP*>(smem_p);
+    const int tid = threadIdx.x;
+    const int warp = tid / 32, lane = tid % 32;
+    const int c = blockIdx.x % a.nchunks;
+    const int bh = blockIdx.x / a.nchunks;
+    const int h = bh % a.Hv;
+    const int b = bh / a.Hv;
+    const int hk = h / a.G;
+    const int t0 = c * kC;
+    const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
+    unsigned char* rec = record_of(a, bh, c);
+    float* TbT = reinterpret_cast<float*>(rec + kRecTb);
+    float* PT = reinterpret_cast<float*>(rec + kRecP);
+    float* Gs = reinterpret_cast<float*>(rec + kRecG);
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const int half = warp / 4;  // TMEM columns 32*half .. +31 of each accumulator
+
+    if (tid == 0) {
+        mbar_init(&sm.mma);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
+                     "r"(128)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, Gs);
+    }
+    // k, q, v in 16-byte granules: [K; Q] into the operand image (shared memory and the
+    // record, where kernel 2 reads it); V stays in registers until the inverse is done.
+    // Consecutive threads take consecutive granules of the image: token
+    // t = (e & 7) + 8 (e >> 7), group g = (e >> 3) & 15, e = tid + 256 u.
+    constexpr int kGr = kC * (kD / 8) / kNT;  // granules per thread
+    uint4 vkeep[kGr];
+#pragma unroll
+    for (int u = 0; u < kGr; ++u) {
+        const int e = tid + kNT * u;
+        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+        uint4 kq = make_uint4(0, 0, 0, 0), qq = kq, vv = kq;
+        if (t < n) {
+            const size_t row = (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD + 8 * g;
+            const size_t vrow = (((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + 8 * g;
+            kq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + row));
+            qq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row));
+            vv = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + vrow));
+        }
+        const uint32_t ok = core_off(t, 8 * g, kD), oq = core_off(kC + t, 8 * g, kD);
+        *reinterpret_cast<uint4*>(sm.op.A1 + ok) = kq;
+        *reinterpret_cast<uint4*>(sm.op.A1 + oq) = qq;
+        *reinterpret_cast<uint4*>(rec + kRecA1 + ok) = kq;
+        *reinterpret_cast<uint4*>(rec + kRecA1 + oq) = qq;
+        vkeep[u] = vv;
+    }
+    async_proxy_fence();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+    constexpr uint32_t kIdesc = umma_idesc(128, kC);
+    if (tid == 0) {
+        const uint32_t a1 = smem_u32(sm.op.A1);
+        for (int ks = 0; ks < kD / 16; ++ks)
+            umma_bf16(tmem, umma_desc(a1 + 256 * ks, (kD / 8) * 128), umma_desc(a1 + 256 * ks, (kD / 8) * 128),
+                      kIdesc, ks != 0 ? 1u : 0u);
+        umma_commit(&sm.mma);
+    }
+    // K^T image for kernel 2, gathered from the K rows of the [K; Q] image:
+    // granule (dk row d, tokens 8 g' .. 8 g' + 7); consecutive threads write consecutive granules.
+    for (int e = tid; e < kD * (kC / 8); e += kNT) {
+        const int d = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;
+        uint16_t x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = *reinterpret_cast<const uint16_t*>(sm.op.A1 + core_off(8 * g + j, d, kD));
+        uint4 w;
+        w.x = x[0] | ((uint32_t)x[1] << 16);
+        w.y = x[2] | ((uint32_t)x[3] << 16);
+        w.z = x[4] | ((uint32_t)x[5] << 16);
+        w.w = x[6] | ((uint32_t)x[7] << 16);
+        *reinterpret_cast<uint4*>(rec + kRecA2 + core_off(d, 8 * g, kC)) = w;
+    }
+    bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
+    if (ok) {
+        tc_fence_after();
+        // D0 row r < 64: k_r . k_i -> A (scaled); row 64 + t: q_t . k_i -> P (record).
+        const int r = (warp % 4) * 32 + lane;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            float v[16];
+            const int i0 = 32 * half + 16 * part;
+            tmem_ld16(tmem + lane_base + (uint32_t)i0, v);
+            if (r < kC) {
+                const float lt = sm.lg[r], bt = sm.bt[r];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int i = i0 + j;
+                    sm.av.A[r][i] = i < r ? bt * expf(lt - sm.lg[i]) * v[j] : 0.f;
+                }
+            } else {
+                const int t = r - kC;
+                const float lt = sm.lg[t];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int i = i0 + j;
+                    PT[i * kC + t] = i <= t ? expf(lt - sm.lg[i]) * v[j] : 0.f;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        invert_unit_lower(sm.av.A, sm.T, sm.op.Y, tid);  // the [K; Q] image is dead: D0 is complete
+        // V rows over A (dead after the inverse)
+#pragma unroll
+        for (int u = 0; u < kGr; ++u) {
+            const int e = tid + kNT * u;
+            const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+            uint32_t* vr = reinterpret_cast<uint32_t*>(&sm.av.Vb[t][8 * g]);
+            vr[0] = vkeep[u].x, vr[1] = vkeep[u].y, vr[2] = vkeep[u].z, vr[3] = vkeep[u].w;
+        }
+        __syncthreads();
+
+        // D1 operands.
+        for (int e = tid; e < kD * (kC / 8); e += kNT) {
+            const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // dv row j, tokens 8g..8g+7
+            uint16_t x[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint16_t*>(&sm.av.Vb[8 * g + m][j]);
+            uint4 w;
+            w.x = x[0] | ((uint32_t)x[1] << 16);
+            w.y = x[2] | ((uint32_t)x[3] << 16);
+            w.z = x[4] | ((uint32_t)x[5] << 16);
+            w.w = x[6] | ((uint32_t)x[7] << 16);
+            *reinterpret_cast<uint4*>(sm.op.d1.VT + core_off(j, 8 * g, kC)) = w;
+        }
+        for (int e = tid; e < kC * (kC / 8); e += kNT) {
+            const int t = e % kC, g = e / kC;  // row t of T diag(beta), columns 8g..8g+7
+            float x[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) x[m] = sm.T[t][8 * g + m] * sm.bt[8 * g + m];
+            uint4 p0, p1, p2;
+            split3x8(x, p0, p1, p2);
+            const uint32_t off = core_off(t, 8 * g, kC);
+            *reinterpret_cast<uint4*>(sm.op.d1.Bp[0] + off) = p0;
+            *reinterpret_cast<uint4*>(sm.op.d1.Bp[1] + off) = p1;
+            *reinterpret_cast<uint4*>(sm.op.d1.Bp[2] + off) = p2;
+        }
+        async_proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            const uint32_t vt = smem_u32(sm.op.d1.VT);
+            for (int part = 0; part < 3; ++part)
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    umma_bf16(tmem + 64, umma_desc(vt + 256 * ks, (kC / 8) * 128),
+                              umma_desc(smem_u32(sm.op.d1.Bp[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
+                              (part | ks) != 0 ? 1u : 0u);
+            umma_commit(&sm.mma);
+        }
+        // Tb = T diag(beta g), transposed, while the MMAs run.
+        for (int e = tid; e < kC * kC; e += kNT) {
+            const int i = e / kC, t = e % kC;
+            TbT[e] = i <= t ? sm.T[t][i] * (sm.bt[i] * expf(sm.lg[i])) : 0.f;
+        }
+        ok = !__syncthreads_or(wait_parity(&sm.mma, 1) ? 0 : 1);
+        if (ok) {
+            tc_fence_after();
+            // D1[j][t] = U[t][j]: lane j of this warp's quadrant, tokens 32*half .. +31.
+            const int j = (warp % 4) * 32 + lane;
+            float* U = reinterpret_cast<float*>(rec + kRecU) + (j / kDVC) * (kC * kUS) + j % kDVC;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float v[16];
+                const int tb = 32 * half + 16 * part;
+                tmem_ld16(tmem + lane_base + 64u + (uint32_t)tb, v);
+#pragma unroll
+                for (int m = 0; m < 16; ++m) U[(tb + m) * kUS] = v[m];
+            }
+        }
+    }
+    if (!ok && tid == 0) {
+        record(a.err, GDN_ERR_TIMEOUT);
+        wait_parity(&sm.mma, 0);
+        wait_parity(&sm.mma, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
 }
 
 // Reads (src, dst) of request b and classifies it: 0 run, 1 padding (skipped
@@ -418,7 +714,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
         const int n = min(kC, a.L - t0);
         const unsigned char* rec = record_of(a, bh, c);
         const float* Ur = reinterpret_cast<const float*>(rec + kRecU + cb * kUSlab);
-        const float* TP = reinterpret_cast<const float*>(rec + kRecTP);
+        const float* TbT = reinterpret_cast<const float*>(rec + kRecTb);
+        const float* PT = reinterpret_cast<const float*>(rec + kRecP);
         const float* Gs = reinterpret_cast<const float*>(rec + kRecG);
         if (tid < kC) {
             const float lgt = Gs[tid], lgC_ = Gs[kC - 1];
@@ -445,8 +742,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
         }
         for (int e = tid; e < kC * kC; e += kNT) {
             const int t = e / kC, i = e % kC;
-            sm.Tb[t][i] = i <= t ? TP[t * kTS + i] : 0.f;
-            sm.P[t][i] = i < t ? TP[i * kTS + t] : (i == t ? Gs[kC + t] : 0.f);
+            sm.Tb[t][i] = TbT[i * kC + t];
+            sm.P[t][i] = PT[i * kC + t];
         }
         __syncthreads();
 
@@ -565,123 +862,27 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 //                       E' = diag(g_C / g) E split into 3 bf16 parts -> 12 MMAs)
 // Operands sit in shared memory in the no-swizzle K-major core layout;
 // accumulators live in 64 TMEM columns (D1 at column 0, D2 at column 32)
-// allocated by warp 0.  Thread 0 issues the MMAs and commits them to an
-// mbarrier, and streams the chunk images: the image of chunk c + 2 is copied
-// (cp.async.bulk, two buffers) while chunk c + 1's waits and chunk c computes.
-// The triangular products (Tb KM, P E) run on the CUDA cores, each thread on a
-// row pair (p, 63 - p) so that every thread does the same 65 row-steps.  Every
-// wait is bounded (2 s); a timeout is recorded and the CTA drains and exits.
+// allocated by warp 0.  Thread 0 issues the MMAs, commits them to an mbarrier,
+// and streams the chunk images with cp.async.bulk: the MMA operands [K; Q] and
+// K^T (one buffer each, refilled for the next chunk as soon as their MMAs
+// complete) and the small image (U slab, Tb^T, P^T, log g; two buffers, two
+// chunks ahead).  The triangular products Tb KM and P E run on the CUDA cores:
+// lane j owns value column j, warp w the rows 4w..4w+3 and 60-4w..63-4w, so a
+// step over i reads one KM (or E) value and two broadcast float4 of Tb^T (P^T).
+// Every wait is bounded (2 s); a timeout is recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Shared-memory matrix descriptor: no swizzle, K-adjacent core matrices 128 B apart
-// (leading byte offset), 8-row groups `sbo` bytes apart (stride byte offset), version 1.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) |
-           (1ull << 46);
-}
-
-// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, both K-major.
-__host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(da), "l"(db), "r"(idesc), "r"(acc)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(1) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
-    uint32_t done = 0;
-    uint64_t t0;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-    while (true) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        if (done) return true;
-        uint64_t t1;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
-        if (t1 - t0 > 2000000000ull) return false;  // 2 s
-    }
-}
-
-// 16 consecutive TMEM columns of this warp's 32 lanes.
-__device__ __forceinline__ void tmem_ld16(uint32_t addr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(addr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// Eight fp32 values as three 16-byte granules of bf16 parts: x = hi + mid + lo.
-__device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& mid, uint4& lo) {
-    uint32_t h[4], m[4], l[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float a0 = x[2 * j], a1 = x[2 * j + 1];
-        h[j] = pack_bf16x2(a0, a1);
-        a0 -= __uint_as_float(h[j] << 16);
-        a1 -= __uint_as_float(h[j] & 0xffff0000u);
-        m[j] = pack_bf16x2(a0, a1);
-        a0 -= __uint_as_float(m[j] << 16);
-        a1 -= __uint_as_float(m[j] & 0xffff0000u);
-        l[j] = pack_bf16x2(a0, a1);
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    mid = make_uint4(m[0], m[1], m[2], m[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
 constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;  // one bf16 part of M^T (32 x 128)
 
 struct SmemTC {
-    unsigned char buf[2][kBufBytes];  // chunk images (A1 A2 U TP G), double-buffered
-    unsigned char bop[3][kBopPart];   // B operand parts: M^T, later E'^T (32 x 64, same slots)
-    float M[kD][kUS];                 // state block [dk][32 columns]
+    unsigned char a1[2 * kC * kD * 2];  // [K; Q] operand of D1
+    unsigned char a2[kD * kC * 2];      // K^T operand of D2
+    unsigned char img[2][kImgBytes];    // small images, double-buffered
+    unsigned char bop[3][kBopPart];     // B operand parts: M^T, later E'^T (32 x 64, same slots)
+    float M[kD][kUS];                   // state block [dk][32 columns]
     float KM[kC][kUS];
-    float QM[kC][kUS];                // g Q M
-    uint64_t full[2];
-    uint64_t mma;
+    float QM[kC][kUS];                  // g Q M
+    uint64_t full[2];                   // small images
+    uint64_t bar_a1, bar_a2, mma;
     uint32_t tmem;
     int src, dst, status;
 };
@@ -699,26 +900,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     constexpr uint32_t kIdesc = umma_idesc(128, kDVC);
     const int nch = a.nchunks;
 
-    // Thread 0 copies chunk c's image into buffer c & 1.
-    auto issue = [&](int c) {
+    // Thread 0's copies.  Every barrier completes once per chunk (or once per
+    // use of its buffer), so the parity of the n-th completion is n & 1.
+    auto issue_small = [&](int c) {
         const unsigned char* rec = record_of(a, bh, c);
-        unsigned char* dst = sm.buf[c & 1];
+        unsigned char* dst = sm.img[c & 1];
         uint64_t* bar = &sm.full[c & 1];
-        mbar_expect_tx(bar, kBufBytes);
-        bulk_g2s(dst, rec, (uint32_t)kRecU, bar);
-        bulk_g2s(dst + kBufU, rec + kRecU + cb * kUSlab, (uint32_t)kUSlab, bar);
-        bulk_g2s(dst + kBufTP, rec + kRecTP, (uint32_t)(kRecBytes - kRecTP), bar);
+        mbar_expect_tx(bar, kImgBytes);
+        bulk_g2s(dst, rec + kRecU + cb * kUSlab, (uint32_t)kUSlab, bar);
+        bulk_g2s(dst + kImgTb, rec + kRecTb, (uint32_t)(kRecBytes - kRecTb), bar);
+    };
+    auto issue_a1 = [&](int c) {
+        mbar_expect_tx(&sm.bar_a1, (uint32_t)kRecA2);
+        bulk_g2s(sm.a1, record_of(a, bh, c) + kRecA1, (uint32_t)kRecA2, &sm.bar_a1);
+    };
+    auto issue_a2 = [&](int c) {
+        mbar_expect_tx(&sm.bar_a2, (uint32_t)(kRecU - kRecA2));
+        bulk_g2s(sm.a2, record_of(a, bh, c) + kRecA2, (uint32_t)(kRecU - kRecA2), &sm.bar_a2);
     };
 
     if (tid == 0) {
         scan_prologue(a, b, sm.src, sm.dst, sm.status);
         mbar_init(&sm.full[0]);
         mbar_init(&sm.full[1]);
+        mbar_init(&sm.bar_a1);
+        mbar_init(&sm.bar_a2);
         mbar_init(&sm.mma);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (sm.status == 0) {
-            issue(0);
-            if (nch > 1) issue(1);
+            issue_a1(0);
+            issue_a2(0);
+            issue_small(0);
+            if (nch > 1) issue_small(1);
         }
     }
     __syncthreads();
@@ -741,25 +954,33 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;          // TMEM columns half*16 .. +15
-    const int tx = tid % 8, p = tid / 8; // triangular phases: columns 4tx..4tx+3, rows p and 63-p
-    const int rlo = p, rhi = kC - 1 - p;
+    const int half = warp / 4;           // TMEM columns half*16 .. +15
+    const int r1 = 4 * warp;             // triangular phases: rows r1..r1+3 and r2..r2+3, column `lane`
+    const int r2 = kC - 4 - 4 * warp;
+    const uint64_t da1 = umma_desc(smem_u32(sm.a1), (kD / 8) * 128);
+    const uint64_t da2 = umma_desc(smem_u32(sm.a2), (kC / 8) * 128);
     bool ok = true;
     int c = 0;
+    int waits_mma = 0;   // completed waits per barrier (all threads); thread 0 also
+    int done_a1 = 0, done_a2 = 0, done_small = 0;  // counts what it issued, below
+    int issued_a1 = 1, issued_a2 = 1, issued_small = min(nch, 2), issued_mma = 0;
 
     for (; c < nch; ++c) {
         const int s = c & 1;
         const int t0 = c * kC;
         const int n = min(kC, a.L - t0);
-        if (__syncthreads_or(wait_parity(&sm.full[s], (uint32_t)(c >> 1) & 1u) ? 0 : 1)) {
+        bool got = wait_parity(&sm.full[s], (uint32_t)(c >> 1) & 1u);
+        got = wait_parity(&sm.bar_a1, (uint32_t)c & 1u) && got;
+        if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        unsigned char* img = sm.buf[s];
-        float* U = reinterpret_cast<float*>(img + kBufU);          // [64][kUS]: U, then E
-        const float* TP = reinterpret_cast<const float*>(img + kBufTP);
-        const float* lg = reinterpret_cast<const float*>(img + kBufG);
-        const float* pd = lg + kC;
+        ++done_small, ++done_a1;
+        unsigned char* img = sm.img[s];
+        float* U = reinterpret_cast<float*>(img);  // [64][kUS]: U, then E
+        const float* TbT = reinterpret_cast<const float*>(img + kImgTb);
+        const float* PT = reinterpret_cast<const float*>(img + kImgP);
+        const float* lg = reinterpret_cast<const float*>(img + kImgG);
 
         // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.
         for (int e = tid; e < kDVC * (kD / 8); e += kNT) {
@@ -779,20 +1000,25 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            const uint32_t a1 = smem_u32(img);
-            for (int part = 0; part < 3; ++part)
+            for (int part = 0; part < 3; ++part) {
+                const uint64_t db = umma_desc(smem_u32(sm.bop[part]), (kD / 8) * 128);
                 for (int ks = 0; ks < kD / 16; ++ks)
-                    umma_bf16(tmem, umma_desc(a1 + 256 * ks, (kD / 8) * 128),
-                              umma_desc(smem_u32(sm.bop[part]) + 256 * ks, (kD / 8) * 128), kIdesc,
-                              (part | ks) != 0 ? 1u : 0u);
+                    umma_bf16(tmem, da1 + 16 * ks, db + 16 * ks, kIdesc, (part | ks) != 0 ? 1u : 0u);
+            }
             umma_commit(&sm.mma);
         }
+        ++issued_mma;
         // The decision to read TMEM is block-uniform (tcgen05.ld is warp-collective).
-        if (__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1)) {
+        if (__syncthreads_or(wait_parity(&sm.mma, (uint32_t)waits_mma & 1u) ? 0 : 1)) {
             ok = false;
             break;
         }
+        ++waits_mma;
         tc_fence_after();
+        if (c + 1 < nch) {  // the [K; Q] buffer is free again
+            if (tid == 0) issue_a1(c + 1);
+            ++issued_a1;
+        }
         {
             float v[16];
             tmem_ld16(tmem + lane_base + (uint32_t)(half * 16), v);
@@ -813,23 +1039,37 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         __syncthreads();
         tc_fence_after();
 
-        // E = U - Tb KM over U: Tb[t][i] = TP[t][i] for i <= t.
+        // E = U - Tb KM over U.  Tb^T[i][t] is zero for t < i, so rows r1.. need
+        // i <= r1 + 3 and rows r2.. need i <= r2 + 3.
         {
-            float4 elo = *reinterpret_cast<const float4*>(&U[rlo * kUS + 4 * tx]);
-            float4 ehi = *reinterpret_cast<const float4*>(&U[rhi * kUS + 4 * tx]);
-            for (int i = 0; i <= rhi; ++i) {
-                const float4 km = *reinterpret_cast<const float4*>(&sm.KM[i][4 * tx]);
-                const float th = TP[rhi * kTS + i];
-                ehi.x = fmaf(-th, km.x, ehi.x), ehi.y = fmaf(-th, km.y, ehi.y);
-                ehi.z = fmaf(-th, km.z, ehi.z), ehi.w = fmaf(-th, km.w, ehi.w);
-                if (i <= rlo) {
-                    const float tl = TP[rlo * kTS + i];
-                    elo.x = fmaf(-tl, km.x, elo.x), elo.y = fmaf(-tl, km.y, elo.y);
-                    elo.z = fmaf(-tl, km.z, elo.z), elo.w = fmaf(-tl, km.w, elo.w);
-                }
+            float e1[4], e2[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                e1[r] = U[(r1 + r) * kUS + lane];
+                e2[r] = U[(r2 + r) * kUS + lane];
             }
-            *reinterpret_cast<float4*>(&U[rlo * kUS + 4 * tx]) = elo;
-            *reinterpret_cast<float4*>(&U[rhi * kUS + 4 * tx]) = ehi;
+#pragma unroll 4
+            for (int i = 0; i <= r1 + 3; ++i) {
+                const float km = sm.KM[i][lane];
+                const float4 ta = *reinterpret_cast<const float4*>(TbT + i * kC + r1);
+                const float4 tb = *reinterpret_cast<const float4*>(TbT + i * kC + r2);
+                e1[0] = fmaf(-ta.x, km, e1[0]), e1[1] = fmaf(-ta.y, km, e1[1]);
+                e1[2] = fmaf(-ta.z, km, e1[2]), e1[3] = fmaf(-ta.w, km, e1[3]);
+                e2[0] = fmaf(-tb.x, km, e2[0]), e2[1] = fmaf(-tb.y, km, e2[1]);
+                e2[2] = fmaf(-tb.z, km, e2[2]), e2[3] = fmaf(-tb.w, km, e2[3]);
+            }
+#pragma unroll 4
+            for (int i = r1 + 4; i <= r2 + 3; ++i) {
+                const float km = sm.KM[i][lane];
+                const float4 tb = *reinterpret_cast<const float4*>(TbT + i * kC + r2);
+                e2[0] = fmaf(-tb.x, km, e2[0]), e2[1] = fmaf(-tb.y, km, e2[1]);
+                e2[2] = fmaf(-tb.z, km, e2[2]), e2[3] = fmaf(-tb.w, km, e2[3]);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                U[(r1 + r) * kUS + lane] = e1[r];
+                U[(r2 + r) * kUS + lane] = e2[r];
+            }
         }
         __syncthreads();
 
@@ -847,55 +1087,69 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             *reinterpret_cast<uint4*>(sm.bop[1] + off) = p1;
             *reinterpret_cast<uint4*>(sm.bop[2] + off) = p2;
         }
+        got = wait_parity(&sm.bar_a2, (uint32_t)c & 1u);
         async_proxy_fence();
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            const uint32_t a2 = smem_u32(img + kBufA2);
-            for (int part = 0; part < 3; ++part)
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem + 32, umma_desc(a2 + 256 * ks, (kC / 8) * 128),
-                              umma_desc(smem_u32(sm.bop[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
-                              (part | ks) != 0 ? 1u : 0u);
-            umma_commit(&sm.mma);
-        }
-
-        // O = QM + P E while the tensor core works; P[t][i] = TP[i][t] for i < t, P[t][t] = pd[t].
-        {
-            float4 olo = *reinterpret_cast<const float4*>(&sm.QM[rlo][4 * tx]);
-            float4 ohi = *reinterpret_cast<const float4*>(&sm.QM[rhi][4 * tx]);
-            for (int i = 0; i < rhi; ++i) {
-                const float4 ev = *reinterpret_cast<const float4*>(&U[i * kUS + 4 * tx]);
-                const float ph = TP[i * kTS + rhi];
-                ohi.x = fmaf(ph, ev.x, ohi.x), ohi.y = fmaf(ph, ev.y, ohi.y);
-                ohi.z = fmaf(ph, ev.z, ohi.z), ohi.w = fmaf(ph, ev.w, ohi.w);
-                if (i < rlo) {
-                    const float pl = TP[i * kTS + rlo];
-                    olo.x = fmaf(pl, ev.x, olo.x), olo.y = fmaf(pl, ev.y, olo.y);
-                    olo.z = fmaf(pl, ev.z, olo.z), olo.w = fmaf(pl, ev.w, olo.w);
-                }
-            }
-            {
-                const float4 eh = *reinterpret_cast<const float4*>(&U[rhi * kUS + 4 * tx]);
-                const float4 el = *reinterpret_cast<const float4*>(&U[rlo * kUS + 4 * tx]);
-                const float dh = pd[rhi], dl = pd[rlo];
-                ohi.x = fmaf(dh, eh.x, ohi.x), ohi.y = fmaf(dh, eh.y, ohi.y);
-                ohi.z = fmaf(dh, eh.z, ohi.z), ohi.w = fmaf(dh, eh.w, ohi.w);
-                olo.x = fmaf(dl, el.x, olo.x), olo.y = fmaf(dl, el.y, olo.y);
-                olo.z = fmaf(dl, el.z, olo.z), olo.w = fmaf(dl, el.w, olo.w);
-            }
-            float* ob = a.out + (((size_t)b * a.L + t0) * a.Hv + h) * kD + col0 + 4 * tx;
-            const size_t row_stride = (size_t)a.Hv * kD;
-            if (rlo < n) *reinterpret_cast<float4*>(ob + rlo * row_stride) = olo;
-            if (rhi < n) *reinterpret_cast<float4*>(ob + rhi * row_stride) = ohi;
-        }
-
-        if (__syncthreads_or(wait_parity(&sm.mma, 1) ? 0 : 1)) {
+        if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
+        ++done_a2;
         tc_fence_after();
+        if (tid == 0) {
+            for (int part = 0; part < 3; ++part) {
+                const uint64_t db = umma_desc(smem_u32(sm.bop[part]), (kC / 8) * 128);
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    umma_bf16(tmem + 32, da2 + 16 * ks, db + 16 * ks, kIdesc, (part | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.mma);
+        }
+        ++issued_mma;
+
+        // O = QM + P E while the tensor core works (P^T[i][t] is zero for t < i).
+        {
+            float o1[4], o2[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                o1[r] = sm.QM[r1 + r][lane];
+                o2[r] = sm.QM[r2 + r][lane];
+            }
+#pragma unroll 4
+            for (int i = 0; i <= r1 + 3; ++i) {
+                const float ev = U[i * kUS + lane];
+                const float4 pa = *reinterpret_cast<const float4*>(PT + i * kC + r1);
+                const float4 pb = *reinterpret_cast<const float4*>(PT + i * kC + r2);
+                o1[0] = fmaf(pa.x, ev, o1[0]), o1[1] = fmaf(pa.y, ev, o1[1]);
+                o1[2] = fmaf(pa.z, ev, o1[2]), o1[3] = fmaf(pa.w, ev, o1[3]);
+                o2[0] = fmaf(pb.x, ev, o2[0]), o2[1] = fmaf(pb.y, ev, o2[1]);
+                o2[2] = fmaf(pb.z, ev, o2[2]), o2[3] = fmaf(pb.w, ev, o2[3]);
+            }
+#pragma unroll 4
+            for (int i = r1 + 4; i <= r2 + 3; ++i) {
+                const float ev = U[i * kUS + lane];
+                const float4 pb = *reinterpret_cast<const float4*>(PT + i * kC + r2);
+                o2[0] = fmaf(pb.x, ev, o2[0]), o2[1] = fmaf(pb.y, ev, o2[1]);
+                o2[2] = fmaf(pb.z, ev, o2[2]), o2[3] = fmaf(pb.w, ev, o2[3]);
+            }
+            float* ob = a.out + (((size_t)b * a.L + t0) * a.Hv + h) * kD + col0 + lane;
+            const size_t row_stride = (size_t)a.Hv * kD;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r1 + r < n) ob[(r1 + r) * row_stride] = o1[r];
+                if (r2 + r < n) ob[(r2 + r) * row_stride] = o2[r];
+            }
+        }
+
+        if (__syncthreads_or(wait_parity(&sm.mma, (uint32_t)waits_mma & 1u) ? 0 : 1)) {
+            ok = false;
+            break;
+        }
+        ++waits_mma;
+        tc_fence_after();
+        if (c + 1 < nch) {  // the K^T buffer is free again
+            if (tid == 0) issue_a2(c + 1);
+            ++issued_a2;
+        }
         {
             float v[16];
             tmem_ld16(tmem + lane_base + 32u + (uint32_t)(half * 16), v);
@@ -910,12 +1164,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
                 *reinterpret_cast<float4*>(mrow + j) = m;
             }
         }
-        // Buffer s (E was written into it) is refilled next by the async proxy.
+        // Small buffer s (E was written into it) is refilled next by the async proxy.
         async_proxy_fence();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0 && c + 2 < nch) issue(c + 2);
+        if (c + 2 < nch) {
+            if (tid == 0) issue_small(c + 2);
+            ++issued_small;
+        }
     }
 
     if (ok) {
@@ -925,12 +1182,14 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             *reinterpret_cast<float4*>(MD + (size_t)i * kD + 4 * j4) = *reinterpret_cast<const float4*>(&sm.M[i][4 * j4]);
         }
     } else if (tid == 0) {
-        // Something never arrived: record it, then give the copies and MMAs still
-        // in flight one more bounded wait each before the shared memory and TMEM go.
+        // Something never arrived: record it, then give every copy and MMA still
+        // outstanding one more bounded wait before shared memory and TMEM go.
         record(a.err, GDN_ERR_TIMEOUT);
-        for (int cc = c; cc < min(c + 2, nch); ++cc) wait_parity(&sm.full[cc & 1], (uint32_t)(cc >> 1) & 1u);
-        wait_parity(&sm.mma, 0);
-        wait_parity(&sm.mma, 1);
+        for (; done_small < issued_small; ++done_small)
+            wait_parity(&sm.full[done_small & 1], (uint32_t)(done_small >> 1) & 1u);
+        for (; done_a1 < issued_a1; ++done_a1) wait_parity(&sm.bar_a1, (uint32_t)done_a1 & 1u);
+        for (; done_a2 < issued_a2; ++done_a2) wait_parity(&sm.bar_a2, (uint32_t)done_a2 & 1u);
+        for (; waits_mma < issued_mma; ++waits_mma) wait_parity(&sm.mma, (uint32_t)waits_mma & 1u);
     }
     tc_fence_before();
     __syncthreads();
@@ -971,18 +1230,22 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     const ChunkArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, static_cast<unsigned char*>(workspace),
                       err_word, num_slots, B, L, Hk, Hv, Hv / Hk, nchunks};
     const bool bf = qkv_dtype == GDN_BF16;
-    const int s1 = (int)sizeof(Smem1), s2 = bf ? (int)sizeof(SmemTC) : (int)sizeof(Smem2);
-    cudaError_t e = bf ? cudaFuncSetAttribute(gdn_chunk_prepare_kernel<__nv_bfloat16>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, s1)
+    const int s1 = bf ? (int)sizeof(SmemP) : (int)sizeof(Smem1), s2 = bf ? (int)sizeof(SmemTC) : (int)sizeof(Smem2);
+    cudaError_t e = bf ? cudaFuncSetAttribute(gdn_chunk_prepare_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1)
                        : cudaFuncSetAttribute(gdn_chunk_prepare_kernel<float>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
+    if (bf) {  // three prepare CTAs per SM need the largest shared-memory carveout
+        e = cudaFuncSetAttribute(gdn_chunk_prepare_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return GDN_ERR_CUDA;
+    }
     e = bf ? cudaFuncSetAttribute(gdn_chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s2)
            : cudaFuncSetAttribute(gdn_chunk_scan_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     const unsigned g1 = (unsigned)(B * Hv * nchunks), g2 = (unsigned)(B * Hv * kNCB);
     if (bf) {
-        gdn_chunk_prepare_kernel<__nv_bfloat16><<<g1, kNT, s1, stream>>>(a);
+        gdn_chunk_prepare_tc_kernel<<<g1, kNT, s1, stream>>>(a);
         gdn_chunk_scan_tc_kernel<<<g2, kNT, s2, stream>>>(a);
     } else {
         gdn_chunk_prepare_kernel<float><<<g1, kNT, s1, stream>>>(a);
