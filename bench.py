@@ -571,16 +571,35 @@ def run_prefill(args):
         raise RuntimeError("device error word set during the prefill benchmark")
     us = 1e3 * e0.elapsed_time(e1) / args.steps
     units = B * L * Hv
-    flops = 7.0 * dk * dv * units  # per element: 2 FMA (u, w) + 1 FMA + 1 multiply (update)
     sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
-    peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # fp32 FMA lanes x 2 flop x median clock
     line = {"metric": METRIC, "workload": f"prefill B={B} L={L} Hk={Hk} Hv={Hv} dk=dv={dk}",
             "kernel": "chunked (gdn_prefill_chunked)" if args.chunked else "token steps (gdn_prefill)", "unit": UNIT,
             "value": units / (us / 1e6), "us_per_call": us, "steps": args.steps, "warmup": args.warmup,
-            "roofline": {"bound": "alu", "achieved": flops / us / 1e6, "peak": peak_tflops, "unit": "TFLOP/s",
-                         "frac": flops / us / 1e6 / peak_tflops,
-                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 flop x median SM clock"},
             "clocks": clocks}
+    if args.chunked:
+        # I/O the method must move: q, k, v (bf16), alpha, beta, out (fp32), the initial
+        # state read and the checkpoint written.  The workspace round trip (written by the
+        # prepare kernel, read back by the scan) is reported beside it.
+        hbm_peak, peak_kind = peaks()
+        io = B * L * (2 * Hk * dk * 2 + Hv * dv * 2 + 2 * Hv * 4 + Hv * dv * 4) + 2 * B * Hv * dk * dv * 4
+        ws_bytes = gdn.gdn_prefill_workspace_bytes(B, L, Hv, dk, dv)
+        chunks = (L + 63) // 64
+        C = 64
+        # per (request, head, chunk): K K^T, Q K^T, U = T diag(beta) V, [K;Q] M, Tb (K M),
+        # P E, K^T E, and the triangular inverse
+        flop_chunk = 2 * C * C * dk * 2 + 2 * C * C * dv + 2 * 2 * C * dk * dv + 2 * C * C * dv * 2 \
+            + 2 * C * dk * dv + C ** 3 / 3
+        line["roofline"] = {"bound": "hbm", "achieved": io / us / 1e3, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": io / us / 1e3 / hbm_peak, "peak_kind": peak_kind, "io_bytes": io,
+                            "workspace_bytes": ws_bytes,
+                            "with_workspace_frac": (io + 2 * ws_bytes) / us / 1e3 / hbm_peak}
+        line["chunked_tflops"] = B * Hv * chunks * flop_chunk / us / 1e6
+    else:
+        flops = 7.0 * dk * dv * units  # per element: 2 FMA (u, w) + 1 FMA + 1 multiply (update)
+        peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # fp32 FMA lanes x 2 flop x median clock
+        line["roofline"] = {"bound": "alu", "achieved": flops / us / 1e6, "peak": peak_tflops, "unit": "TFLOP/s",
+                            "frac": flops / us / 1e6 / peak_tflops,
+                            "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 flop x median SM clock"}
     print(json.dumps(line), flush=True)
 
 
