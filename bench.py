@@ -377,6 +377,15 @@ def cpu_baseline(budget_s: float = 12.0, Hv: int = 32):
                       f"tokens*heads), C++ double-precision oracle, {threads} threads, {t:.1f} s"}
 
 
+def headline_config(args, world: int) -> dict:
+    """The `config` object of the large-decode line, shared by both arms."""
+    return {"workload": WORKLOAD, "variant": args.variant, "graph": bool(args.graph),
+            "fused_prologue": bool(args.fused), "B": args.batch, "layers": args.layers, "Hk": 16, "Hv": 32,
+            "dk": 128, "dv": 128, "qkv": "bf16", "state": "f32", "slots_per_layer": args.slots,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (4 GiB of state touched per step), no flush"}
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle, timed for K steps on a bounded per-step sample."""
     rank = int(os.environ.get("RANK", "0"))
@@ -399,9 +408,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_requests_per_step": n_req, "layers_per_step": 1},
+        "config": headline_config(args, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"each step: one in-place call on {n_req} requests of layer 0"},
+                         "sample": f"each step: one in-place call on {n_req} of the {args.batch} requests of "
+                                   f"layer 0 ({n_req * 32} tokens*heads), C++ double-precision oracle"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -721,11 +731,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "variant": args.variant, "graph": bool(args.graph),
-                   "fused_prologue": bool(args.fused), "B": wk.B, "layers": L, "Hk": wk.Hk, "Hv": wk.Hv, "dk": wk.dk,
-                   "dv": wk.dv, "qkv": "bf16", "state": "f32", "slots_per_layer": wk.num_slots,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (4 GiB of state touched per step), no flush"},
+        "config": headline_config(args, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy bandwidth", "kernel": kernel,
