@@ -110,13 +110,26 @@ def _ptr_or_null(t: Optional[torch.Tensor], name: str) -> Optional[int]:
     return None if t is None else _dev(t, name, torch.int32)
 
 
-def _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out):
+def _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=None):
+    """Pointers and sizes for the decode and prefill entry points.  The library sees plain
+    pointers, so every tensor's shape is checked against pool and q here: a mismatch
+    would otherwise read or write past a buffer.  dst_idx holds dst_per_request entries
+    per request (T by default; 1 for a prefill)."""
     if pool.dim() != 4 or q.dim() != 4 or v.dim() != 4:
         raise ValueError("pool, q, k, v must be 4-D")
     num_slots, Hv, dk, dv = pool.shape
     B, T, Hk = q.shape[0], q.shape[1], q.shape[2]
     if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype: bfloat16 or float32")
+    want = {"q": (B, T, Hk, dk), "k": (B, T, Hk, dk), "v": (B, T, Hv, dv), "alpha": (B, T, Hv),
+            "beta": (B, T, Hv), "out": (B, T, Hv, dv)}
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta), ("out", out)):
+        if tuple(t.shape) != want[name]:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want[name]} from pool {tuple(pool.shape)}"
+                             f" and q {tuple(q.shape)}")
+    per = T if dst_per_request is None else dst_per_request
+    if src_idx.numel() != B or dst_idx.numel() != B * per:
+        raise ValueError(f"src_idx must hold B = {B} entries and dst_idx B * {per}")
     return (_dev(pool, "pool", torch.float32), int(num_slots),
             _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32),
             _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
@@ -180,9 +193,7 @@ def gdn_prefill(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor
     """Enqueue a prefill (see gdn_prefill in include/gdn_step.h): q, k [B, L, Hk, dk],
     v [B, L, Hv, dv], alpha/beta [B, L, Hv], out [B, L, Hv, dv]; only the state after the
     last token is stored, to pool[dst_idx[b]] (dst_idx [B])."""
-    if dst_idx.numel() != src_idx.numel():
-        raise ValueError("dst_idx must hold one slot per request")
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1)
     status = load_library().gdn_prefill(*args, _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_prefill")
@@ -199,9 +210,7 @@ def gdn_prefill_chunked(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torc
                         err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
     """gdn_prefill computed chunk by chunk (see gdn_prefill_chunked in include/gdn_step.h);
     ``workspace`` is a CUDA tensor of at least gdn_prefill_workspace_bytes(...) bytes."""
-    if dst_idx.numel() != src_idx.numel():
-        raise ValueError("dst_idx must hold one slot per request")
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1)
     nbytes = workspace.numel() * workspace.element_size()
     status = load_library().gdn_prefill_chunked(*args, _dev(workspace, "workspace"), nbytes,
                                                 _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
@@ -219,6 +228,8 @@ def gdn_commit(accept_len: torch.Tensor, committed: torch.Tensor, cur: torch.Ten
     if cur.dim() != 2:
         raise ValueError("cur must be [B, T]")
     B, T = cur.shape
+    if accept_len.numel() != B or committed.numel() != B:
+        raise ValueError("accept_len and committed must hold B entries")
     status = load_library().gdn_commit(
         _dev(accept_len, "accept_len", torch.int32), _dev(committed, "committed", torch.int32),
         _dev(cur, "cur", torch.int32), int(B), int(T), int(num_slots),

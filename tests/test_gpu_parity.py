@@ -279,6 +279,31 @@ def test_invalid_arguments_raise(torch_cuda):
         gdn.gdn_decode_step(pool, x["src"], x["dst"], x["q"], x["k"], x["v"].float(), x["alpha"], x["beta"], out)
 
 
+def test_mismatched_shapes_are_rejected_by_the_binding(torch_cuda):
+    """The library takes plain pointers and cannot see buffer sizes; the binding checks every
+    tensor's shape against pool and q before anything is enqueued."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    s = wl.decode_b16().steps[0]
+    x = step_to_device(s)
+    pool = torch.zeros((64, 32, 128, 128), device="cuda")
+    out = torch.zeros((16, 1, 32, 128), device="cuda")
+    good = dict(pool=pool, src_idx=x["src"], dst_idx=x["dst"], q=x["q"], k=x["k"], v=x["v"], alpha=x["alpha"],
+                beta=x["beta"], out=out)
+    bad = {"k": x["k"][:8], "v": x["v"][:, :, :16], "alpha": x["alpha"][:, :, :8], "out": out[:, :, :, :64],
+           "dst_idx": x["dst"][:8], "src_idx": x["src"][:4]}
+    for name, t in bad.items():
+        with pytest.raises(ValueError):
+            gdn.gdn_decode_step(**{**good, name: t.contiguous()})
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):  # a prefill takes one destination per request
+        gdn.gdn_prefill_chunked(**{**good, "dst_idx": torch.zeros(32, dtype=torch.int32, device="cuda")},
+                                workspace=ws)
+    torch.cuda.synchronize()
+    assert not bool(pool.any())  # nothing ran
+
+
 def test_variant_conditions_are_checked(torch_cuda):
     torch = torch_cuda
     from hybrid_linear_attention_step_b200 import gdn
