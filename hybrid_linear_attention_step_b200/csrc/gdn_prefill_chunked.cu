@@ -856,13 +856,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 
 // ---------------------------------------------------------------------------
 // Kernel 2, tensor-core form (bf16 inputs).  Per chunk:
-//   D1 = [K; Q] M      (M=128: rows 0..63 are K M, rows 64..127 Q M; N = kDVC;
-//                       K = dk in 8 steps; M split into 3 bf16 parts -> 24 MMAs)
-//   D2 = K^T E'        (M=128 rows of dk, N = kDVC, K = 64 tokens in 4 steps,
-//                       E' = diag(g_C / g) E split into 3 bf16 parts -> 12 MMAs)
-// Operands sit in shared memory in the no-swizzle K-major core layout;
-// accumulators live in 64 TMEM columns (D1 at column 0, D2 at column 32)
-// allocated by warp 0.  Thread 0 issues the MMAs, commits them to an mbarrier,
+//   D1 = [K; Q] [M_hi M_mid M_lo]  (M=128: rows 0..63 K, rows 64..127 Q; the fp32
+//                                   state block split into three bf16 parts stacked
+//                                   along N = 3 x 32; K = dk in 8 steps: 8 MMAs)
+//   D2 = K^T [E'_hi E'_mid E'_lo]  (M=128 rows of dk, N = 3 x 32, K = 64 tokens in
+//                                   4 steps, E' = diag(g_C / g) E: 4 MMAs)
+// The three column groups of each accumulator are added when TMEM is read, so the
+// A tile is read once per k-step for all three parts.  Operands sit in shared
+// memory in the no-swizzle K-major core layout; the accumulators take 2 x 96 of
+// 256 TMEM columns (D1 at column 0, D2 at column 128) allocated by warp 0.  Thread 0 issues the MMAs, commits them to an mbarrier,
 // and streams the chunk images with cp.async.bulk: the MMA operands [K; Q] and
 // K^T (one buffer each, refilled for the next chunk as soon as their MMAs
 // complete) and the small image (U slab, Tb^T, P^T, log g; two buffers, two
@@ -871,13 +873,16 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 // step over i reads one KM (or E) value and two broadcast float4 of Tb^T (P^T).
 // Every wait is bounded (2 s); a timeout is recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;  // one bf16 part of M^T (32 x 128)
+constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;   // one bf16 part of M^T (32 x 128)
+constexpr uint32_t kBopPartE = (uint32_t)kDVC * kC * 2;  // one bf16 part of E'^T (32 x 64)
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemD2 = 128;
 
 struct SmemTC {
     unsigned char a1[2 * kC * kD * 2];  // [K; Q] operand of D1
     unsigned char a2[kD * kC * 2];      // K^T operand of D2
     unsigned char img[2][kImgBytes];    // small images, double-buffered
-    unsigned char bop[3][kBopPart];     // B operand parts: M^T, later E'^T (32 x 64, same slots)
+    unsigned char bop[3 * kBopPart];    // B operand, three stacked parts: M^T, later E'^T
     float M[kD][kUS];                   // state block [dk][32 columns]
     float KM[kC][kUS];
     float QM[kC][kUS];                  // g Q M
@@ -897,7 +902,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
     const int col0 = cb * kDVC;
-    constexpr uint32_t kIdesc = umma_idesc(128, kDVC);
+    constexpr uint32_t kIdesc = umma_idesc(128, 3 * kDVC);
     const int nch = a.nchunks;
 
     // Thread 0's copies.  Every barrier completes once per chunk (or once per
@@ -938,7 +943,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     if (sm.status != 0) return;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
-                     "r"(64)
+                     "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -991,20 +996,17 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             uint4 p0, p1, p2;
             split3x8(x, p0, p1, p2);
             const uint32_t off = core_off(jj, 8 * g, kD);
-            *reinterpret_cast<uint4*>(sm.bop[0] + off) = p0;
-            *reinterpret_cast<uint4*>(sm.bop[1] + off) = p1;
-            *reinterpret_cast<uint4*>(sm.bop[2] + off) = p2;
+            *reinterpret_cast<uint4*>(sm.bop + off) = p0;
+            *reinterpret_cast<uint4*>(sm.bop + kBopPart + off) = p1;
+            *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPart + off) = p2;
         }
         async_proxy_fence();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            for (int part = 0; part < 3; ++part) {
-                const uint64_t db = umma_desc(smem_u32(sm.bop[part]), (kD / 8) * 128);
-                for (int ks = 0; ks < kD / 16; ++ks)
-                    umma_bf16(tmem, da1 + 16 * ks, db + 16 * ks, kIdesc, (part | ks) != 0 ? 1u : 0u);
-            }
+            const uint64_t db = umma_desc(smem_u32(sm.bop), (kD / 8) * 128);
+            for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(tmem, da1 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
             umma_commit(&sm.mma);
         }
         ++issued_mma;
@@ -1020,8 +1022,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             ++issued_a1;
         }
         {
-            float v[16];
+            float v[16], v1[16], v2[16];
             tmem_ld16(tmem + lane_base + (uint32_t)(half * 16), v);
+            tmem_ld16(tmem + lane_base + (uint32_t)(kDVC + half * 16), v1);
+            tmem_ld16(tmem + lane_base + (uint32_t)(2 * kDVC + half * 16), v2);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += v1[j] + v2[j];
             const int row = (warp % 4) * 32 + lane;
             float* dstrow;
             float g = 1.f;
@@ -1083,9 +1089,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             uint4 p0, p1, p2;
             split3x8(x, p0, p1, p2);
             const uint32_t off = core_off(jj, 8 * g, kC);
-            *reinterpret_cast<uint4*>(sm.bop[0] + off) = p0;
-            *reinterpret_cast<uint4*>(sm.bop[1] + off) = p1;
-            *reinterpret_cast<uint4*>(sm.bop[2] + off) = p2;
+            *reinterpret_cast<uint4*>(sm.bop + off) = p0;
+            *reinterpret_cast<uint4*>(sm.bop + kBopPartE + off) = p1;
+            *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPartE + off) = p2;
         }
         got = wait_parity(&sm.bar_a2, (uint32_t)c & 1u);
         async_proxy_fence();
@@ -1097,11 +1103,9 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         ++done_a2;
         tc_fence_after();
         if (tid == 0) {
-            for (int part = 0; part < 3; ++part) {
-                const uint64_t db = umma_desc(smem_u32(sm.bop[part]), (kC / 8) * 128);
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem + 32, da2 + 16 * ks, db + 16 * ks, kIdesc, (part | ks) != 0 ? 1u : 0u);
-            }
+            const uint64_t db = umma_desc(smem_u32(sm.bop), (kC / 8) * 128);
+            for (int ks = 0; ks < kC / 16; ++ks)
+                umma_bf16(tmem + kTmemD2, da2 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
             umma_commit(&sm.mma);
         }
         ++issued_mma;
@@ -1151,8 +1155,12 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             ++issued_a2;
         }
         {
-            float v[16];
-            tmem_ld16(tmem + lane_base + 32u + (uint32_t)(half * 16), v);
+            float v[16], v1[16], v2[16];
+            tmem_ld16(tmem + lane_base + kTmemD2 + (uint32_t)(half * 16), v);
+            tmem_ld16(tmem + lane_base + kTmemD2 + (uint32_t)(kDVC + half * 16), v1);
+            tmem_ld16(tmem + lane_base + kTmemD2 + (uint32_t)(2 * kDVC + half * 16), v2);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += v1[j] + v2[j];
             const int i = (warp % 4) * 32 + lane;  // dk row
             const float gC = expf(lg[kC - 1]);
             float* mrow = &sm.M[i][half * 16];
@@ -1195,7 +1203,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
 }  // namespace
