@@ -258,50 +258,56 @@ __device__ __forceinline__ void gate_scan(const ChunkArgs& a, int b, int h, int 
     }
 }
 
-// T = (I + A)^-1 for strictly lower-triangular A (all threads; A complete on
-// entry, T complete on return).  Blocked in 16 x 16: diagonal blocks by forward
-// substitution (one warp each), then block rows I = 1..3:
-// T_IJ = -T_II sum_{J<=K<I} A_IK T_KJ.
+// T = (I + A)^-1 for strictly lower-triangular A (all threads; A complete and zero
+// on and above the diagonal on entry, T complete on return).  Blocked in 16 x 16:
+// diagonal blocks by forward substitution (one warp each, lane j owns column j),
+// then block rows I = 1..3: T_I,<I = -T_II (A_I,<I T_<I,<I).  Every dot product runs
+// over a fixed, unrolled length: the terms beyond the triangle are exact zeros (A
+// above its diagonal, T above its diagonal, which starts zeroed), so no loop bound
+// depends on the lane and the loads pipeline.
 __device__ __forceinline__ void invert_unit_lower(const float (*A)[kC + 1], float (*T)[kC + 1], float (*Y)[48],
                                                   int tid) {
     const int w = tid / 32, lane = tid % 32;
-    if (w < 4) {
-        const int o = w * 16;
+    for (int e = tid; e < kC * kC; e += kNT) T[e / kC][e % kC] = 0.f;
+    __syncthreads();
+    if (w < 4 && lane < 16) {
+        const int o = w * 16, j = lane;
         for (int r = 0; r < 16; ++r) {
-            if (lane < 16) {
-                const int j = lane;
-                float val = (r == j) ? 1.f : 0.f;
-                if (j < r) {
-                    float acc = 0.f;
-                    for (int m = j; m < r; ++m) acc = fmaf(A[o + r][o + m], T[o + m][o + j], acc);
-                    val = -acc;
-                }
-                T[o + r][o + j] = val;
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; m += 2) {
+                acc0 = fmaf(A[o + r][o + m], T[o + m][o + j], acc0);
+                acc1 = fmaf(A[o + r][o + m + 1], T[o + m + 1][o + j], acc1);
             }
-            __syncwarp();
+            T[o + r][o + j] = (r == j ? 1.f : 0.f) - (acc0 + acc1);
+            __syncwarp(0x0000ffffu);
         }
-    }
-    // zero the strictly upper blocks
-    for (int e = tid; e < kC * kC; e += kNT) {
-        const int r = e / kC, j = e % kC;
-        if (j / 16 > r / 16) T[r][j] = 0.f;
     }
     __syncthreads();
+#pragma unroll
     for (int I = 1; I < 4; ++I) {
-        // Y[r][J*16 + j] = sum_{K=J}^{I-1} sum_m A[16I + r][16K + m] T[16K + m][16J + j]
+        // Y[r][col] = sum_{kk < 16 I} A[16 I + r][kk] T[kk][col], col < 16 I
         for (int e = tid; e < 16 * 16 * I; e += kNT) {
             const int r = e / (16 * I), col = e % (16 * I);
-            const int J = col / 16, j = col % 16;
-            float acc = 0.f;
-            for (int kk2 = 16 * J; kk2 < 16 * I; ++kk2) acc = fmaf(A[16 * I + r][kk2], T[kk2][16 * J + j], acc);
-            Y[r][col] = acc;
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 16 * I; kk += 2) {
+                acc0 = fmaf(A[16 * I + r][kk], T[kk][col], acc0);
+                acc1 = fmaf(A[16 * I + r][kk + 1], T[kk + 1][col], acc1);
+            }
+            Y[r][col] = acc0 + acc1;
         }
         __syncthreads();
+        // T[16 I + r][col] = -sum_m T[16 I + r][16 I + m] Y[m][col]
         for (int e = tid; e < 16 * 16 * I; e += kNT) {
             const int r = e / (16 * I), col = e % (16 * I);
-            float acc = 0.f;
-            for (int m = 0; m <= r; ++m) acc = fmaf(T[16 * I + r][16 * I + m], Y[m][col], acc);
-            T[16 * I + r][col] = -acc;
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; m += 2) {
+                acc0 = fmaf(T[16 * I + r][16 * I + m], Y[m][col], acc0);
+                acc1 = fmaf(T[16 * I + r][16 * I + m + 1], Y[m + 1][col], acc1);
+            }
+            T[16 * I + r][col] = -(acc0 + acc1);
         }
         __syncthreads();
     }
