@@ -176,7 +176,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
-__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
+// Bounded wait for the completion of the mbarrier phase with this parity: false
+// once limit_ns of global time have passed without it (2 s in every pipeline).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     uint32_t done = 0;
     uint64_t t0;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
@@ -190,7 +193,7 @@ __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity) {
         if (done) return true;
         uint64_t t1;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
-        if (t1 - t0 > 2000000000ull) return false;  // 2 s
+        if (t1 - t0 > limit_ns) return false;
     }
 }
 
@@ -1212,7 +1215,26 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
+// Self-test of the bounded wait: one CTA waits on an mbarrier that nothing ever
+// arrives on, with the given limit, and records GDN_ERR_TIMEOUT when it gives up.
+__global__ void gdn_wait_selftest_kernel(uint64_t limit_ns, int32_t* err) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const bool got = wait_parity(&bar, 0u, limit_ns);
+    if (__syncthreads_or(got ? 0 : 1) && threadIdx.x == 0) record(err, GDN_ERR_TIMEOUT);
+}
+
 }  // namespace
+
+extern "C" gdn_status gdn_wait_selftest(uint64_t limit_ns, int32_t* err_word, cudaStream_t stream) {
+    if (err_word == nullptr || limit_ns == 0 || limit_ns > kWaitLimitNs) return GDN_ERR_INVALID_ARG;
+    gdn_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, err_word);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
 
 extern "C" size_t gdn_prefill_workspace_bytes(int32_t B, int32_t L, int32_t Hv, int32_t dk, int32_t dv) {
     if (B < 0 || L < 1 || Hv < 1 || dk != kD || dv != kD) return 0;

@@ -78,6 +78,8 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_commit.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
     lib.gdn_check_step.restype = i32
     lib.gdn_check_step.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+    lib.gdn_wait_selftest.restype = i32
+    lib.gdn_wait_selftest.argtypes = [ctypes.c_uint64, vp, vp]
     lib.gdn_get_error.restype = i32
     lib.gdn_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     lib.gdn_status_string.restype = ctypes.c_char_p
@@ -255,6 +257,16 @@ def gdn_check_step(src_idx: torch.Tensor, dst_idx: torch.Tensor, num_slots: int,
         _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_check_step")
+    return status
+
+
+def gdn_wait_selftest(limit_ns: int, err_word: torch.Tensor, stream=None, check: bool = True) -> int:
+    """Enqueue the bounded-wait self-test (see gdn_wait_selftest in include/gdn_step.h):
+    a wait on an mbarrier nothing arrives on, which records GDN_ERR_TIMEOUT after limit_ns."""
+    status = load_library().gdn_wait_selftest(int(limit_ns), _dev(err_word, "err_word", torch.int32),
+                                              _stream_handle(stream))
+    if check and status != GDN_OK:
+        raise GdnError(status, "gdn_wait_selftest")
     return status
 
 

@@ -82,9 +82,9 @@ typedef enum gdn_variant {
     GDN_VARIANT_STREAM = 1, /* persistent bulk-copy pipeline through shared memory: T == 1,
                                dk == dv == 128, every buffer 16-byte aligned, B*Hv % 4 == 0 */
     GDN_VARIANT_TILE = 2,   /* state tile held in registers: (dk, dv) in {(128, 128), (64, 64)},
-                               pool and out 16-byte aligned, any T (T == 1: one CTA per 64-column
-                               block of a (request, head) tile; T > 1: one CTA per tile, carried
-                               across the tokens) */
+                               pool and out 16-byte aligned, any T; one CTA per 64-column block
+                               of a (request, head) tile, which for T > 1 carries its columns
+                               across the tokens */
     GDN_VARIANT_COLUMN = 3  /* one thread per value column: any shape and alignment */
 } gdn_variant;
 
@@ -308,6 +308,23 @@ gdn_status gdn_check_step(const int32_t* src_idx, const int32_t* dst_idx, int32_
 #define GDN_CHECK_NOALLOC_MAX_SLOTS (1 << 18)
 gdn_status gdn_check_step_noalloc(const int32_t* src_idx, const int32_t* dst_idx, int32_t B, int32_t T,
                                   int32_t num_slots, int32_t* err_word, cudaStream_t stream);
+
+/*
+ * gdn_wait_selftest -- exercise the bounded wait of the copy and MMA pipelines.
+ *
+ * No counterpart on the source pages: a self-test of this library's failure
+ * detection.  The bulk-copy pipelines (the STREAM decode variant, the chunked
+ * prefill) wait on mbarriers with a limit on global time; a wait that runs out
+ * records GDN_ERR_TIMEOUT and the kernel drains and returns instead of hanging.
+ * This call runs that same wait in one CTA on an mbarrier that nothing arrives
+ * on, so it always runs out after limit_ns nanoseconds and records
+ * GDN_ERR_TIMEOUT in *err_word.  Nothing faults; the context stays usable.
+ *
+ *   limit_ns   1 .. 2,000,000,000 (the pipelines' own limit is the maximum)
+ *   err_word   device int32, required
+ * Returns GDN_ERR_INVALID_ARG for a null err_word or a limit out of range.
+ */
+gdn_status gdn_wait_selftest(uint64_t limit_ns, int32_t* err_word, cudaStream_t stream);
 
 /*
  * gdn_get_error -- read and clear a device error word.

@@ -104,3 +104,12 @@ def test_product_path_never_imports_the_oracle():
         text = p.read_text()
         assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), p
         assert "gdn_oracle" not in text, p
+
+
+def test_wait_selftest_validates_on_the_host(lib):
+    f = lib.gdn_wait_selftest
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]
+    assert f(1000, None, None) == 1          # no error word
+    assert f(0, 8, None) == 1                # empty limit
+    assert f(2_000_000_001, 8, None) == 1    # above the pipelines' own limit

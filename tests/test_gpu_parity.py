@@ -685,3 +685,26 @@ def test_prefill_chunked_edge_cases(torch_cuda):
     o = out.cpu().numpy()
     assert np.all(o[[1, 3]] == -7.0)
     assert rel_err(o[[0, 2]], ref_out[[0, 2]]) <= TOL_OUT_BF16
+
+
+def test_bounded_wait_runs_out_and_reports_timeout(torch_cuda):
+    """The pipelines' bounded mbarrier wait, run on a barrier that nothing arrives on:
+    it gives up after its limit, records GDN_ERR_TIMEOUT, and the context stays usable."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gdn.gdn_wait_selftest(20_000_000, err)  # 20 ms
+    e1.record()
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_error(err) == gdn.GDN_ERR_TIMEOUT
+    assert e0.elapsed_time(e1) >= 19.0
+    w = wl.decode_b16()
+    dev = to_torch(w.pool)
+    out = run_gpu(dev, w.steps[0], err=err)
+    ref_pool, ref_out, _ = run_oracle(w.pool, w.steps[0])
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    check_pool(dev.cpu().numpy(), ref_pool, w.pool, w.steps[0].dst_idx)
+    assert rel_err(out, ref_out) <= TOL_OUT_BF16
