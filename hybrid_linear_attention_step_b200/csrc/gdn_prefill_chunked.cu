@@ -29,13 +29,14 @@
 // overflows; g_t itself may underflow to zero, which is its true value to fp32
 // precision.
 //
-// Workspace record of one (request, head, chunk), bytes, laid out as the
-// shared-memory images kernel 2 copies in (bulk copies, 16-byte granules):
-//   A1  [K; Q] as bf16, 128 rows x 128 (dk) in the no-swizzle K-major core
-//       layout of the tensor-core operand (bf16 inputs only)
+// Workspace record of one (request, head, chunk), bytes.  The first parts are laid
+// out as the shared-memory images the scan copies in (bulk copies, 16-byte granules):
+//   A1  [W_hi; W_mid] then [W_lo; Q] as bf16, two 128 x 128 (dk) tiles in the
+//       no-swizzle K-major core layout of the tensor-core operand, where
+//       W = Tb K is split into three bf16 parts (bf16 inputs only)
 //   A2  K^T as bf16, 128 (dk) rows x 64 tokens, same layout (bf16 inputs only)
 //   U   four column slabs [4][64][36] fp32 (32 columns + 4 padding each)
-//   TbT [64][64] fp32: Tb transposed, TbT[i][t] = Tb[t][i], zero for t < i
+//   TbT [64][64] fp32: Tb transposed, TbT[i][t] = Tb[t][i], zero for t < i (fp32 inputs)
 //   PT  [64][64] fp32: P transposed, PT[i][t] = P[t][i], zero for t < i
 //   G   log g [64]
 
@@ -57,19 +58,21 @@ constexpr int kPad = 4;         // row padding of [C][D] shared arrays in the fp
 
 // Workspace record (bytes).
 constexpr size_t kRecA1 = 0;
-constexpr size_t kRecA2 = kRecA1 + (size_t)2 * kC * kD * 2;
+constexpr size_t kA1Tile = (size_t)2 * kC * kD * 2;  // one 128 x 128 bf16 operand tile
+constexpr size_t kRecA2 = kRecA1 + 2 * kA1Tile;
 constexpr size_t kRecU = kRecA2 + (size_t)kD * kC * 2;
 constexpr size_t kUSlab = (size_t)kC * kUS * 4;
 constexpr size_t kRecTb = kRecU + kNCB * kUSlab;
 constexpr size_t kRecP = kRecTb + (size_t)kC * kC * 4;
 constexpr size_t kRecG = kRecP + (size_t)kC * kC * 4;
 constexpr size_t kRecBytes = kRecG + (size_t)kC * 4;
-// One CTA's small image of a chunk in shared memory: its U slab | TbT PT G.
-constexpr uint32_t kImgTb = (uint32_t)kUSlab;
-constexpr uint32_t kImgP = kImgTb + (uint32_t)(kRecP - kRecTb);
-constexpr uint32_t kImgG = kImgP + (uint32_t)(kRecG - kRecP);
-constexpr uint32_t kImgBytes = kImgG + (uint32_t)(kRecBytes - kRecG);
-static_assert(kRecA2 % 16 == 0 && kRecU % 16 == 0 && kRecTb % 16 == 0 && kRecBytes % 16 == 0, "16-byte records");
+// One scan CTA's small image of a chunk in shared memory: its U slab | P^T | log g.
+constexpr uint32_t kImgP = (uint32_t)kUSlab;
+constexpr uint32_t kImgG = kImgP + (uint32_t)(kC * kC * 4);
+constexpr uint32_t kImgBytes = kImgG + (uint32_t)(kC * 4);
+static_assert(kRecG == kRecP + (size_t)kC * kC * 4, "P^T and log g are copied together");
+static_assert(kRecA2 % 16 == 0 && kRecU % 16 == 0 && kRecTb % 16 == 0 && kRecP % 16 == 0 && kRecBytes % 16 == 0,
+              "16-byte records");
 static_assert(kUSlab % 16 == 0 && kImgBytes % 16 == 0, "16-byte bulk copies");
 
 struct ChunkArgs {
@@ -440,25 +443,34 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 1, tensor-core form (bf16 inputs).  The products whose operands are the
-// chunk's bf16 inputs run as tcgen05 MMAs with fp32 accumulation in TMEM:
-//   D0 = [K; Q] K^T                 (M = 128, N = 64, K = dk: 8 MMAs, exact products)
-//   D1 = V^T (T diag(beta))^T = U^T (M = 128 = dv, N = 64, K = 64 tokens; the fp32
-//                                    factor in three bf16 parts: 12 MMAs)
-// The inverse T and the elementwise gate scalings stay on the CUDA cores.
+// Kernel 1, tensor-core form (bf16 inputs).  The products with a bf16 input
+// operand run as tcgen05 MMAs with fp32 accumulation in TMEM:
+//   D0 = [K; Q] K^T                    (M = 128, N = 64, K = dk: 8 MMAs, exact products)
+//   D1 = V^T (T diag(beta))^T = U^T    (M = 128 = dv, N = 64, K = 64 tokens; the fp32
+//                                       factor in three bf16 parts: 12 MMAs)
+//   D2 = K^T (T diag(beta g))^T = W^T  (the same with Tb: W = Tb K, 12 MMAs)
+// W is split into three bf16 parts and stored as the scan's A operands
+// [W_hi; W_mid] and [W_lo; Q], so that the scan forms E = U - W M0 and Q M0 on the
+// tensor cores with no triangular product.  The inverse T and the gate scalings
+// stay on the CUDA cores.
 // ---------------------------------------------------------------------------
 struct SmemP {
     union {
-        unsigned char A1[2 * kC * kD * 2];     // [K; Q] operand (also B = K of D0)
-        float Y[16][48];                       // scratch of the inverse (after D0)
+        unsigned char A1[2 * kC * kD * 2];        // [K; Q] operand of D0 (also B = K)
+        float Y[16][48];                          // scratch of the inverse (after D0)
         struct {
-            unsigned char VT[kD * kC * 2];     // V^T operand of D1
-            unsigned char Bp[3][kC * kC * 2];  // (T diag(beta)) parts, B of D1
+            unsigned char VT[kD * kC * 2];        // V^T operand of D1
+            unsigned char Bp[3][kC * kC * 2];     // (T diag(beta)) parts, B of D1
         } d1;
+        struct {
+            unsigned char KT[kD * kC * 2];        // K^T operand of D2
+            unsigned char Bt[3][kC * kC * 2];     // (T diag(beta g)) parts, B of D2
+        } d2;
+        float W[kC][kD + 4];                      // W staged for its split (row stride spreads banks)
     } op;
     union {
         float A[kC][kC + 1];
-        __nv_bfloat16 Vb[kC][kD + 2];  // V rows after the inverse (odd word stride for the column gathers)
+        __nv_bfloat16 R[kC][kD + 2];  // V rows, later K rows (odd word stride for the column gathers)
     } av;
     float T[kC][kC + 1];
     float lg[kC];
@@ -467,6 +479,44 @@ struct SmemP {
     uint32_t tmem;
 };
 static_assert(sizeof(SmemP) <= 74 * 1024 + 1024, "three prepare CTAs per SM");
+
+// Column gather of a bf16 row block R (rows = tokens) into a K-major operand image
+// with kD rows (dk or dv) and kC columns (tokens); optionally also to global memory.
+// Consecutive threads write consecutive 16-byte granules.
+__device__ __forceinline__ void gather_transposed(const __nv_bfloat16 (*R)[kD + 2], unsigned char* img,
+                                                  unsigned char* global_img, int tid) {
+    for (int e = tid; e < kD * (kC / 8); e += kNT) {
+        const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // row j, tokens 8g..8g+7
+        uint16_t x[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint16_t*>(&R[8 * g + m][j]);
+        uint4 w;
+        w.x = x[0] | ((uint32_t)x[1] << 16);
+        w.y = x[2] | ((uint32_t)x[3] << 16);
+        w.z = x[4] | ((uint32_t)x[5] << 16);
+        w.w = x[6] | ((uint32_t)x[7] << 16);
+        const uint32_t off = core_off(j, 8 * g, kC);
+        *reinterpret_cast<uint4*>(img + off) = w;
+        if (global_img != nullptr) *reinterpret_cast<uint4*>(global_img + off) = w;
+    }
+}
+
+// B operand (rows t, columns i) = T[t][i] * scale[i], in three bf16 parts.
+__device__ __forceinline__ void split_scaled_T(const float (*T)[kC + 1], const float* scale,
+                                               unsigned char (*parts)[kC * kC * 2], int tid) {
+    for (int e = tid; e < kC * (kC / 8); e += kNT) {
+        const int t = e % kC, g = e / kC;
+        float x[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) x[m] = T[t][8 * g + m] * scale[8 * g + m];
+        uint4 p0, p1, p2;
+        split3x8(x, p0, p1, p2);
+        const uint32_t off = core_off(t, 8 * g, kC);
+        *reinterpret_cast<uint4*>(parts[0] + off) = p0;
+        *reinterpret_cast<uint4*>(parts[1] + off) = p1;
+        *reinterpret_cast<uint4*>(parts[2] + off) = p2;
+    }
+}
 
 __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_p[];
@@ -481,11 +531,12 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     const int t0 = c * kC;
     const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
     unsigned char* rec = record_of(a, bh, c);
-    float* TbT = reinterpret_cast<float*>(rec + kRecTb);
     float* PT = reinterpret_cast<float*>(rec + kRecP);
     float* Gs = reinterpret_cast<float*>(rec + kRecG);
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const int half = warp / 4;  // TMEM columns 32*half .. +31 of each accumulator
+    constexpr uint32_t kIdesc = umma_idesc(128, kC);
+    constexpr uint32_t kTmemU = 64;  // D1; D0 and then D2 use columns 0..63
 
     if (tid == 0) {
         mbar_init(&sm.mma);
@@ -498,9 +549,9 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, Gs);
     }
-    // k, q, v in 16-byte granules: [K; Q] into the operand image (shared memory and the
-    // record, where kernel 2 reads it); V stays in registers until the inverse is done.
-    // Consecutive threads take consecutive granules of the image: token
+    // k, q, v in 16-byte granules: [K; Q] into the D0 operand image, Q also into the
+    // record's [W_lo; Q] tile (rows 64..127); V stays in registers until the inverse is
+    // done.  Consecutive threads take consecutive granules of the image: token
     // t = (e & 7) + 8 (e >> 7), group g = (e >> 3) & 15, e = tid + 256 u.
     constexpr int kGr = kC * (kD / 8) / kNT;  // granules per thread
     uint4 vkeep[kGr];
@@ -516,11 +567,10 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             qq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row));
             vv = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + vrow));
         }
-        const uint32_t ok = core_off(t, 8 * g, kD), oq = core_off(kC + t, 8 * g, kD);
-        *reinterpret_cast<uint4*>(sm.op.A1 + ok) = kq;
+        const uint32_t oq = core_off(kC + t, 8 * g, kD);
+        *reinterpret_cast<uint4*>(sm.op.A1 + core_off(t, 8 * g, kD)) = kq;
         *reinterpret_cast<uint4*>(sm.op.A1 + oq) = qq;
-        *reinterpret_cast<uint4*>(rec + kRecA1 + ok) = kq;
-        *reinterpret_cast<uint4*>(rec + kRecA1 + oq) = qq;
+        *reinterpret_cast<uint4*>(rec + kRecA1 + kA1Tile + oq) = qq;
         vkeep[u] = vv;
     }
     async_proxy_fence();
@@ -528,7 +578,6 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    constexpr uint32_t kIdesc = umma_idesc(128, kC);
     if (tid == 0) {
         const uint32_t a1 = smem_u32(sm.op.A1);
         for (int ks = 0; ks < kD / 16; ++ks)
@@ -536,22 +585,10 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                       kIdesc, ks != 0 ? 1u : 0u);
         umma_commit(&sm.mma);
     }
-    // K^T image for kernel 2, gathered from the K rows of the [K; Q] image:
-    // granule (dk row d, tokens 8 g' .. 8 g' + 7); consecutive threads write consecutive granules.
-    for (int e = tid; e < kD * (kC / 8); e += kNT) {
-        const int d = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;
-        uint16_t x[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) x[j] = *reinterpret_cast<const uint16_t*>(sm.op.A1 + core_off(8 * g + j, d, kD));
-        uint4 w;
-        w.x = x[0] | ((uint32_t)x[1] << 16);
-        w.y = x[2] | ((uint32_t)x[3] << 16);
-        w.z = x[4] | ((uint32_t)x[5] << 16);
-        w.w = x[6] | ((uint32_t)x[7] << 16);
-        *reinterpret_cast<uint4*>(rec + kRecA2 + core_off(d, 8 * g, kC)) = w;
-    }
+    int waits = 0, issued = 1;
     bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
     if (ok) {
+        ++waits;
         tc_fence_after();
         // D0 row r < 64: k_r . k_i -> A (scaled); row 64 + t: q_t . k_i -> P (record).
         const int r = (warp % 4) * 32 + lane;
@@ -585,36 +622,15 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         for (int u = 0; u < kGr; ++u) {
             const int e = tid + kNT * u;
             const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-            uint32_t* vr = reinterpret_cast<uint32_t*>(&sm.av.Vb[t][8 * g]);
+            uint32_t* vr = reinterpret_cast<uint32_t*>(&sm.av.R[t][8 * g]);
             vr[0] = vkeep[u].x, vr[1] = vkeep[u].y, vr[2] = vkeep[u].z, vr[3] = vkeep[u].w;
         }
+        if (tid < kC) sm.lg[tid] = sm.bt[tid] * expf(sm.lg[tid]);  // beta g: log g is in the record already
         __syncthreads();
 
-        // D1 operands.
-        for (int e = tid; e < kD * (kC / 8); e += kNT) {
-            const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // dv row j, tokens 8g..8g+7
-            uint16_t x[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint16_t*>(&sm.av.Vb[8 * g + m][j]);
-            uint4 w;
-            w.x = x[0] | ((uint32_t)x[1] << 16);
-            w.y = x[2] | ((uint32_t)x[3] << 16);
-            w.z = x[4] | ((uint32_t)x[5] << 16);
-            w.w = x[6] | ((uint32_t)x[7] << 16);
-            *reinterpret_cast<uint4*>(sm.op.d1.VT + core_off(j, 8 * g, kC)) = w;
-        }
-        for (int e = tid; e < kC * (kC / 8); e += kNT) {
-            const int t = e % kC, g = e / kC;  // row t of T diag(beta), columns 8g..8g+7
-            float x[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) x[m] = sm.T[t][8 * g + m] * sm.bt[8 * g + m];
-            uint4 p0, p1, p2;
-            split3x8(x, p0, p1, p2);
-            const uint32_t off = core_off(t, 8 * g, kC);
-            *reinterpret_cast<uint4*>(sm.op.d1.Bp[0] + off) = p0;
-            *reinterpret_cast<uint4*>(sm.op.d1.Bp[1] + off) = p1;
-            *reinterpret_cast<uint4*>(sm.op.d1.Bp[2] + off) = p2;
-        }
+        // D1 = U^T: V^T and (T diag(beta)) in parts.
+        gather_transposed(sm.av.R, sm.op.d1.VT, nullptr, tid);
+        split_scaled_T(sm.T, sm.bt, sm.op.d1.Bp, tid);
         async_proxy_fence();
         tc_fence_before();
         __syncthreads();
@@ -623,18 +639,27 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             const uint32_t vt = smem_u32(sm.op.d1.VT);
             for (int part = 0; part < 3; ++part)
                 for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem + 64, umma_desc(vt + 256 * ks, (kC / 8) * 128),
+                    umma_bf16(tmem + kTmemU, umma_desc(vt + 256 * ks, (kC / 8) * 128),
                               umma_desc(smem_u32(sm.op.d1.Bp[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
                               (part | ks) != 0 ? 1u : 0u);
             umma_commit(&sm.mma);
         }
-        // Tb = T diag(beta g), transposed, while the MMAs run.
-        for (int e = tid; e < kC * kC; e += kNT) {
-            const int i = e / kC, t = e % kC;
-            TbT[e] = i <= t ? sm.T[t][i] * (sm.bt[i] * expf(sm.lg[i])) : 0.f;
+        ++issued;
+        // K rows again (just read, so from L2) into the row buffer for the K^T image.
+#pragma unroll
+        for (int u = 0; u < kGr; ++u) {
+            const int e = tid + kNT * u;
+            const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+            uint4 kq = make_uint4(0, 0, 0, 0);
+            if (t < n)
+                kq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) +
+                                                          (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD + 8 * g));
+            uint32_t* kr = reinterpret_cast<uint32_t*>(&sm.av.R[t][8 * g]);
+            kr[0] = kq.x, kr[1] = kq.y, kr[2] = kq.z, kr[3] = kq.w;
         }
         ok = !__syncthreads_or(wait_parity(&sm.mma, 1) ? 0 : 1);
         if (ok) {
+            ++waits;
             tc_fence_after();
             // D1[j][t] = U[t][j]: lane j of this warp's quadrant, tokens 32*half .. +31.
             const int j = (warp % 4) * 32 + lane;
@@ -643,16 +668,60 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             for (int part = 0; part < 2; ++part) {
                 float v[16];
                 const int tb = 32 * half + 16 * part;
-                tmem_ld16(tmem + lane_base + 64u + (uint32_t)tb, v);
+                tmem_ld16(tmem + lane_base + kTmemU + (uint32_t)tb, v);
 #pragma unroll
                 for (int m = 0; m < 16; ++m) U[(tb + m) * kUS] = v[m];
+            }
+            // D2 = W^T: K^T (also the scan's operand, to the record) and (T diag(beta g)) in parts.
+            gather_transposed(sm.av.R, sm.op.d2.KT, rec + kRecA2, tid);
+            split_scaled_T(sm.T, sm.lg, sm.op.d2.Bt, tid);
+            async_proxy_fence();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                const uint32_t kt = smem_u32(sm.op.d2.KT);
+                for (int part = 0; part < 3; ++part)
+                    for (int ks = 0; ks < kC / 16; ++ks)
+                        umma_bf16(tmem, umma_desc(kt + 256 * ks, (kC / 8) * 128),
+                                  umma_desc(smem_u32(sm.op.d2.Bt[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
+                                  (part | ks) != 0 ? 1u : 0u);
+                umma_commit(&sm.mma);
+            }
+            ++issued;
+            ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
+            if (ok) {
+                ++waits;
+                tc_fence_after();
+                // D2[d][t] = W[t][d] -> W staged row-major (the operands of D2 are dead).
+                const int d = (warp % 4) * 32 + lane;
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    float v[16];
+                    const int tb = 32 * half + 16 * part;
+                    tmem_ld16(tmem + lane_base + (uint32_t)tb, v);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) sm.op.W[tb + m][d] = v[m];
+                }
+                __syncthreads();
+                // [W_hi; W_mid] and [W_lo; (Q, written above)] to the record.
+                for (int e = tid; e < kC * (kD / 8); e += kNT) {
+                    const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+                    const float4 w0 = *reinterpret_cast<const float4*>(&sm.op.W[t][8 * g]);
+                    const float4 w1 = *reinterpret_cast<const float4*>(&sm.op.W[t][8 * g + 4]);
+                    const float x[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    uint4 p0, p1, p2;
+                    split3x8(x, p0, p1, p2);
+                    *reinterpret_cast<uint4*>(rec + kRecA1 + core_off(t, 8 * g, kD)) = p0;
+                    *reinterpret_cast<uint4*>(rec + kRecA1 + core_off(kC + t, 8 * g, kD)) = p1;
+                    *reinterpret_cast<uint4*>(rec + kRecA1 + kA1Tile + core_off(t, 8 * g, kD)) = p2;
+                }
             }
         }
     }
     if (!ok && tid == 0) {
         record(a.err, GDN_ERR_TIMEOUT);
-        wait_parity(&sm.mma, 0);
-        wait_parity(&sm.mma, 1);
+        for (; waits < issued; ++waits) wait_parity(&sm.mma, (uint32_t)waits & 1u);
     }
     tc_fence_before();
     __syncthreads();
@@ -864,37 +933,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 2, tensor-core form (bf16 inputs).  Per chunk:
-//   D1 = [K; Q] [M_hi M_mid M_lo]  (M=128: rows 0..63 K, rows 64..127 Q; the fp32
-//                                   state block split into three bf16 parts stacked
-//                                   along N = 3 x 32; K = dk in 8 steps: 8 MMAs)
-//   D2 = K^T [E'_hi E'_mid E'_lo]  (M=128 rows of dk, N = 3 x 32, K = 64 tokens in
-//                                   4 steps, E' = diag(g_C / g) E: 4 MMAs)
-// The three column groups of each accumulator are added when TMEM is read, so the
-// A tile is read once per k-step for all three parts.  Operands sit in shared
-// memory in the no-swizzle K-major core layout; the accumulators take 2 x 96 of
-// 256 TMEM columns (D1 at column 0, D2 at column 128) allocated by warp 0.  Thread 0 issues the MMAs, commits them to an mbarrier,
-// and streams the chunk images with cp.async.bulk: the MMA operands [K; Q] and
-// K^T (one buffer each, refilled for the next chunk as soon as their MMAs
-// complete) and the small image (U slab, Tb^T, P^T, log g; two buffers, two
-// chunks ahead).  The triangular products Tb KM and P E run on the CUDA cores:
-// lane j owns value column j, warp w the rows 4w..4w+3 and 60-4w..63-4w, so a
-// step over i reads one KM (or E) value and two broadcast float4 of Tb^T (P^T).
-// Every wait is bounded (2 s); a timeout is recorded and the CTA drains and exits.
+// Kernel 2, tensor-core form (bf16 inputs).  Per chunk, with the fp32 state block M
+// (128 x 32) split into three bf16 parts stacked along N = 3 x 32:
+//   D1a = [W_hi; W_mid] [M_hi M_mid M_lo]   (8 MMAs, K = dk)
+//   D1b = [W_lo; Q]     [M_hi M_mid M_lo]   (8 MMAs)
+//   E   = U - (W_hi + W_mid + W_lo) M       (rows 0..63 of D1a and D1b, rows 64..127 of D1a)
+//   QM  = diag(g) Q M                       (rows 64..127 of D1b)
+//   D2  = K^T [E'_hi E'_mid E'_lo],  E' = diag(g_C / g) E   (4 MMAs, K = 64 tokens)
+//   M  <- g_C M + D2
+// O = QM + P E is formed on the CUDA cores while the D2 MMAs run.  The column
+// groups of each accumulator are added when TMEM is read.  Operands sit in shared
+// memory in the no-swizzle K-major core layout; the accumulators take 3 x 96 of 512
+// TMEM columns (D1a at 0, D1b at 128, D2 at 256), allocated by warp 0.  Thread 0
+// issues the MMAs, commits them to an mbarrier, and streams the chunk images with
+// cp.async.bulk: the A operands ([W; Q] tiles, K^T; one buffer each, refilled for
+// the next chunk as soon as their MMAs complete) and the small image (U slab, P^T,
+// log g; two buffers, two chunks ahead).  Every wait is bounded (2 s); a timeout is
+// recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;   // one bf16 part of M^T (32 x 128)
 constexpr uint32_t kBopPartE = (uint32_t)kDVC * kC * 2;  // one bf16 part of E'^T (32 x 64)
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemD2 = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemD1b = 128;
+constexpr uint32_t kTmemD2 = 256;
 
 struct SmemTC {
-    unsigned char a1[2 * kC * kD * 2];  // [K; Q] operand of D1
+    unsigned char a1[2 * kA1Tile];      // [W_hi; W_mid] | [W_lo; Q]
     unsigned char a2[kD * kC * 2];      // K^T operand of D2
     unsigned char img[2][kImgBytes];    // small images, double-buffered
     unsigned char bop[3 * kBopPart];    // B operand, three stacked parts: M^T, later E'^T
     float M[kD][kUS];                   // state block [dk][32 columns]
-    float KM[kC][kUS];
-    float QM[kC][kUS];                  // g Q M
+    float S[kC][kUS];                   // W_mid M, from the warps that read it to those that form E
+    float QM[kC][kUS];                  // diag(g) Q M
     uint64_t full[2];                   // small images
     uint64_t bar_a1, bar_a2, mma;
     uint32_t tmem;
@@ -922,11 +992,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         uint64_t* bar = &sm.full[c & 1];
         mbar_expect_tx(bar, kImgBytes);
         bulk_g2s(dst, rec + kRecU + cb * kUSlab, (uint32_t)kUSlab, bar);
-        bulk_g2s(dst + kImgTb, rec + kRecTb, (uint32_t)(kRecBytes - kRecTb), bar);
+        bulk_g2s(dst + kImgP, rec + kRecP, (uint32_t)(kRecBytes - kRecP), bar);
     };
     auto issue_a1 = [&](int c) {
-        mbar_expect_tx(&sm.bar_a1, (uint32_t)kRecA2);
-        bulk_g2s(sm.a1, record_of(a, bh, c) + kRecA1, (uint32_t)kRecA2, &sm.bar_a1);
+        mbar_expect_tx(&sm.bar_a1, (uint32_t)(2 * kA1Tile));
+        bulk_g2s(sm.a1, record_of(a, bh, c) + kRecA1, (uint32_t)(2 * kA1Tile), &sm.bar_a1);
     };
     auto issue_a2 = [&](int c) {
         mbar_expect_tx(&sm.bar_a2, (uint32_t)(kRecU - kRecA2));
@@ -968,10 +1038,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;           // TMEM columns half*16 .. +15
-    const int r1 = 4 * warp;             // triangular phases: rows r1..r1+3 and r2..r2+3, column `lane`
-    const int r2 = kC - 4 - 4 * warp;
+    const int half = warp / 4;             // TMEM columns half*16 .. +15 of each 32-column group
+    const int row = (warp % 4) * 32 + lane;  // TMEM lane
     const uint64_t da1 = umma_desc(smem_u32(sm.a1), (kD / 8) * 128);
+    const uint64_t da1b = umma_desc(smem_u32(sm.a1 + kA1Tile), (kD / 8) * 128);
     const uint64_t da2 = umma_desc(smem_u32(sm.a2), (kC / 8) * 128);
     bool ok = true;
     int c = 0;
@@ -979,10 +1049,18 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     int done_a1 = 0, done_a2 = 0, done_small = 0;  // counts what it issued, below
     int issued_a1 = 1, issued_a2 = 1, issued_small = min(nch, 2), issued_mma = 0;
 
+    // Sum of the three column groups (bf16 parts) of an accumulator, 16 columns at col.
+    auto read3 = [&](uint32_t col, float (&v)[16]) {
+        float v1[16], v2[16];
+        tmem_ld16(tmem + lane_base + col, v);
+        tmem_ld16(tmem + lane_base + col + kDVC, v1);
+        tmem_ld16(tmem + lane_base + col + 2 * kDVC, v2);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = (v2[j] + v1[j]) + v[j];
+    };
+
     for (; c < nch; ++c) {
         const int s = c & 1;
-        const int t0 = c * kC;
-        const int n = min(kC, a.L - t0);
         bool got = wait_parity(&sm.full[s], (uint32_t)(c >> 1) & 1u);
         got = wait_parity(&sm.bar_a1, (uint32_t)c & 1u) && got;
         if (__syncthreads_or(got ? 0 : 1)) {
@@ -992,9 +1070,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         ++done_small, ++done_a1;
         unsigned char* img = sm.img[s];
         float* U = reinterpret_cast<float*>(img);  // [64][kUS]: U, then E
-        const float* TbT = reinterpret_cast<const float*>(img + kImgTb);
-        const float* PT = reinterpret_cast<const float*>(img + kImgP);
         const float* lg = reinterpret_cast<const float*>(img + kImgG);
+        const int t0 = c * kC;
+        const int n = min(kC, a.L - t0);
+        const float* PT = reinterpret_cast<const float*>(img + kImgP);
 
         // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.
         for (int e = tid; e < kDVC * (kD / 8); e += kNT) {
@@ -1016,6 +1095,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         if (tid == 0) {
             const uint64_t db = umma_desc(smem_u32(sm.bop), (kD / 8) * 128);
             for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(tmem, da1 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
+            for (int ks = 0; ks < kD / 16; ++ks)
+                umma_bf16(tmem + kTmemD1b, da1b + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
             umma_commit(&sm.mma);
         }
         ++issued_mma;
@@ -1026,64 +1107,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         }
         ++waits_mma;
         tc_fence_after();
-        if (c + 1 < nch) {  // the [K; Q] buffer is free again
+        if (c + 1 < nch) {  // the [W; Q] buffer is free again
             if (tid == 0) issue_a1(c + 1);
             ++issued_a1;
         }
+        // Rows 64..127: W_mid M (handed over through S) and Q M (scaled by g, to the record).
+        // Rows 0..63: E = U - (W_hi M + W_lo M + W_mid M), in place over U and to the record.
         {
-            float v[16], v1[16], v2[16];
-            tmem_ld16(tmem + lane_base + (uint32_t)(half * 16), v);
-            tmem_ld16(tmem + lane_base + (uint32_t)(kDVC + half * 16), v1);
-            tmem_ld16(tmem + lane_base + (uint32_t)(2 * kDVC + half * 16), v2);
+            float va[16], vb[16];
+            read3((uint32_t)(half * 16), va);
+            read3(kTmemD1b + (uint32_t)(half * 16), vb);
+            if (row >= kC) {
+                const int t = row - kC;
+                const float g = expf(lg[t]);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += v1[j] + v2[j];
-            const int row = (warp % 4) * 32 + lane;
-            float* dstrow;
-            float g = 1.f;
+                for (int j = 0; j < 16; j += 4) {
+                    *reinterpret_cast<float4*>(&sm.S[t][half * 16 + j]) = make_float4(va[j], va[j + 1], va[j + 2], va[j + 3]);
+                    *reinterpret_cast<float4*>(&sm.QM[t][half * 16 + j]) =
+                        make_float4(vb[j] * g, vb[j + 1] * g, vb[j + 2] * g, vb[j + 3] * g);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
             if (row < kC) {
-                dstrow = &sm.KM[row][half * 16];
-            } else {
-                dstrow = &sm.QM[row - kC][half * 16];
-                g = expf(lg[row - kC]);
-            }
+                float* ur = U + row * kUS + half * 16;
 #pragma unroll
-            for (int j = 0; j < 16; j += 4)
-                *reinterpret_cast<float4*>(dstrow + j) = make_float4(v[j] * g, v[j + 1] * g, v[j + 2] * g, v[j + 3] * g);
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // E = U - Tb KM over U.  Tb^T[i][t] is zero for t < i, so rows r1.. need
-        // i <= r1 + 3 and rows r2.. need i <= r2 + 3.
-        {
-            float e1[4], e2[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                e1[r] = U[(r1 + r) * kUS + lane];
-                e2[r] = U[(r2 + r) * kUS + lane];
-            }
-#pragma unroll 4
-            for (int i = 0; i <= r1 + 3; ++i) {
-                const float km = sm.KM[i][lane];
-                const float4 ta = *reinterpret_cast<const float4*>(TbT + i * kC + r1);
-                const float4 tb = *reinterpret_cast<const float4*>(TbT + i * kC + r2);
-                e1[0] = fmaf(-ta.x, km, e1[0]), e1[1] = fmaf(-ta.y, km, e1[1]);
-                e1[2] = fmaf(-ta.z, km, e1[2]), e1[3] = fmaf(-ta.w, km, e1[3]);
-                e2[0] = fmaf(-tb.x, km, e2[0]), e2[1] = fmaf(-tb.y, km, e2[1]);
-                e2[2] = fmaf(-tb.z, km, e2[2]), e2[3] = fmaf(-tb.w, km, e2[3]);
-            }
-#pragma unroll 4
-            for (int i = r1 + 4; i <= r2 + 3; ++i) {
-                const float km = sm.KM[i][lane];
-                const float4 tb = *reinterpret_cast<const float4*>(TbT + i * kC + r2);
-                e2[0] = fmaf(-tb.x, km, e2[0]), e2[1] = fmaf(-tb.y, km, e2[1]);
-                e2[2] = fmaf(-tb.z, km, e2[2]), e2[3] = fmaf(-tb.w, km, e2[3]);
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                U[(r1 + r) * kUS + lane] = e1[r];
-                U[(r2 + r) * kUS + lane] = e2[r];
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(ur + j);
+                    const float4 m = *reinterpret_cast<const float4*>(&sm.S[row][half * 16 + j]);
+                    *reinterpret_cast<float4*>(ur + j) =
+                        make_float4(u.x - ((vb[j] + m.x) + va[j]), u.y - ((vb[j + 1] + m.y) + va[j + 1]),
+                                    u.z - ((vb[j + 2] + m.z) + va[j + 2]), u.w - ((vb[j + 3] + m.w) + va[j + 3]));
+                }
             }
         }
         __syncthreads();
@@ -1119,8 +1174,11 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         }
         ++issued_mma;
 
-        // O = QM + P E while the tensor core works (P^T[i][t] is zero for t < i).
+        // O = QM + P E on the CUDA cores while the tensor core works.  Lane j owns value
+        // column j; warp w the rows 4w..4w+3 and 60-4w..63-4w; P^T[i][t] is zero for
+        // t < i, so each row group stops at its own last row.
         {
+            const int r1 = 4 * warp, r2 = kC - 4 - 4 * warp;
             float o1[4], o2[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -1164,15 +1222,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             ++issued_a2;
         }
         {
-            float v[16], v1[16], v2[16];
-            tmem_ld16(tmem + lane_base + kTmemD2 + (uint32_t)(half * 16), v);
-            tmem_ld16(tmem + lane_base + kTmemD2 + (uint32_t)(kDVC + half * 16), v1);
-            tmem_ld16(tmem + lane_base + kTmemD2 + (uint32_t)(2 * kDVC + half * 16), v2);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += v1[j] + v2[j];
-            const int i = (warp % 4) * 32 + lane;  // dk row
+            float v[16];
+            read3(kTmemD2 + (uint32_t)(half * 16), v);
             const float gC = expf(lg[kC - 1]);
-            float* mrow = &sm.M[i][half * 16];
+            float* mrow = &sm.M[row][half * 16];  // dk row
 #pragma unroll
             for (int j = 0; j < 16; j += 4) {
                 float4 m = *reinterpret_cast<float4*>(mrow + j);
@@ -1256,7 +1309,7 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
         return GDN_ERR_INVALID_ARG;
     const int nchunks = (L + kC - 1) / kC;
     if (workspace_bytes < gdn_prefill_workspace_bytes(B, L, Hv, dk, dv)) return GDN_ERR_INVALID_ARG;
-    if ((int64_t)B * Hv * nchunks >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)B * Hv * nchunks * kNCB >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
     // 16-byte vector accesses: workspace, pool, out, q, k, v (rows of 128 elements keep the alignment).
     const uintptr_t align = reinterpret_cast<uintptr_t>(workspace) | reinterpret_cast<uintptr_t>(pool) |
                             reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(q) |
