@@ -35,9 +35,11 @@
 //       no-swizzle K-major core layout of the tensor-core operand, where
 //       W = Tb K is split into three bf16 parts (bf16 inputs only)
 //   A2  K^T as bf16, 128 (dk) rows x 64 tokens, same layout (bf16 inputs only)
+//   PA  [P_hi; P_mid] then [P_lo; P_lo], P split into three bf16 parts, two 128 x 64
+//       operand tiles (bf16 inputs only)
 //   U   four column slabs [4][64][36] fp32 (32 columns + 4 padding each)
 //   TbT [64][64] fp32: Tb transposed, TbT[i][t] = Tb[t][i], zero for t < i (fp32 inputs)
-//   PT  [64][64] fp32: P transposed, PT[i][t] = P[t][i], zero for t < i
+//   PT  [64][64] fp32: P transposed, PT[i][t] = P[t][i], zero for t < i (fp32 inputs)
 //   G   log g [64]
 
 #include "gdn_step.h"
@@ -60,18 +62,19 @@ constexpr int kPad = 4;         // row padding of [C][D] shared arrays in the fp
 constexpr size_t kRecA1 = 0;
 constexpr size_t kA1Tile = (size_t)2 * kC * kD * 2;  // one 128 x 128 bf16 operand tile
 constexpr size_t kRecA2 = kRecA1 + 2 * kA1Tile;
-constexpr size_t kRecU = kRecA2 + (size_t)kD * kC * 2;
+constexpr size_t kA2Tile = (size_t)kD * kC * 2;       // one 128 x 64 bf16 operand tile
+constexpr size_t kRecPA = kRecA2 + kA2Tile;
+constexpr size_t kRecU = kRecPA + 2 * kA2Tile;
 constexpr size_t kUSlab = (size_t)kC * kUS * 4;
 constexpr size_t kRecTb = kRecU + kNCB * kUSlab;
 constexpr size_t kRecP = kRecTb + (size_t)kC * kC * 4;
 constexpr size_t kRecG = kRecP + (size_t)kC * kC * 4;
 constexpr size_t kRecBytes = kRecG + (size_t)kC * 4;
-// One scan CTA's small image of a chunk in shared memory: its U slab | P^T | log g.
-constexpr uint32_t kImgP = (uint32_t)kUSlab;
-constexpr uint32_t kImgG = kImgP + (uint32_t)(kC * kC * 4);
+// One scan CTA's small image of a chunk in shared memory: its U slab | log g.
+constexpr uint32_t kImgG = (uint32_t)kUSlab;
 constexpr uint32_t kImgBytes = kImgG + (uint32_t)(kC * 4);
-static_assert(kRecG == kRecP + (size_t)kC * kC * 4, "P^T and log g are copied together");
-static_assert(kRecA2 % 16 == 0 && kRecU % 16 == 0 && kRecTb % 16 == 0 && kRecP % 16 == 0 && kRecBytes % 16 == 0,
+static_assert(kRecA2 % 16 == 0 && kRecPA % 16 == 0 && kRecU % 16 == 0 && kRecTb % 16 == 0 && kRecP % 16 == 0 &&
+                  kRecBytes % 16 == 0,
               "16-byte records");
 static_assert(kUSlab % 16 == 0 && kImgBytes % 16 == 0, "16-byte bulk copies");
 
@@ -531,7 +534,6 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     const int t0 = c * kC;
     const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
     unsigned char* rec = record_of(a, bh, c);
-    float* PT = reinterpret_cast<float*>(rec + kRecP);
     float* Gs = reinterpret_cast<float*>(rec + kRecG);
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const int half = warp / 4;  // TMEM columns 32*half .. +31 of each accumulator
@@ -605,12 +607,24 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                     sm.av.A[r][i] = i < r ? bt * expf(lt - sm.lg[i]) * v[j] : 0.f;
                 }
             } else {
+                // P row t, columns i0..i0+15, in three bf16 parts: [P_hi; P_mid] and [P_lo; P_lo].
                 const int t = r - kC;
                 const float lt = sm.lg[t];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int i = i0 + j;
-                    PT[i * kC + t] = i <= t ? expf(lt - sm.lg[i]) * v[j] : 0.f;
+                for (int g8 = 0; g8 < 16; g8 += 8) {
+                    float x[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int i = i0 + g8 + j;
+                        x[j] = i <= t ? expf(lt - sm.lg[i]) * v[g8 + j] : 0.f;
+                    }
+                    uint4 p0, p1, p2;
+                    split3x8(x, p0, p1, p2);
+                    unsigned char* pa = rec + kRecPA;
+                    *reinterpret_cast<uint4*>(pa + core_off(t, i0 + g8, kC)) = p0;
+                    *reinterpret_cast<uint4*>(pa + core_off(kC + t, i0 + g8, kC)) = p1;
+                    *reinterpret_cast<uint4*>(pa + kA2Tile + core_off(t, i0 + g8, kC)) = p2;
+                    *reinterpret_cast<uint4*>(pa + kA2Tile + core_off(kC + t, i0 + g8, kC)) = p2;
                 }
             }
         }
@@ -940,15 +954,17 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 //   E   = U - (W_hi + W_mid + W_lo) M       (rows 0..63 of D1a and D1b, rows 64..127 of D1a)
 //   QM  = diag(g) Q M                       (rows 64..127 of D1b)
 //   D2  = K^T [E'_hi E'_mid E'_lo],  E' = diag(g_C / g) E   (4 MMAs, K = 64 tokens)
-//   M  <- g_C M + D2
-// O = QM + P E is formed on the CUDA cores while the D2 MMAs run.  The column
-// groups of each accumulator are added when TMEM is read.  Operands sit in shared
-// memory in the no-swizzle K-major core layout; the accumulators take 3 x 96 of 512
-// TMEM columns (D1a at 0, D1b at 128, D2 at 256), allocated by warp 0.  Thread 0
-// issues the MMAs, commits them to an mbarrier, and streams the chunk images with
-// cp.async.bulk: the A operands ([W; Q] tiles, K^T; one buffer each, refilled for
-// the next chunk as soon as their MMAs complete) and the small image (U slab, P^T,
-// log g; two buffers, two chunks ahead).  Every wait is bounded (2 s); a timeout is
+//   DOa = [P_hi; P_mid] [E_hi E_mid E_lo],  DOb = [P_lo; P_lo] [E parts]  (4 + 4 MMAs)
+//   O   = QM + (P_hi + P_mid + P_lo) E,     M <- g_C M + D2
+// The sequential chain holds no CUDA-core contraction.  The column groups of each
+// accumulator are added when TMEM is read, and rows that two TMEM quadrants hold
+// are combined through shared memory.  Operands sit in shared memory in the
+// no-swizzle K-major core layout; the accumulators take 3 x 96 of 512 TMEM columns
+// (D1a, then DOa, at 0; D1b, then DOb, at 128; D2 at 256), allocated by warp 0.
+// Thread 0 issues the MMAs, commits them to an mbarrier, and streams the chunk
+// images with cp.async.bulk: the A operands ([W; Q] tiles; K^T with the P tiles;
+// one buffer each, refilled for the next chunk as soon as their MMAs complete) and
+// the small image (U slab, log g; two buffers, two chunks ahead).  Every wait is bounded (2 s); a timeout is
 // recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;   // one bf16 part of M^T (32 x 128)
@@ -959,11 +975,12 @@ constexpr uint32_t kTmemD2 = 256;
 
 struct SmemTC {
     unsigned char a1[2 * kA1Tile];      // [W_hi; W_mid] | [W_lo; Q]
-    unsigned char a2[kD * kC * 2];      // K^T operand of D2
+    unsigned char a2[3 * kA2Tile];      // K^T (D2), [P_hi; P_mid] (DOa), [P_lo; P_lo] (DOb)
     unsigned char img[2][kImgBytes];    // small images, double-buffered
     unsigned char bop[3 * kBopPart];    // B operand, three stacked parts: M^T, later E'^T
+    unsigned char bopE[3 * kBopPartE];  // B operand of DO: E^T in three stacked parts
     float M[kD][kUS];                   // state block [dk][32 columns]
-    float S[kC][kUS];                   // W_mid M, from the warps that read it to those that form E
+    float S[kC][kUS];                   // rows handed between TMEM quadrants: W_mid M, then QM + P_mid E
     float QM[kC][kUS];                  // diag(g) Q M
     uint64_t full[2];                   // small images
     uint64_t bar_a1, bar_a2, mma;
@@ -992,15 +1009,15 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         uint64_t* bar = &sm.full[c & 1];
         mbar_expect_tx(bar, kImgBytes);
         bulk_g2s(dst, rec + kRecU + cb * kUSlab, (uint32_t)kUSlab, bar);
-        bulk_g2s(dst + kImgP, rec + kRecP, (uint32_t)(kRecBytes - kRecP), bar);
+        bulk_g2s(dst + kImgG, rec + kRecG, (uint32_t)(kC * 4), bar);
     };
     auto issue_a1 = [&](int c) {
         mbar_expect_tx(&sm.bar_a1, (uint32_t)(2 * kA1Tile));
         bulk_g2s(sm.a1, record_of(a, bh, c) + kRecA1, (uint32_t)(2 * kA1Tile), &sm.bar_a1);
     };
     auto issue_a2 = [&](int c) {
-        mbar_expect_tx(&sm.bar_a2, (uint32_t)(kRecU - kRecA2));
-        bulk_g2s(sm.a2, record_of(a, bh, c) + kRecA2, (uint32_t)(kRecU - kRecA2), &sm.bar_a2);
+        mbar_expect_tx(&sm.bar_a2, (uint32_t)(3 * kA2Tile));
+        bulk_g2s(sm.a2, record_of(a, bh, c) + kRecA2, (uint32_t)(3 * kA2Tile), &sm.bar_a2);
     };
 
     if (tid == 0) {
@@ -1043,6 +1060,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     const uint64_t da1 = umma_desc(smem_u32(sm.a1), (kD / 8) * 128);
     const uint64_t da1b = umma_desc(smem_u32(sm.a1 + kA1Tile), (kD / 8) * 128);
     const uint64_t da2 = umma_desc(smem_u32(sm.a2), (kC / 8) * 128);
+    const uint64_t dpa = umma_desc(smem_u32(sm.a2 + kA2Tile), (kC / 8) * 128);
+    const uint64_t dpb = umma_desc(smem_u32(sm.a2 + 2 * kA2Tile), (kC / 8) * 128);
     bool ok = true;
     int c = 0;
     int waits_mma = 0;   // completed waits per barrier (all threads); thread 0 also
@@ -1073,7 +1092,6 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         const float* lg = reinterpret_cast<const float*>(img + kImgG);
         const int t0 = c * kC;
         const int n = min(kC, a.L - t0);
-        const float* PT = reinterpret_cast<const float*>(img + kImgP);
 
         // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.
         for (int e = tid; e < kDVC * (kD / 8); e += kNT) {
@@ -1143,19 +1161,27 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         }
         __syncthreads();
 
-        // B of D2: E' = diag(g_C / g) E, transposed (32 rows x 64 tokens), three bf16 parts.
+        // B of D2: E' = diag(g_C / g) E, and B of DO: E, both transposed (32 rows x 64
+        // tokens) in three bf16 parts.
         {
             const int jj = tid % kDVC, g = tid / kDVC;  // 32 x 8 granules, one per thread
             const float lgC = lg[kC - 1];
-            float x[8];
+            float x[8], y[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = U[(8 * g + j) * kUS + jj] * expf(lgC - lg[8 * g + j]);
+            for (int j = 0; j < 8; ++j) {
+                x[j] = U[(8 * g + j) * kUS + jj];
+                y[j] = x[j] * expf(lgC - lg[8 * g + j]);
+            }
             uint4 p0, p1, p2;
-            split3x8(x, p0, p1, p2);
             const uint32_t off = core_off(jj, 8 * g, kC);
+            split3x8(y, p0, p1, p2);
             *reinterpret_cast<uint4*>(sm.bop + off) = p0;
             *reinterpret_cast<uint4*>(sm.bop + kBopPartE + off) = p1;
             *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPartE + off) = p2;
+            split3x8(x, p0, p1, p2);
+            *reinterpret_cast<uint4*>(sm.bopE + off) = p0;
+            *reinterpret_cast<uint4*>(sm.bopE + kBopPartE + off) = p1;
+            *reinterpret_cast<uint4*>(sm.bopE + 2 * kBopPartE + off) = p2;
         }
         got = wait_parity(&sm.bar_a2, (uint32_t)c & 1u);
         async_proxy_fence();
@@ -1168,48 +1194,16 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         tc_fence_after();
         if (tid == 0) {
             const uint64_t db = umma_desc(smem_u32(sm.bop), (kC / 8) * 128);
+            const uint64_t de = umma_desc(smem_u32(sm.bopE), (kC / 8) * 128);
             for (int ks = 0; ks < kC / 16; ++ks)
                 umma_bf16(tmem + kTmemD2, da2 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
+            for (int ks = 0; ks < kC / 16; ++ks)
+                umma_bf16(tmem, dpa + 16 * ks, de + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
+            for (int ks = 0; ks < kC / 16; ++ks)
+                umma_bf16(tmem + kTmemD1b, dpb + 16 * ks, de + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
             umma_commit(&sm.mma);
         }
         ++issued_mma;
-
-        // O = QM + P E on the CUDA cores while the tensor core works.  Lane j owns value
-        // column j; warp w the rows 4w..4w+3 and 60-4w..63-4w; P^T[i][t] is zero for
-        // t < i, so each row group stops at its own last row.
-        {
-            const int r1 = 4 * warp, r2 = kC - 4 - 4 * warp;
-            float o1[4], o2[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                o1[r] = sm.QM[r1 + r][lane];
-                o2[r] = sm.QM[r2 + r][lane];
-            }
-#pragma unroll 4
-            for (int i = 0; i <= r1 + 3; ++i) {
-                const float ev = U[i * kUS + lane];
-                const float4 pa = *reinterpret_cast<const float4*>(PT + i * kC + r1);
-                const float4 pb = *reinterpret_cast<const float4*>(PT + i * kC + r2);
-                o1[0] = fmaf(pa.x, ev, o1[0]), o1[1] = fmaf(pa.y, ev, o1[1]);
-                o1[2] = fmaf(pa.z, ev, o1[2]), o1[3] = fmaf(pa.w, ev, o1[3]);
-                o2[0] = fmaf(pb.x, ev, o2[0]), o2[1] = fmaf(pb.y, ev, o2[1]);
-                o2[2] = fmaf(pb.z, ev, o2[2]), o2[3] = fmaf(pb.w, ev, o2[3]);
-            }
-#pragma unroll 4
-            for (int i = r1 + 4; i <= r2 + 3; ++i) {
-                const float ev = U[i * kUS + lane];
-                const float4 pb = *reinterpret_cast<const float4*>(PT + i * kC + r2);
-                o2[0] = fmaf(pb.x, ev, o2[0]), o2[1] = fmaf(pb.y, ev, o2[1]);
-                o2[2] = fmaf(pb.z, ev, o2[2]), o2[3] = fmaf(pb.w, ev, o2[3]);
-            }
-            float* ob = a.out + (((size_t)b * a.L + t0) * a.Hv + h) * kD + col0 + lane;
-            const size_t row_stride = (size_t)a.Hv * kD;
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                if (r1 + r < n) ob[(r1 + r) * row_stride] = o1[r];
-                if (r2 + r < n) ob[(r2 + r) * row_stride] = o2[r];
-            }
-        }
 
         if (__syncthreads_or(wait_parity(&sm.mma, (uint32_t)waits_mma & 1u) ? 0 : 1)) {
             ok = false;
@@ -1217,9 +1211,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         }
         ++waits_mma;
         tc_fence_after();
-        if (c + 1 < nch) {  // the K^T buffer is free again
+        if (c + 1 < nch) {  // the K^T and P buffer is free again
             if (tid == 0) issue_a2(c + 1);
             ++issued_a2;
+        }
+        // O: rows 64..127 of DOa (P_mid E) plus QM go through S to the warps holding rows
+        // 0..63 of DOa (P_hi E) and DOb (P_lo E), which write the chunk's outputs.
+        {
+            float vo[16];
+            read3((uint32_t)(half * 16), vo);
+            if (row >= kC) {
+                const int t = row - kC;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 q = *reinterpret_cast<const float4*>(&sm.QM[t][half * 16 + j]);
+                    *reinterpret_cast<float4*>(&sm.S[t][half * 16 + j]) =
+                        make_float4(q.x + vo[j], q.y + vo[j + 1], q.z + vo[j + 2], q.w + vo[j + 3]);
+                }
+            }
+            float vl[16];
+            read3(kTmemD1b + (uint32_t)(half * 16), vl);
+            tc_fence_before();
+            __syncthreads();
+            if (row < n) {
+                float* ob = a.out + (((size_t)b * a.L + t0 + row) * a.Hv + h) * kD + col0 + half * 16;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 sq = *reinterpret_cast<const float4*>(&sm.S[row][half * 16 + j]);
+                    *reinterpret_cast<float4*>(ob + j) =
+                        make_float4(sq.x + (vl[j] + vo[j]), sq.y + (vl[j + 1] + vo[j + 1]),
+                                    sq.z + (vl[j + 2] + vo[j + 2]), sq.w + (vl[j + 3] + vo[j + 3]));
+                }
+            }
         }
         {
             float v[16];
