@@ -216,6 +216,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t addr, float (&v)[16]) {
     for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Loads of 16 TMEM columns whose completion is awaited once for several of them:
+// issue them, then tmem_wait_ld(), then tie_regs() on each destination so that no
+// use of the registers is scheduled before the wait.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t addr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(addr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tie_regs(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]));
+}
+
 // Eight fp32 values as three 16-byte granules of bf16 parts: x = hi + mid + lo.
 __device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& mid, uint4& lo) {
     uint32_t h[4], m[4], l[4];
@@ -1068,14 +1086,18 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     int done_a1 = 0, done_a2 = 0, done_small = 0;  // counts what it issued, below
     int issued_a1 = 1, issued_a2 = 1, issued_small = min(nch, 2), issued_mma = 0;
 
-    // Sum of the three column groups (bf16 parts) of an accumulator, 16 columns at col.
+    // Sum of the three column groups (bf16 parts) of an accumulator, 16 columns at col:
+    // the three loads are in flight together.
     auto read3 = [&](uint32_t col, float (&v)[16]) {
-        float v1[16], v2[16];
-        tmem_ld16(tmem + lane_base + col, v);
-        tmem_ld16(tmem + lane_base + col + kDVC, v1);
-        tmem_ld16(tmem + lane_base + col + 2 * kDVC, v2);
+        uint32_t r0[16], r1[16], r2[16];
+        tmem_ld16_issue(tmem + lane_base + col, r0);
+        tmem_ld16_issue(tmem + lane_base + col + kDVC, r1);
+        tmem_ld16_issue(tmem + lane_base + col + 2 * kDVC, r2);
+        tmem_wait_ld();
+        tie_regs(r0), tie_regs(r1), tie_regs(r2);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = (v2[j] + v1[j]) + v[j];
+        for (int j = 0; j < 16; ++j)
+            v[j] = (__uint_as_float(r2[j]) + __uint_as_float(r1[j])) + __uint_as_float(r0[j]);
     };
 
     for (; c < nch; ++c) {
