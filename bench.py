@@ -595,7 +595,7 @@ def run_prefill(args):
         ws_bytes = gdn.gdn_prefill_workspace_bytes(B, L, Hv, dk, dv)
         chunks = (L + 63) // 64
         C = 64
-        # per (request, head, chunk): K K^T, Q K^T, U = T diag(beta) V, [K;Q] M, Tb (K M),
+        # per (request, head, chunk): K K^T, Q K^T, U = T diag(beta) V, W = Tb K, [W;Q] M,
         # P E, K^T E, and the triangular inverse
         flop_chunk = 2 * C * C * dk * 2 + 2 * C * C * dv + 2 * 2 * C * dk * dv + 2 * C * C * dv * 2 \
             + 2 * C * dk * dv + C ** 3 / 3
