@@ -17,17 +17,19 @@
 //     E   = U - Tb (K M0)                              (C x dv)
 //     O   = diag(g) (Q M0) + P E,  P[t][i] = (g_t/g_i)(q_t . k_i), i <= t
 //     M_C = g_C M0 + K^T diag(g_C / g) E                (dk x dv)
-// Kernel 1 builds, for every (request, head, chunk) in parallel, U, Tb, P and
-// the log-gates (log g_t) into the caller's workspace; kernel 2 walks the chunks
-// of each (request, head, column block) in order, carrying M in shared memory.
-// The large products of kernel 2 ([K; Q] M0 and K^T E) have one operand that is
-// exact in bf16 (the bf16 inputs k, q) and one fp32 operand; with bf16 inputs
-// they run on the tensor cores (tcgen05, accumulators in TMEM) with the fp32
-// operand split into three bf16 parts (hi + mid + lo carries 24 bits), which
-// keeps fp32 accuracy.  The triangular products stay on the CUDA cores.
-// Ratios g_t / g_i are formed as exp(log g_t - log g_i) <= 1, so nothing
-// overflows; g_t itself may underflow to zero, which is its true value to fp32
-// precision.
+// Kernel 1 builds, for every (request, head, chunk) in parallel, everything that
+// does not depend on the state into the caller's workspace; kernel 2 walks the
+// chunks of each (request, head, column block) in order, carrying M in shared
+// memory.  With bf16 inputs both kernels run their products on the tensor cores
+// (tcgen05, accumulators in TMEM).  An operand that is not a bf16 input is fp32
+// and enters as three bf16 parts (hi + mid + lo carries 24 bits), with every part
+// product formed, which keeps fp32 accuracy.  In that form kernel 1 also computes
+// W = Tb K, so that kernel 2 evaluates the same algebra re-associated:
+//     E = U - W M0,   O = diag(g) (Q M0) + P E,   M_C = g_C M0 + K^T diag(g_C / g) E,
+// all as MMAs.  With fp32 inputs (not exact in bf16) both kernels run on the CUDA
+// cores in the first form.  Ratios g_t / g_i are formed as exp(log g_t - log g_i)
+// <= 1, so nothing overflows; g_t itself may underflow to zero, which is its true
+// value to fp32 precision.
 //
 // Workspace record of one (request, head, chunk), bytes.  The first parts are laid
 // out as the shared-memory images the scan copies in (bulk copies, 16-byte granules):
