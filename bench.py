@@ -374,7 +374,21 @@ def cpu_baseline(budget_s: float = 12.0, Hv: int = 32):
     t = oracle_time(n_req, threads)
     return {"value": n_req * Hv / t, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"one in-place call on {n_req} of the 256 requests of layer 0 ({n_req * Hv} "
-                      f"tokens*heads), C++ double-precision oracle, {threads} threads, {t:.1f} s"}
+                      f"tokens*heads), C++ double-precision oracle, {threads} threads, {t:.1f} s",
+            "single_thread_value": Hv / max(t1, 1e-9), "host": host_info()}
+
+
+def host_info() -> dict:
+    """The CPU the oracle ran on: model, cores this process may use, logical CPUs."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu_model": model, "affinity_cores": cpu_cores(), "logical_cpus": os.cpu_count()}
 
 
 def headline_config(args, world: int) -> dict:
@@ -409,7 +423,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": headline_config(args, 1),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "host": host_info(),
                          "sample": f"each step: one in-place call on {n_req} of the {args.batch} requests of "
                                    f"layer 0 ({n_req * 32} tokens*heads), C++ double-precision oracle"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
