@@ -621,6 +621,8 @@ CHUNKED_SHAPES = [
     (2, 65, 1, 2, wl.BF16, False),
     (2, 200, 2, 2, wl.F32, False),
     (1, 1000, 1, 2, wl.BF16, True),
+    (4, 130, 2, 2, wl.BF16, False),   # one value head per key head, ragged last chunk
+    (2, 96, 1, 4, wl.BF16, True),     # four value heads per key head, in place
 ]
 
 
