@@ -968,7 +968,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 
 // ---------------------------------------------------------------------------
 // Kernel 2, tensor-core form (bf16 inputs).  Per chunk, with the fp32 state block M
-// (128 x 32) split into three bf16 parts stacked along N = 3 x 32:
+// (128 x 32, held in registers: each thread owns the 16 elements it reads from D2)
+// split into three bf16 parts stacked along N = 3 x 32:
 //   D1a = [W_hi; W_mid] [M_hi M_mid M_lo]   (8 MMAs, K = dk)
 //   D1b = [W_lo; Q]     [M_hi M_mid M_lo]   (8 MMAs)
 //   E   = U - (W_hi + W_mid + W_lo) M       (rows 0..63 of D1a and D1b, rows 64..127 of D1a)
@@ -999,7 +1000,6 @@ struct SmemTC {
     unsigned char img[2][kImgBytes];    // small images, double-buffered
     unsigned char bop[3 * kBopPart];    // B operand, three stacked parts: M^T, later E'^T
     unsigned char bopE[3 * kBopPartE];  // B operand of DO: E^T in three stacked parts
-    float M[kD][kUS];                   // state block [dk][32 columns]
     float S[kC][kUS];                   // rows handed between TMEM quadrants: W_mid M, then QM + P_mid E
     float QM[kC][kUS];                  // diag(g) Q M
     uint64_t full[2];                   // small images
@@ -1007,6 +1007,27 @@ struct SmemTC {
     uint32_t tmem;
     int src, dst, status;
 };
+
+// 8 x 8 transpose of 32-bit values across each group of 8 lanes: on entry lane l
+// (l = lane % 8) holds row l of the block in x[0..7]; on return it holds column l
+// (x[r] = row r's element l).  Three butterfly stages exchange 4 x 4, 2 x 2 and
+// 1 x 1 sub-blocks with the partner lane l ^ s.
+__device__ __forceinline__ void transpose8(float (&x)[8], int lane) {
+#pragma unroll
+    for (int s = 4; s >= 1; s >>= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            if (c & s) continue;
+            const float send = upper ? x[c] : x[c + s];
+            const float got = __shfl_xor_sync(0xffffffffu, send, s);
+            if (upper)
+                x[c] = got;
+            else
+                x[c + s] = got;
+        }
+    }
+}
 
 __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_tc[];
@@ -1063,20 +1084,25 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const int half = warp / 4;             // TMEM columns half*16 .. +15 of each 32-column group
+    const int row = (warp % 4) * 32 + lane;  // TMEM lane
+    // The state block lives in registers: this thread owns M[row][half*16 .. +15], the
+    // elements it reads from D2 in every state update.
+    float m[16];
     {
-        const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) + col0;
-        for (int e = tid; e < kD * (kDVC / 4); e += kNT) {
-            const int i = e / (kDVC / 4), j4 = e % (kDVC / 4);
-            *reinterpret_cast<float4*>(&sm.M[i][4 * j4]) = *reinterpret_cast<const float4*>(M0 + (size_t)i * kD + 4 * j4);
+        const float4* M0 = reinterpret_cast<const float4*>(a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) +
+                                                           (size_t)row * kD + col0 + half * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = M0[j];
+            m[4 * j] = v.x, m[4 * j + 1] = v.y, m[4 * j + 2] = v.z, m[4 * j + 3] = v.w;
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;             // TMEM columns half*16 .. +15 of each 32-column group
-    const int row = (warp % 4) * 32 + lane;  // TMEM lane
     const uint64_t da1 = umma_desc(smem_u32(sm.a1), (kD / 8) * 128);
     const uint64_t da1b = umma_desc(smem_u32(sm.a1 + kA1Tile), (kD / 8) * 128);
     const uint64_t da2 = umma_desc(smem_u32(sm.a2), (kC / 8) * 128);
@@ -1117,15 +1143,18 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         const int t0 = c * kC;
         const int n = min(kC, a.L - t0);
 
-        // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.
-        for (int e = tid; e < kDVC * (kD / 8); e += kNT) {
-            const int jj = e % kDVC, g = e / kDVC;
+        // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.  Each
+        // group of 8 lanes transposes its 8 rows x 16 columns, so that lane l holds columns
+        // l and 8 + l of those rows: two granules.
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
             float x[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = sm.M[8 * g + j][jj];
+            for (int j = 0; j < 8; ++j) x[j] = m[8 * blk + j];
+            transpose8(x, lane);
             uint4 p0, p1, p2;
             split3x8(x, p0, p1, p2);
-            const uint32_t off = core_off(jj, 8 * g, kD);
+            const uint32_t off = core_off(half * 16 + 8 * blk + (lane & 7), row & ~7, kD);
             *reinterpret_cast<uint4*>(sm.bop + off) = p0;
             *reinterpret_cast<uint4*>(sm.bop + kBopPart + off) = p1;
             *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPart + off) = p2;
@@ -1272,14 +1301,8 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             float v[16];
             read3(kTmemD2 + (uint32_t)(half * 16), v);
             const float gC = expf(lg[kC - 1]);
-            float* mrow = &sm.M[row][half * 16];  // dk row
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                float4 m = *reinterpret_cast<float4*>(mrow + j);
-                m.x = fmaf(gC, m.x, v[j]), m.y = fmaf(gC, m.y, v[j + 1]);
-                m.z = fmaf(gC, m.z, v[j + 2]), m.w = fmaf(gC, m.w, v[j + 3]);
-                *reinterpret_cast<float4*>(mrow + j) = m;
-            }
+            for (int j = 0; j < 16; ++j) m[j] = fmaf(gC, m[j], v[j]);
         }
         // Small buffer s (E was written into it) is refilled next by the async proxy.
         async_proxy_fence();
@@ -1293,11 +1316,10 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     }
 
     if (ok) {
-        float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + col0;
-        for (int e = tid; e < kD * (kDVC / 4); e += kNT) {
-            const int i = e / (kDVC / 4), j4 = e % (kDVC / 4);
-            *reinterpret_cast<float4*>(MD + (size_t)i * kD + 4 * j4) = *reinterpret_cast<const float4*>(&sm.M[i][4 * j4]);
-        }
+        float4* MD = reinterpret_cast<float4*>(a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)row * kD +
+                                               col0 + half * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) MD[j] = make_float4(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
     } else if (tid == 0) {
         // Something never arrived: record it, then give every copy and MMA still
         // outstanding one more bounded wait before shared memory and TMEM go.
