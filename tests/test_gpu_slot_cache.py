@@ -137,3 +137,62 @@ def test_slot_cache_session_on_gpu():
             oracle.decode_step(replay, np.array([i % 2], np.int32), np.array([[(i + 1) % 2]], np.int32), q, k, v, a,
                                b, o)
         assert rel_err(pool_d[slot].cpu().numpy(), replay[len(seq) % 2]) <= TOL_STATE
+
+
+@pytest.mark.parametrize("chunked", [False, True], ids=["token_steps", "chunked"])
+def test_prefill_checkpoint_then_fork_and_decode(chunked):
+    """The intended flow end to end: a prefill writes a prompt's state into the request's
+    slot, the cache keeps it as a checkpoint, a second request extending the prompt shares
+    it and forks on its first decode step.  States match an oracle replay of each token
+    history; the checkpoint's bytes never change."""
+    import torch
+
+    from hybrid_linear_attention_step_b200 import gdn
+    from hybrid_linear_attention_step_b200.slot_cache import SlotCache
+
+    num_slots = 8
+    cache = SlotCache(num_slots)
+    pool_d = torch.zeros((num_slots, Hv, DK, DV), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rng = np.random.default_rng(11)
+    ctx = [int(x) for x in rng.integers(0, 50, 130)]  # two chunks and a ragged tail
+
+    r0, slot, matched, needs_init = cache.open(ctx)
+    assert matched == 0 and needs_init
+    x = [to_torch(t) for t in batch_inputs([[]], [ctx])]
+    idx = torch.tensor([slot], dtype=torch.int32, device="cuda")
+    out = torch.zeros((1, len(ctx), Hv, DV), device="cuda")
+    if chunked:
+        ws = torch.empty(gdn.gdn_prefill_workspace_bytes(1, len(ctx), Hv, DK, DV), dtype=torch.uint8,
+                         device="cuda")
+        gdn.gdn_prefill_chunked(pool_d, idx, idx, *x, out, ws, err_word=err)
+    else:
+        gdn.gdn_prefill(pool_d, idx, idx, *x, out, err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    assert cache.checkpoint(r0, ctx) == slot
+    ckpt = pool_d[slot].cpu().numpy().copy()
+
+    def replay(seq, st=None, start=0):
+        """Oracle state after the tokens seq[start:], from st (zero if None), one token at a time."""
+        st = np.zeros((1, Hv, DK, DV), np.float32) if st is None else st.copy()
+        for i in range(start, len(seq)):
+            q, k, v, a, b = token_inputs(seq[: i + 1])
+            o = np.zeros((1, 1, Hv, DV), np.float32)
+            zero = np.zeros(1, np.int32)
+            oracle.decode_step(st, zero, zero.reshape(1, 1), q, k, v, a, b, o, nthreads=8)
+        return st
+
+    ref_ctx = replay(ctx)
+    assert rel_err(ckpt, ref_ctx[0]) <= TOL_STATE
+    ext = ctx + [7]
+    r1, s1, matched1, needs1 = cache.open(ext)
+    assert (s1, matched1, needs1) == (slot, len(ctx), False)
+    src, dst = cache.plan([r1])
+    assert src[0] == slot and dst[0, 0] != slot  # copy-on-write fork
+    x1 = [to_torch(t) for t in batch_inputs([ctx], [[7]])]
+    out1 = torch.zeros((1, 1, Hv, DV), device="cuda")
+    gdn.gdn_decode_step(pool_d, to_torch(src), to_torch(dst), *x1, out1, err_word=err)
+    cache.commit([r1])
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    assert np.array_equal(pool_d[slot].cpu().numpy().view(np.uint32), ckpt.view(np.uint32))
+    assert rel_err(pool_d[int(dst[0, 0])].cpu().numpy(), replay(ext, ref_ctx, len(ctx))[0]) <= TOL_STATE
