@@ -372,9 +372,14 @@ def cpu_baseline(budget_s: float = 12.0, Hv: int = 32):
     n_req = int(max(1, min(256, budget_s * cores / max(t1, 1e-6) * 0.8)))
     threads = min(cores, n_req)
     t = oracle_time(n_req, threads)
-    return {"value": n_req * Hv / t, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"one in-place call on {n_req} of the 256 requests of layer 0 ({n_req * Hv} "
-                      f"tokens*heads), C++ double-precision oracle, {threads} threads, {t:.1f} s",
+    calls, total = 1, t
+    while total < budget_s and calls < 8:  # successive steps of the same requests, up to the budget
+        total += oracle_time(n_req, threads)
+        calls += 1
+    return {"value": calls * n_req * Hv / total, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{calls} successive in-place calls on {n_req} of the 256 requests of layer 0 "
+                      f"({calls * n_req * Hv} tokens*heads), C++ double-precision oracle, {threads} threads, "
+                      f"{total:.1f} s",
             "single_thread_value": Hv / max(t1, 1e-9), "host": host_info()}
 
 
