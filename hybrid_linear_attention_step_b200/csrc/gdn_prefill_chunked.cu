@@ -1128,6 +1128,27 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
             v[j] = (__uint_as_float(r2[j]) + __uint_as_float(r1[j])) + __uint_as_float(r0[j]);
     };
 
+    // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.  Each
+    // group of 8 lanes transposes its 8 rows x 16 columns, so that lane l holds columns
+    // l and 8 + l of those rows: two granules.  The caller fences and synchronises.
+    auto split_m = [&]() {
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = m[8 * blk + j];
+            transpose8(x, lane);
+            uint4 p0, p1, p2;
+            split3x8(x, p0, p1, p2);
+            const uint32_t off = core_off(half * 16 + 8 * blk + (lane & 7), row & ~7, kD);
+            *reinterpret_cast<uint4*>(sm.bop + off) = p0;
+            *reinterpret_cast<uint4*>(sm.bop + kBopPart + off) = p1;
+            *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPart + off) = p2;
+        }
+        async_proxy_fence();
+    };
+    split_m();  // the first chunk's; the barrier after the first wait orders it before the MMAs
+
     for (; c < nch; ++c) {
         const int s = c & 1;
         bool got = wait_parity(&sm.full[s], (uint32_t)(c >> 1) & 1u);
@@ -1143,26 +1164,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         const int t0 = c * kC;
         const int n = min(kC, a.L - t0);
 
-        // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.  Each
-        // group of 8 lanes transposes its 8 rows x 16 columns, so that lane l holds columns
-        // l and 8 + l of those rows: two granules.
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            float x[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = m[8 * blk + j];
-            transpose8(x, lane);
-            uint4 p0, p1, p2;
-            split3x8(x, p0, p1, p2);
-            const uint32_t off = core_off(half * 16 + 8 * blk + (lane & 7), row & ~7, kD);
-            *reinterpret_cast<uint4*>(sm.bop + off) = p0;
-            *reinterpret_cast<uint4*>(sm.bop + kBopPart + off) = p1;
-            *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPart + off) = p2;
-        }
-        async_proxy_fence();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        // (B of D1, the parts of M, was built after the previous state update.)
         if (tid == 0) {
             const uint64_t db = umma_desc(smem_u32(sm.bop), (kD / 8) * 128);
             for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(tmem, da1 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
@@ -1304,6 +1306,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
 #pragma unroll
             for (int j = 0; j < 16; ++j) m[j] = fmaf(gC, m[j], v[j]);
         }
+        if (c + 1 < nch) split_m();  // the next chunk's B of D1 (the D2 MMAs, last readers of bop, are done)
         // Small buffer s (E was written into it) is refilled next by the async proxy.
         async_proxy_fence();
         tc_fence_before();
