@@ -113,3 +113,43 @@ def test_wait_selftest_validates_on_the_host(lib):
     assert f(1000, None, None) == 1          # no error word
     assert f(0, 8, None) == 1                # empty limit
     assert f(2_000_000_001, 8, None) == 1    # above the pipelines' own limit
+
+
+def _prefill_chunked(lib, **kw):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    f = lib.gdn_prefill_chunked
+    f.restype = i32
+    f.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, ctypes.c_size_t,
+                  vp, vp]
+    a = dict(pool=16, num_slots=4, src=16, dst=16, q=16, k=16, v=16, alpha=16, beta=16, out=16,
+             B=1, L=100, Hk=1, Hv=2, dk=128, dv=128, dtype=1, ws=16, ws_bytes=1 << 30, err=None, stream=None)
+    a.update(kw)
+    return f(*a.values())
+
+
+def test_prefill_workspace_size(lib):
+    w = lib.gdn_prefill_workspace_bytes
+    w.restype = ctypes.c_size_t
+    w.argtypes = [ctypes.c_int32] * 5
+    one = w(1, 1, 1, 128, 128)
+    assert one > 0 and one % 16 == 0
+    assert w(1, 64, 1, 128, 128) == one          # one chunk holds 64 tokens
+    assert w(1, 65, 1, 128, 128) == 2 * one      # a ragged tail takes a chunk of its own
+    assert w(3, 130, 5, 128, 128) == 3 * 5 * 3 * one
+    assert w(1, 64, 1, 64, 64) == 0              # shapes the chunked path does not support
+    assert w(1, 0, 1, 128, 128) == 0
+
+
+def test_prefill_chunked_validates_on_the_host(lib):
+    lib.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_prefill_workspace_bytes.argtypes = [ctypes.c_int32] * 5
+    need = lib.gdn_prefill_workspace_bytes(1, 100, 2, 128, 128)
+    assert _prefill_chunked(lib, dk=64, dv=64) == 1                  # unsupported head size
+    assert _prefill_chunked(lib, Hk=3, Hv=4) == 1                    # Hv not a multiple of Hk
+    assert _prefill_chunked(lib, L=0) == 1
+    assert _prefill_chunked(lib, dtype=5) == 1
+    assert _prefill_chunked(lib, ws=None) == 1                       # no workspace
+    assert _prefill_chunked(lib, ws_bytes=need - 16) == 1            # short workspace
+    assert _prefill_chunked(lib, ws=24, ws_bytes=need) == 1          # workspace not 16-byte aligned
+    assert _prefill_chunked(lib, out=20, ws_bytes=need) == 1         # out not 16-byte aligned
+    assert _prefill_chunked(lib, B=0, pool=None, ws=None) == 0       # empty batch: no-op
