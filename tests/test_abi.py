@@ -153,3 +153,18 @@ def test_prefill_chunked_validates_on_the_host(lib):
     assert _prefill_chunked(lib, ws=24, ws_bytes=need) == 1          # workspace not 16-byte aligned
     assert _prefill_chunked(lib, out=20, ws_bytes=need) == 1         # out not 16-byte aligned
     assert _prefill_chunked(lib, B=0, pool=None, ws=None) == 0       # empty batch: no-op
+
+
+def test_prefill_validates_on_the_host(lib):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    f = lib.gdn_prefill
+    f.restype = i32
+    f.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    a = dict(pool=16, num_slots=4, src=16, dst=16, q=16, k=16, v=16, alpha=16, beta=16, out=16,
+             B=1, L=10, Hk=1, Hv=2, dk=128, dv=128, dtype=1, err=None, stream=None)
+    call = lambda **kw: f(*{**a, **kw}.values())
+    assert call(L=0) == 1
+    assert call(Hk=2, Hv=3) == 1
+    assert call(dtype=9) == 1
+    assert call(src=None) == 1
+    assert call(B=0, pool=None) == 0  # empty batch: no-op
