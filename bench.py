@@ -43,11 +43,10 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
-# source it was taken on (sha256 of gdn_step.cu).  See profiles/.
+# source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
                "source_sha256": "2749ceb8bdba484ccb2c638bc20fa1bd165c2b17abd6d9fd3899c0caa34bbfaa",
-               "bytes_per_launch": 541164544 + 483485952,
-               "profile": "profiles/gdn_tile1_kernel_large_decode.md"}
+               "bytes_per_launch": 541164544 + 483485952}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
@@ -65,6 +64,9 @@ def algorithmic_bytes_per_unit(dk: int, dv: int, G: int, in_bytes: int = 2, T: i
     return state + qk + dv * in_bytes + 8.0 + 4.0 * dv
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -76,6 +78,17 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s) for a kernel timed in isolation."""
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            return float(json.loads(p.read_text())["bf16_tflops"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 def source_sha256() -> str:
     return hashlib.sha256(KERNEL_SOURCE.read_bytes()).hexdigest()
 
@@ -83,90 +96,119 @@ def source_sha256() -> str:
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works.
+    """SM clocks and clock-event (throttle) reasons sampled while the GPU works.
 
-    A reader thread collects one CSV line per sample; ``start`` returns once the
-    first sample has arrived (or after a few seconds if nvidia-smi is absent).
+    Reads only.  NVML is polled from a thread every ``interval_ms`` (2 ms by default, so
+    even a timed region of a few tens of milliseconds holds several samples); where
+    NVML is not importable, ``nvidia-smi -lms`` is read instead.  ``mark`` sets the
+    timed window; ``stop`` summarises the samples inside it.
     """
 
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
-              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("sw_power_cap", 0x4))
+    SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+                  "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: str, interval_ms: int = 50):
-        self.proc = None
-        self.gpu_index = gpu_index
+    def __init__(self, device_index: int = 0, interval_ms: float = 2.0):
+        self.device_index = device_index
         self.interval_ms = interval_ms
         self.window = None
-        self.lines = []
-        self.thread = None
+        self.rows = []          # dicts: ts, sm, sm_max, reasons (set of names)
+        self.source = None
+        self._stop = False
+        self._thread = None
+        self._proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.time(), line))
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device_index)
+        try:
+            return pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _poll_nvml(self, handle):
+        import pynvml
+
+        sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+        while not self._stop:
+            try:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle))
+                self.rows.append(dict(ts=time.time(), sm=sm, sm_max=sm_max,
+                                      reasons={n for n, m in self.REASONS if bits & m}))
+            except Exception:
+                pass
+            time.sleep(self.interval_ms / 1e3)
+
+    def _poll_smi(self):
+        for line in self._proc.stdout:
+            r = next(csv.reader([line]), [])
+            if len(r) < 11:
+                continue
+            try:
+                act = {n for n, col in (("hw_slowdown", 7), ("hw_thermal_slowdown", 8), ("sw_thermal_slowdown", 9),
+                                        ("sw_power_cap", 10)) if r[col].strip().lower() == "active"}
+                self.rows.append(dict(ts=time.time(), sm=float(r[2]), sm_max=float(r[3]), reasons=act))
+            except ValueError:
+                continue
 
     def start(self, wait_s: float = 5.0):
         import threading
 
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", f"-lms={self.interval_ms}"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            handle = self._nvml_handle()
+            self.source = f"nvml every {self.interval_ms:g} ms"
+            self._thread = threading.Thread(target=self._poll_nvml, args=(handle,), daemon=True)
         except Exception:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
-        self.thread.start()
+            try:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+                smi_id = vis[self.device_index].strip() if vis and vis[0].strip() else str(self.device_index)
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={smi_id}", f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms=50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                return
+            self.source = "nvidia-smi every 50 ms"
+            self._thread = threading.Thread(target=self._poll_smi, daemon=True)
+        self._thread.start()
         t0 = time.time()
-        while not self.lines and time.time() - t0 < wait_s and self.proc.poll() is None:
-            time.sleep(0.01)
+        while not self.rows and time.time() - t0 < wait_s:
+            time.sleep(0.005)
 
     def mark(self, t0: float, t1: float):
         self.window = (t0, t1)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=10)
-        except Exception:
-            self.proc.kill()
-        if self.thread is not None:
-            self.thread.join(timeout=5)
-        rows = []
-        for t_host, line in list(self.lines):
-            r = next(csv.reader([line]), [])
-            if len(r) < 11:
-                continue
+        self._stop = True
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                rows.append(dict(ts=t_host, sm=float(r[2]), sm_max=float(r[3]), power=float(r[4]),
-                                 util=float(r[5]), hw=r[7].strip(), hw_th=r[8].strip(),
-                                 sw_th=r[9].strip(), pcap=r[10].strip()))
-            except ValueError:
-                continue
+                self._proc.wait(timeout=10)
+            except Exception:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        rows = list(self.rows)
         if not rows:
             return None
         picked, where = rows, "all"
         if self.window:
-            inside = [r for r in rows if self.window[0] <= r["ts"] <= self.window[1] + 0.1]
-            if len(inside) >= 3:
+            inside = [r for r in rows if self.window[0] <= r["ts"] <= self.window[1]]
+            if inside:
                 picked, where = inside, "timed"
-            else:
-                busy = [r for r in rows if r["util"] >= 50]
-                if busy:
-                    picked, where = busy, "busy"
-        reasons = set()
-        for r in picked:
-            for key, name in (("hw", "hw_slowdown"), ("hw_th", "hw_thermal_slowdown"),
-                              ("sw_th", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[key].lower() == "active":
-                    reasons.add(name)
+        reasons = set().union(*(r["reasons"] for r in picked))
         return {"sm_mhz": statistics.median(r["sm"] for r in picked),
                 "sm_max_mhz": max(r["sm_max"] for r in picked),
-                "reasons": sorted(reasons), "samples": len(picked), "window": where}
+                "sm_mhz_min": min(r["sm"] for r in picked),
+                "reasons": sorted(reasons), "samples": len(picked), "window": where, "source": self.source}
 
 
 # ----------------------------------------------------------- the workload
@@ -452,17 +494,83 @@ def workload_bytes(w, s) -> dict:
     return {"nominal": nominal, "minimum": minimum, "units": s.B * s.T * s.Hv}
 
 
-def run_workload(args):
-    """Times one of the smaller workloads (decode_b16, prefix_cow, speculative):
-    ``--steps`` decode calls, back to back (warm L2) and, separately, each call
-    after an L2-flushing write (cold), optionally replayed from a CUDA graph."""
+def _time_calls(call, n: int, stream, graph: bool) -> float:
+    """Microseconds per call over ``n`` back-to-back calls (eager, or one captured graph)."""
+    import torch
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g = None
+    if graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            call()  # one eager call on the capture stream before capturing
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                call()
+        g.replay()
+        torch.cuda.synchronize()
+    ev0.record(stream)
+    if g is not None:
+        g.replay()
+    else:
+        for _ in range(n):
+            call()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    return 1e3 * ev0.elapsed_time(ev1) / n
+
+
+def _time_cold(call, reps: int, stream) -> float:
+    """Median microseconds of one call right after a write of 256 MiB (twice the L2)."""
+    import torch
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    cold = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cold.append(1e3 * e0.elapsed_time(e1))
+    return statistics.median(cold)
+
+
+def oracle_workload_baseline(w, s) -> dict:
+    """The oracle on one whole call of a smaller workload, on the host cores."""
+    import numpy as np
+
+    import oracle
+
+    threads = min(cpu_cores(), s.B)
+    pool = w.pool.copy()
+    out = np.zeros((s.B, s.T, s.Hv, s.dv), np.float32)
+    t0 = time.perf_counter()
+    oracle.decode_step(pool, s.src_idx, np.ascontiguousarray(s.dst_idx.reshape(s.B, s.T)), s.q, s.k, s.v,
+                       s.alpha, s.beta, out, nthreads=threads)
+    dt = time.perf_counter() - t0
+    units = s.B * s.T * s.Hv
+    return {"value": units / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one whole call ({units} tokens*heads), C++ double-precision oracle, {dt:.2f} s"}
+
+
+def measure_workload(name: str, calls: int = 200, warmup: int = 10, variant: str = "auto",
+                     cold_reps: int = 50, graph_too: bool = True, cpu: bool = True) -> dict:
+    """One of the smaller decode workloads (decode_b16, prefix_cow, speculative): its call
+    timed warm (back to back, eager and replayed from one CUDA graph) and cold (after an
+    L2-flushing write), the speculative commit, algorithmic bandwidth against the copy
+    peak, and the oracle on the same call."""
     import numpy as np
     import torch
 
     from hybrid_linear_attention_step_b200 import gdn, workloads as wl
 
-    torch.cuda.set_device(0)
-    w = wl.WORKLOADS[args.workload]()
+    w = wl.WORKLOADS[name]()
     s = w.steps[0]
     to_dev = lambda a: (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
                         if a.dtype == np.uint16 else torch.from_numpy(np.ascontiguousarray(a)).cuda())
@@ -475,96 +583,101 @@ def run_workload(args):
 
     def call():
         args_ = (pool, x["src_idx"], dst, x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
-        if args.variant == "auto":
+        if variant == "auto":
             gdn.gdn_decode_step(*args_, err_word=err)
         else:
-            gdn.gdn_decode_step_variant(*args_, args.variant, err_word=err)
+            gdn.gdn_decode_step_variant(*args_, variant, err_word=err)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         call()
     torch.cuda.synchronize()
-    K = args.steps
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    graph = None
-    if args.graph:
-        side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            call()  # one eager call on the capture stream before capturing
-        stream.wait_stream(side)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for _ in range(K):
-                call()
-        graph.replay()
-        torch.cuda.synchronize()
-    ev0.record(stream)
-    if graph is not None:
-        graph.replay()
-    else:
-        for _ in range(K):
-            call()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    warm_us = 1e3 * ev0.elapsed_time(ev1) / K
-
-    # cold: an L2-sized write before every call, the call alone bracketed by events
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    cold = []
-    for _ in range(min(K, 50)):
-        flush.fill_(1)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        call()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        cold.append(1e3 * e0.elapsed_time(e1))
-    cold_us = statistics.median(cold)
+    warm_us = _time_calls(call, calls, stream, graph=False)
+    graph_us = _time_calls(call, calls, stream, graph=True) if graph_too else None
+    cold_us = _time_cold(call, min(calls, cold_reps), stream)
     code = gdn.gdn_get_error(err)
     if code != 0:
         raise RuntimeError(f"device error word set: {gdn.status_string(code)}")
 
-    commit_us = None
+    commit = None
     if s.accept_len is not None:
         committed = x["src_idx"].clone()
         acc = to_dev(s.accept_len)
+        ccall = lambda: gdn.gdn_commit(acc, committed, dst, w.num_slots, err_word=err)
         for _ in range(3):
-            gdn.gdn_commit(acc, committed, dst, w.num_slots)
+            ccall()
         torch.cuda.synchronize()
-        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        c0.record(stream)
-        for _ in range(100):
-            gdn.gdn_commit(acc, committed, dst, w.num_slots)
-        c1.record(stream)
-        torch.cuda.synchronize()
-        commit_us = 1e3 * c0.elapsed_time(c1) / 100
+        commit = {"us_per_call_eager": _time_calls(ccall, 100, stream, graph=False),
+                  "us_per_call_graph": _time_calls(ccall, 100, stream, graph=True),
+                  "note": "eager calls are bound by the host launch path; the graph figure is device time"}
+        if gdn.gdn_get_error(err) != 0:
+            raise RuntimeError("device error word set by the commit")
 
     hbm_peak, peak_kind = peaks()
     nb = workload_bytes(w, s)
-    line = {
-        "metric": METRIC, "workload": args.workload, "unit": UNIT, "variant": args.variant,
-        "graph": bool(args.graph), "steps": K, "warmup": args.warmup,
-        "value": nb["units"] / (warm_us / 1e6), "us_per_call_warm": warm_us, "us_per_call_cold": cold_us,
-        "bytes_per_call_nominal": nb["nominal"], "bytes_per_call_min": nb["minimum"],
-        "gbs_warm_nominal": nb["nominal"] / warm_us / 1e3, "gbs_cold_nominal": nb["nominal"] / cold_us / 1e3,
-        "gbs_cold_min": nb["minimum"] / cold_us / 1e3, "peak_gbs": hbm_peak, "peak_kind": peak_kind,
-        "commit_us": commit_us,
+    best_warm = min(warm_us, graph_us) if graph_us else warm_us
+    entry = {
+        "workload": name, "variant": variant,
         "config": {"B": s.B, "T": s.T, "Hk": s.Hk, "Hv": s.Hv, "dk": s.dk, "dv": s.dv, "slots": w.num_slots,
-                   "dtype": s.dtype},
+                   "qkv": s.dtype, "state": "f32"},
+        "units_per_call": nb["units"], "calls": calls,
+        "us_per_call_warm": warm_us, "us_per_call_graph": graph_us, "us_per_call_cold": cold_us,
+        "value_warm": nb["units"] / (best_warm / 1e6), "value_cold": nb["units"] / (cold_us / 1e6), "unit": UNIT,
+        "bytes_per_call_nominal": nb["nominal"], "bytes_per_call_min": nb["minimum"],
+        "gbs_cold_nominal": nb["nominal"] / cold_us / 1e3, "gbs_cold_min": nb["minimum"] / cold_us / 1e3,
+        "gbs_warm_nominal": nb["nominal"] / best_warm / 1e3,
+        "frac_cold_nominal": nb["nominal"] / cold_us / 1e3 / hbm_peak,
+        "frac_cold_min": nb["minimum"] / cold_us / 1e3 / hbm_peak,
+        "peak_gbs": hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
+        "l2": "warm: the call's inputs may sit in L2; cold: after a 256 MiB write",
+        "commit": commit,
     }
-    print(json.dumps(line), flush=True)
+    if cpu:
+        entry["cpu_baseline"] = oracle_workload_baseline(w, s)
+    del pool, out
+    torch.cuda.empty_cache()
+    return entry
 
 
-def run_prefill(args):
-    """Times gdn_prefill on a long-prompt batch: B requests x L tokens, Hk=16, Hv=32,
-    dk=dv=128, bf16 inputs; only the final states are stored (checkpoints)."""
+PREFILL_SHAPE = dict(Hk=16, Hv=32, dk=128, dv=128)
+
+
+def oracle_prefill_baseline(q, k, v, a, b, pool_host, pairs, L) -> dict:
+    """The oracle's prefill on a sample of (request, head) pairs over the whole prompt."""
+    import numpy as np
+
+    import oracle
+
+    c = PREFILL_SHAPE
+    G = c["Hv"] // c["Hk"]
+    n = len(pairs)
+    sq = np.stack([q[bb, :, h // G] for bb, h in pairs])[:, :, None, :].copy()
+    sk = np.stack([k[bb, :, h // G] for bb, h in pairs])[:, :, None, :].copy()
+    sv = np.stack([v[bb, :, h] for bb, h in pairs])[:, :, None, :].copy()
+    sa = np.stack([a[bb, :, h] for bb, h in pairs])[:, :, None].copy()
+    sb = np.stack([b[bb, :, h] for bb, h in pairs])[:, :, None].copy()
+    ref_pool = np.zeros((2 * n, 1, c["dk"], c["dv"]), np.float32)
+    ref_pool[:n, 0] = [pool_host[bb, h] for bb, h in pairs]
+    out = np.zeros((n, L, 1, c["dv"]), np.float32)
+    idx = np.arange(n, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill(ref_pool, idx, idx + n, sq, sk, sv, sa, sb, out, nthreads=n)
+    dt = time.perf_counter() - t0
+    return {"value": n * L / dt, "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": f"{n} (request, head) pairs x {L} tokens ({n * L} tokens*heads), C++ double-precision "
+                      f"oracle token loop, {dt:.1f} s"}
+
+
+def measure_prefill(B: int = 4, L: int = 2048, chunked: bool = True, calls: int = 20, warmup: int = 3,
+                    cpu: bool = True, clocks: bool = False) -> dict:
+    """gdn_prefill_chunked (or gdn_prefill) on B requests x L tokens, Hk=16, Hv=32, dk=dv=128,
+    bf16 inputs; only the final states are stored (checkpoints)."""
     import numpy as np
     import torch
 
     from hybrid_linear_attention_step_b200 import gdn, workloads as wl
 
-    torch.cuda.set_device(0)
-    B, L, Hk, Hv, dk, dv = args.prefill_batch, args.prefill_len, 16, 32, 128, 128
+    c = PREFILL_SHAPE
+    Hk, Hv, dk, dv = c["Hk"], c["Hv"], c["dk"], c["dv"]
     rng = np.random.default_rng(6)
     q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, dk, dv, wl.BF16)
     bf = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
@@ -576,60 +689,91 @@ def run_prefill(args):
     dst = torch.arange(B, 2 * B, dtype=torch.int32, device="cuda")
     out = torch.empty((B, L, Hv, dv), dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    if args.chunked:
+    if chunked:
         ws = torch.empty(gdn.gdn_prefill_workspace_bytes(B, L, Hv, dk, dv), dtype=torch.uint8, device="cuda")
         call = lambda: gdn.gdn_prefill_chunked(pool, src, dst, xq, xk, xv, xa, xb, out, ws, err_word=err)
     else:
         call = lambda: gdn.gdn_prefill(pool, src, dst, xq, xk, xv, xa, xb, out, err_word=err)
-    for _ in range(args.warmup):
+    pool_host = pool[:B].cpu().numpy() if cpu else None
+    for _ in range(warmup):
         call()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stream = torch.cuda.current_stream()
-    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0")
-    sampler.start()
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if sampler:
+        sampler.start()
     w0 = time.time()
-    e0.record(stream)
-    for _ in range(args.steps):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    sampler.mark(w0, time.time())
-    clocks = sampler.stop()
+    us = _time_calls(call, calls, stream, graph=False)
+    if sampler:
+        sampler.mark(w0, time.time())
     if gdn.gdn_get_error(err) != 0:
         raise RuntimeError("device error word set during the prefill benchmark")
-    us = 1e3 * e0.elapsed_time(e1) / args.steps
     units = B * L * Hv
-    sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
-    line = {"metric": METRIC, "workload": f"prefill B={B} L={L} Hk={Hk} Hv={Hv} dk=dv={dk}",
-            "kernel": "chunked (gdn_prefill_chunked)" if args.chunked else "token steps (gdn_prefill)", "unit": UNIT,
-            "value": units / (us / 1e6), "us_per_call": us, "steps": args.steps, "warmup": args.warmup,
-            "clocks": clocks}
-    if args.chunked:
-        # I/O the method must move: q, k, v (bf16), alpha, beta, out (fp32), the initial
-        # state read and the checkpoint written.  The workspace round trip (written by the
-        # prepare kernel, read back by the scan) is reported beside it.
-        hbm_peak, peak_kind = peaks()
-        io = B * L * (2 * Hk * dk * 2 + Hv * dv * 2 + 2 * Hv * 4 + Hv * dv * 4) + 2 * B * Hv * dk * dv * 4
+    entry = {"workload": f"prefill B={B} L={L} Hk={Hk} Hv={Hv} dk=dv={dk}, bf16 q/k/v, fp32 state",
+             "kernel": "chunked (gdn_prefill_chunked)" if chunked else "token steps (gdn_prefill)",
+             "units_per_call": units, "calls": calls, "us_per_call": us, "value": units / (us / 1e6), "unit": UNIT,
+             "l2": "inputs, outputs and workspace larger than L2"}
+    hbm_peak, peak_kind = peaks()
+    # I/O the method must move: q, k, v (bf16), alpha, beta, out (fp32), the initial
+    # state read and the checkpoint written.
+    io = B * L * (2 * Hk * dk * 2 + Hv * dv * 2 + 2 * Hv * 4 + Hv * dv * 4) + 2 * B * Hv * dk * dv * 4
+    entry["io_bytes"] = io
+    entry["io_gbs"] = io / us / 1e3
+    entry["io_frac"] = io / us / 1e3 / hbm_peak
+    entry["peak_gbs"] = hbm_peak
+    entry["peak_kind"] = f"{peak_kind} copy bandwidth"
+    if chunked:
         ws_bytes = gdn.gdn_prefill_workspace_bytes(B, L, Hv, dk, dv)
         chunks = (L + 63) // 64
         C = 64
-        # per (request, head, chunk): K K^T, Q K^T, U = T diag(beta) V, W = Tb K, [W;Q] M,
-        # P E, K^T E, and the triangular inverse
-        flop_chunk = 2 * C * C * dk * 2 + 2 * C * C * dv + 2 * 2 * C * dk * dv + 2 * C * C * dv * 2 \
-            + 2 * C * dk * dv + C ** 3 / 3
-        line["roofline"] = {"bound": "hbm", "achieved": io / us / 1e3, "peak": hbm_peak, "unit": "GB/s",
-                            "frac": io / us / 1e3 / hbm_peak, "peak_kind": peak_kind, "io_bytes": io,
-                            "workspace_bytes": ws_bytes,
-                            "with_workspace_frac": (io + 2 * ws_bytes) / us / 1e3 / hbm_peak}
-        line["chunked_tflops"] = B * Hv * chunks * flop_chunk / us / 1e6
-    else:
-        flops = 7.0 * dk * dv * units  # per element: 2 FMA (u, w) + 1 FMA + 1 multiply (update)
-        peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # fp32 FMA lanes x 2 flop x median clock
-        line["roofline"] = {"bound": "alu", "achieved": flops / us / 1e6, "peak": peak_tflops, "unit": "TFLOP/s",
-                            "frac": flops / us / 1e6 / peak_tflops,
-                            "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 flop x median SM clock"}
-    print(json.dumps(line), flush=True)
+        # per (request, head, chunk) in exact arithmetic: K K^T and Q K^T, the triangular
+        # solve for U and W, W M and Q M, P E, K^T E
+        flop_chunk = 2 * 2 * C * C * dk + C * C * (dk + dv) + 2 * 2 * C * dk * dv + 2 * C * C * dv \
+            + 2 * C * dk * dv
+        tflops = B * Hv * chunks * flop_chunk / us / 1e6
+        tpk, tkind = tensor_peak()
+        entry.update({"workspace_bytes": ws_bytes, "with_workspace_frac": (io + 2 * ws_bytes) / us / 1e3 / hbm_peak,
+                      "tflops_algorithmic": tflops, "tensor_peak_tflops": tpk,
+                      "tensor_peak_kind": f"{tkind} dense bf16", "tensor_frac": tflops / tpk})
+    if sampler:
+        entry["clocks"] = sampler.stop()
+    if cpu:
+        pairs = [(i % B, (7 * i) % Hv) for i in range(min(cpu_cores(), 16))]
+        entry["cpu_baseline"] = oracle_prefill_baseline(q, k, v, a, b, pool_host, pairs, L)
+    del pool, out
+    if chunked:
+        del ws
+    torch.cuda.empty_cache()
+    return entry
+
+
+def run_workload(args):
+    """`--workload decode_b16|prefix_cow|speculative`: one line for that workload."""
+    import torch
+
+    torch.cuda.set_device(0)
+    e = measure_workload(args.workload, calls=args.steps, warmup=args.warmup, variant=args.variant,
+                         cpu=not args.no_cpu_baseline)
+    print(json.dumps({"metric": METRIC, **e}), flush=True)
+
+
+def run_prefill(args):
+    """`--workload prefill [--chunked]`: one line for the prefill."""
+    import torch
+
+    torch.cuda.set_device(0)
+    e = measure_prefill(args.prefill_batch, args.prefill_len, args.chunked, calls=args.steps, warmup=args.warmup,
+                        cpu=not args.no_cpu_baseline, clocks=True)
+    print(json.dumps({"metric": METRIC, **e}), flush=True)
+
+
+def measure_configs(cpu: bool) -> dict:
+    """The other synthetic workloads beside the headline, each with its oracle baseline."""
+    out = {}
+    for name in ("decode_b16", "prefix_cow", "speculative"):
+        out[name] = measure_workload(name, cpu=cpu)
+    out["prefill_chunked"] = measure_prefill(4, 2048, True, cpu=cpu)
+    return out
 
 
 # ------------------------------------------------------------------ main
@@ -646,9 +790,7 @@ def run_ours(args):
     if args.fused:
         kernel = kernel.replace(",bf16>", ",bf16,fused>")
     stream = torch.cuda.current_stream()
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
-    smi_id = vis.split(",")[local].strip() if vis else str(local)
-    sampler = ClockSampler(smi_id)
+    sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
 
     for _ in range(args.warmup):
@@ -746,20 +888,31 @@ def run_ours(args):
     value = world * K * wk.units_per_step / (elapsed_ms / 1e3)
     step_gbs = bytes_per_launch * L * K / (elapsed_ms / 1e3) / 1e9  # equals roofline.achieved here
 
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic,
+                "peak_kind": f"{peak_kind} copy bandwidth", "kernel": kernel,
+                "bytes_per_launch": bytes_per_launch, "launch_us": launch_ms * 1e3}
+    if traffic:
+        # The copy probe behind the peak moves its bytes through L2 like any kernel; this
+        # kernel's algorithmic bytes slightly exceed what DRAM sees (ncu traffic), so the
+        # DRAM-side fraction is reported beside the algorithmic one.
+        roofline["frac_traffic"] = traffic / (launch_ms / 1e3) / 1e9 / hbm_peak
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": headline_config(args, world),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": traffic,
-                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": kernel,
-                     "bytes_per_launch": bytes_per_launch, "launch_us": launch_ms * 1e3},
+        "roofline": roofline,
         "hbm_gbs_step": step_gbs, "launch_events": launch_events, "frac_of_8tbs_step": step_gbs / 8000.0,
         "e2e": e2e, "gpu_launches": K * L, "clocks": clocks,
     }
+    if clocks and clocks.get("sm_mhz"):
+        # time x clock: comparable across runs whose SM clocks differ
+        line["ms_x_sm_mhz_per_step"] = elapsed_ms / K * clocks["sm_mhz"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
+    if rank == 0 and world == 1 and not args.no_configs:
+        line["configs"] = measure_configs(cpu=not args.no_cpu_baseline)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -791,6 +944,8 @@ def main():
                     "gate pre-activations and unnormalised q, k, folded into the kernel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="large workload: leave out the smaller workloads' entries (configs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

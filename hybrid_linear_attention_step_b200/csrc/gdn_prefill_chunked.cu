@@ -1377,7 +1377,9 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     if (dk != kD || dv != kD) return GDN_ERR_INVALID_ARG;
     if (qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (B == 0) return GDN_OK;
-    if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out || !workspace)
+    // err_word is required: a bounded wait that runs out leaves the request's checkpoint
+    // and outputs unwritten and reports it only there.
+    if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha || !beta || !out || !workspace || !err_word)
         return GDN_ERR_INVALID_ARG;
     const int nchunks = (L + kC - 1) / kC;
     if (workspace_bytes < gdn_prefill_workspace_bytes(B, L, Hv, dk, dv)) return GDN_ERR_INVALID_ARG;

@@ -357,6 +357,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     const int b = unit / a.Hv;
     const int T = MULTI ? a.T : 1;
 
+    grid_dependency_wait();  // launched with programmatic dependent launch, as gdn_tile1_kernel
     int src, dst0 = 0;
     const int status = request_status(a, b, a.prefill ? 1 : T, src, dst0);
     if (status != kRun) {
@@ -372,6 +373,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     float4 s[RPT];
 #pragma unroll
     for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+    allow_dependent_launch();
 
     const int hk = h / a.G;
     // Token t's inputs: thread j < DK fetches k_j and q_j, thread j < DVC its v
@@ -896,6 +898,10 @@ __global__ void __launch_bounds__(NT, 1) gdn_stream_kernel(StepArgs a) {
 
 __global__ void gdn_commit_kernel(const int32_t* __restrict__ accept_len, int32_t* __restrict__ committed,
                                   const int32_t* __restrict__ cur, int B, int T, int num_slots, int32_t* err) {
+    // Launched with programmatic dependent launch: the decode call before it may still
+    // be draining when this grid starts, so wait for it before reading its tables.
+    grid_dependency_wait();
+    allow_dependent_launch();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     const int acc = accept_len[b];
@@ -958,6 +964,28 @@ constexpr int kMaxDk = 4096;
 #define GDN_TILE_MAXREG 100
 #endif
 
+// Launches a kernel that calls grid_dependency_wait() before its first memory
+// access with programmatic dependent launch (plain stream order without it).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, unsigned threads, cudaStream_t stream, Args... args) {
+#if GDN_USE_PDL
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+#else
+    kernel<<<grid, threads, 0, stream>>>(args...);
+    return cudaSuccess;
+#endif
+}
+
 template <int DK, int DV, bool FUSE>
 gdn_status launch_tile_impl(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
     constexpr int DVC = DV < GDN_TILE_COLS ? DV : GDN_TILE_COLS;
@@ -966,36 +994,17 @@ gdn_status launch_tile_impl(const StepArgs& a, int32_t dtype, cudaStream_t strea
     constexpr int MINB = MINB0 < 1 ? 1 : (MINB0 > 16 ? 16 : MINB0);
     const dim3 grid((unsigned)(a.B * a.Hv * (DV / DVC)));
     const bool bf = dtype == GDN_BF16;
+    cudaError_t e;
     if (a.T == 1) {
-#if GDN_USE_PDL
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = grid;
-        cfg.blockDim = dim3(NT);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const cudaError_t e =
-            bf ? cudaLaunchKernelEx(&cfg, gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, FUSE>, a)
-               : cudaLaunchKernelEx(&cfg, gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float, FUSE>, a);
-        if (e != cudaSuccess) return GDN_ERR_CUDA;
-#else
-        if (bf)
-            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, FUSE><<<grid, NT, 0, stream>>>(a);
-        else
-            gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float, FUSE><<<grid, NT, 0, stream>>>(a);
-#endif
+        e = bf ? launch_pdl(gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, FUSE>, grid, NT, stream, a)
+               : launch_pdl(gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float, FUSE>, grid, NT, stream, a);
     } else {
         // The fused multi-token form needs a few more registers than 5 CTAs/SM allow.
         constexpr int MINB_T = (FUSE && MINB > 1) ? MINB - 1 : MINB;
-        if (bf)
-            gdn_tile_kernel<DK, DV, DVC, NT, MINB_T, __nv_bfloat16, true, FUSE><<<grid, NT, 0, stream>>>(a);
-        else
-            gdn_tile_kernel<DK, DV, DVC, NT, MINB_T, float, true, FUSE><<<grid, NT, 0, stream>>>(a);
+        e = bf ? launch_pdl(gdn_tile_kernel<DK, DV, DVC, NT, MINB_T, __nv_bfloat16, true, FUSE>, grid, NT, stream, a)
+               : launch_pdl(gdn_tile_kernel<DK, DV, DVC, NT, MINB_T, float, true, FUSE>, grid, NT, stream, a);
     }
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -1070,14 +1079,17 @@ gdn_status launch(const StepArgs& a, int32_t dtype, int32_t variant, cudaStream_
         // family serves every shape it supports.
         if (tile_ok(a))
             variant = GDN_VARIANT_TILE;
-        else if (stream_ok(a))
+        else if (stream_ok(a) && a.err != nullptr)
             variant = GDN_VARIANT_STREAM;
         else
             variant = GDN_VARIANT_COLUMN;
     }
     switch (variant) {
         case GDN_VARIANT_STREAM:
-            if (!stream_ok(a)) return GDN_ERR_INVALID_ARG;
+            // Its bounded waits report a timeout only through the error word, and a
+            // unit abandoned that way leaves its destination unwritten: without the
+            // word such a call could not be told from a successful one.
+            if (!stream_ok(a) || a.err == nullptr) return GDN_ERR_INVALID_ARG;
             return bf ? launch_stream<256, __nv_bfloat16>(a, stream) : launch_stream<256, float>(a, stream);
         case GDN_VARIANT_TILE:
             if (!tile_ok(a)) return GDN_ERR_INVALID_ARG;
@@ -1159,8 +1171,9 @@ extern "C" gdn_status gdn_commit(const int32_t* accept_len, int32_t* committed, 
     if (B == 0) return GDN_OK;
     if (!accept_len || !committed || !cur) return GDN_ERR_INVALID_ARG;
     const int threads = 256;
-    gdn_commit_kernel<<<(B + threads - 1) / threads, threads, 0, stream>>>(accept_len, committed, cur, B, T,
-                                                                           num_slots, err_word);
+    if (launch_pdl(gdn_commit_kernel, dim3((unsigned)((B + threads - 1) / threads)), threads, stream, accept_len,
+                   committed, cur, (int)B, (int)T, (int)num_slots, err_word) != cudaSuccess)
+        return GDN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -106,6 +106,17 @@ struct gdn_slot_cache {
         return false;
     }
 
+    // Slots that evictions could free: each distinct checkpoint slot that no
+    // request holds (all of its holders are checkpoints).
+    int64_t evictable_slots() const {
+        std::set<int32_t> slots;
+        for (const auto& e : lru) {
+            const int32_t s = e.second->slot;
+            if (ref[(size_t)s] == tree_ref[(size_t)s]) slots.insert(s);
+        }
+        return (int64_t)slots.size();
+    }
+
     // A free slot with reference count 1, evicting if needed; -1 if none.
     int32_t alloc() {
         if (free_list.empty() && !evict_one()) return -1;
@@ -248,6 +259,18 @@ gdn_status gdn_slot_cache_plan(gdn_slot_cache* c, const int32_t* reqs, int32_t B
             if (!c->valid_req(reqs[b]) || c->reqs[(size_t)reqs[b]].plan_T != 0 || !seen.insert(reqs[b]).second)
                 return GDN_ERR_INVALID_ARG;
         }
+        // Count the fresh slots first: the plan fails before it takes a slot or
+        // evicts a checkpoint, so a failing call changes nothing.  Taking slots
+        // never changes which requests own theirs, nor which checkpoints are
+        // evictable (the planned requests hold their own slots), so the count is exact.
+        int64_t fresh = 0;
+        for (int32_t b = 0; b < B; ++b) {
+            const Request& r = c->reqs[(size_t)reqs[b]];
+            fresh += (T == 1 && c->ref[(size_t)r.slot] == 1) ? 0 : T;
+        }
+        if (fresh > (int64_t)c->free_list.size() &&
+            fresh > (int64_t)c->free_list.size() + c->evictable_slots())
+            return GDN_ERR_CAPACITY;
         std::vector<int32_t> taken;  // fresh slots of this plan, returned if it fails
         for (int32_t b = 0; b < B; ++b) {
             Request& r = c->reqs[(size_t)reqs[b]];

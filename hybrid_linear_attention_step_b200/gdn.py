@@ -209,13 +209,15 @@ def gdn_prefill_workspace_bytes(B: int, L: int, Hv: int, dk: int, dv: int) -> in
 def gdn_prefill_chunked(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
                         q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                         alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
-                        err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
+                        err_word: torch.Tensor, stream=None, check: bool = True) -> int:
     """gdn_prefill computed chunk by chunk (see gdn_prefill_chunked in include/gdn_step.h);
-    ``workspace`` is a CUDA tensor of at least gdn_prefill_workspace_bytes(...) bytes."""
+    ``workspace`` is a CUDA tensor of at least gdn_prefill_workspace_bytes(...) bytes.
+    ``err_word`` (int32 CUDA tensor) is required: a copy or tensor-core wait that runs out is
+    reported only there."""
     args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1)
     nbytes = workspace.numel() * workspace.element_size()
     status = load_library().gdn_prefill_chunked(*args, _dev(workspace, "workspace"), nbytes,
-                                                _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+                                                _dev(err_word, "err_word", torch.int32), _stream_handle(stream))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_prefill_chunked")
     return status

@@ -46,7 +46,14 @@
  * launch returns GDN_ERR_CUDA.  Index errors are found on the device: the
  * affected request is skipped (nothing of it is written) and GDN_ERR_INDEX is
  * recorded in *err_word (first error wins) when err_word is not NULL; read and
- * clear it with gdn_get_error.  Kernels never trap, assert or wait unboundedly.
+ * clear it with gdn_get_error.  Kernels never trap or assert, and every wait a
+ * kernel spins on (copy and tensor-core completions) gives up after 2 s and
+ * records GDN_ERR_TIMEOUT.  One wait is not the kernel's own: the chunked
+ * prefill's tensor-memory allocation (tcgen05.alloc) blocks until the SM has the
+ * columns free.  Its kernels ask for no more than one resident CTA of theirs
+ * leaves (shared memory keeps a second one off the SM), so only a tensor-memory
+ * user outside this library running on the same SM (another stream's sm_100
+ * kernel that holds columns) can delay it, until that kernel releases them.
  */
 #ifndef GDN_STEP_H
 #define GDN_STEP_H
@@ -80,7 +87,8 @@ typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 typedef enum gdn_variant {
     GDN_VARIANT_AUTO = 0,   /* what gdn_decode_step uses: the first of TILE, STREAM, COLUMN that applies */
     GDN_VARIANT_STREAM = 1, /* persistent bulk-copy pipeline through shared memory: T == 1,
-                               dk == dv == 128, every buffer 16-byte aligned, B*Hv % 4 == 0 */
+                               dk == dv == 128, every buffer 16-byte aligned, B*Hv % 4 == 0,
+                               err_word not NULL (a timed-out copy is reported there only) */
     GDN_VARIANT_TILE = 2,   /* state tile held in registers: (dk, dv) in {(128, 128), (64, 64)},
                                pool and out 16-byte aligned, any T; one CTA per 64-column block
                                of a (request, head) tile, which for T > 1 carries its columns
@@ -212,8 +220,12 @@ gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, c
  *                    dk, dv) bytes, 16-byte aligned, caller-owned; contents on entry
  *                    do not matter and on return are unspecified.  Calls sharing one
  *                    workspace must not overlap.
- * Unsupported shapes, a missing or short workspace, or a workspace, pool, out, q, k
- * or v that is not 16-byte aligned return GDN_ERR_INVALID_ARG.
+ *   err_word         device int32, required here (unlike gdn_prefill): besides index
+ *                    errors, a copy or tensor-core wait that runs out (2 s) records
+ *                    GDN_ERR_TIMEOUT, and the affected requests' checkpoints and
+ *                    outputs are then left unwritten.
+ * Unsupported shapes, a missing or short workspace, a NULL err_word, or a workspace,
+ * pool, out, q, k or v that is not 16-byte aligned return GDN_ERR_INVALID_ARG.
  */
 gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const int32_t* src_idx, const int32_t* dst_idx,
                                const void* q, const void* k, const void* v, const float* alpha,
@@ -298,7 +310,11 @@ gdn_status gdn_check_step(const int32_t* src_idx, const int32_t* dst_idx, int32_
  *   before anything is enqueued.
  *   Set-up: the first call on a device (with that device current) looks up the
  *   array's device address with cudaGetSymbolAddress and keeps it for later calls;
- *   make that first call before any stream capture begins.
+ *   make that first call before any stream capture begins.  The kept address
+ *   belongs to the device's current primary context: it does not survive
+ *   cudaDeviceReset (after a reset the module is loaded afresh and the array may
+ *   move), so do not call this entry point again after resetting a device it was
+ *   used on.
  *   Sharing: every call on a device uses the same array.  Each call resets the part
  *   it uses before checking, but calls that overlap on the GPU (different streams,
  *   or different host threads, without ordering between them) race on the array

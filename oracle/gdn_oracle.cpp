@@ -185,20 +185,6 @@ void solve_request(const Problem& p, int64_t b, float* states, float* outs) {
 
 }  // namespace
 
-extern "C" {
-
-// One decode call, with the optional fused prologue (flags: 1 = alpha/beta hold
-// raw x, y; 2 = L2-normalise q and k).  pool: [num_slots][Hv][dk][dv] fp32,
-// updated in place.
-// src_idx: [B]; dst_idx: [B][T]; q, k: [B][T][Hk][dk]; v: [B][T][Hv][dv]
-// (dtype 0 = fp32, 1 = bf16 bit patterns); alpha, beta: [B][T][Hv] fp32;
-// out: [B][T][Hv][dv] fp32.  All buffers are host memory owned by the caller.
-// Every request is solved from the pre-call pool before anything is written;
-// writes then go out in (b, t) order.  nthreads <= 1 runs single-threaded.
-// Returns the number of requests skipped for an out-of-range index (padding
-// requests are not counted), or -1 for invalid sizes.
-}  // extern "C"
-
 namespace {
 
 int64_t run_calls(float* pool, int64_t num_slots, const int32_t* src_idx, const int32_t* dst_idx, const void* q,
@@ -261,6 +247,16 @@ int64_t run_calls(float* pool, int64_t num_slots, const int32_t* src_idx, const 
 
 extern "C" {
 
+// One decode call, with the optional fused prologue (flags: 1 = alpha/beta hold
+// raw x, y; 2 = L2-normalise q and k).  pool: [num_slots][Hv][dk][dv] fp32,
+// updated in place.
+// src_idx: [B]; dst_idx: [B][T]; q, k: [B][T][Hk][dk]; v: [B][T][Hv][dv]
+// (dtype 0 = fp32, 1 = bf16 bit patterns); alpha, beta: [B][T][Hv] fp32;
+// out: [B][T][Hv][dv] fp32.  All buffers are host memory owned by the caller.
+// Every request is solved from the pre-call pool before anything is written;
+// writes then go out in (b, t) order.  nthreads <= 1 runs single-threaded.
+// Returns the number of requests skipped for an out-of-range index (padding
+// requests are not counted), or -1 for invalid sizes.
 int64_t oracle_gdn_decode_step_fused(float* pool, int64_t num_slots, const int32_t* src_idx,
                                      const int32_t* dst_idx, const void* q, const void* k,
                                      const void* v, const float* alpha, const float* beta, float* out,

@@ -52,7 +52,8 @@ def run_gpu(pool_dev, s: wl.Step, out_fill=-7.0, err=None, stream=None, variant=
     """Runs one CUDA decode call on ``pool_dev`` (updated in place); returns out (host).
 
     ``variant`` None goes through gdn_decode_step; a name pins one kernel through
-    gdn_decode_step_variant."""
+    gdn_decode_step_variant.  Without ``err`` the call gets an error word of its own,
+    which must read GDN_OK afterwards."""
     import torch
 
     from hybrid_linear_attention_step_b200 import gdn
@@ -60,11 +61,16 @@ def run_gpu(pool_dev, s: wl.Step, out_fill=-7.0, err=None, stream=None, variant=
     x = step_to_device(s, pool_dev.device)
     out = torch.full((s.B, s.T, s.Hv, s.dv), out_fill, dtype=torch.float32, device=pool_dev.device)
     args = (pool_dev, x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+    own_err = err is None
+    if own_err:
+        err = torch.zeros(1, dtype=torch.int32, device=pool_dev.device)
     if variant is None:
         gdn.gdn_decode_step(*args, err_word=err, stream=stream)
     else:
         gdn.gdn_decode_step_variant(*args, variant, err_word=err, stream=stream)
     torch.cuda.synchronize()
+    if own_err:
+        assert gdn.gdn_get_error(err, stream=stream) == gdn.GDN_OK
     return out.cpu().numpy()
 
 

@@ -122,7 +122,7 @@ def _prefill_chunked(lib, **kw):
     f.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, ctypes.c_size_t,
                   vp, vp]
     a = dict(pool=16, num_slots=4, src=16, dst=16, q=16, k=16, v=16, alpha=16, beta=16, out=16,
-             B=1, L=100, Hk=1, Hv=2, dk=128, dv=128, dtype=1, ws=16, ws_bytes=1 << 30, err=None, stream=None)
+             B=1, L=100, Hk=1, Hv=2, dk=128, dv=128, dtype=1, ws=16, ws_bytes=1 << 30, err=16, stream=None)
     a.update(kw)
     return f(*a.values())
 
@@ -152,6 +152,7 @@ def test_prefill_chunked_validates_on_the_host(lib):
     assert _prefill_chunked(lib, ws_bytes=need - 16) == 1            # short workspace
     assert _prefill_chunked(lib, ws=24, ws_bytes=need) == 1          # workspace not 16-byte aligned
     assert _prefill_chunked(lib, out=20, ws_bytes=need) == 1         # out not 16-byte aligned
+    assert _prefill_chunked(lib, err=None, ws_bytes=need) == 1       # the error word is required
     assert _prefill_chunked(lib, B=0, pool=None, ws=None) == 0       # empty batch: no-op
 
 
@@ -168,3 +169,15 @@ def test_prefill_validates_on_the_host(lib):
     assert call(dtype=9) == 1
     assert call(src=None) == 1
     assert call(B=0, pool=None) == 0  # empty batch: no-op
+
+
+def test_stream_variant_requires_the_error_word(lib):
+    """The bulk-copy decode kernel reports a timed-out copy only through the error word, so
+    the call is refused without one (checked on the host, before any CUDA call)."""
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    f = lib.gdn_decode_step_variant
+    f.restype = i32
+    f.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    args = [16, 8, 16, 16, 16, 16, 16, 16, 16, 16, 4, 1, 1, 1, 128, 128, 1]
+    assert f(*args, None, 1, None) == 1      # GDN_VARIANT_STREAM, no error word
+    assert f(*args, None, 9, None) == 1      # no such variant

@@ -25,7 +25,10 @@ def test_large_decode_sampled_parity():
 
     wk = bench.LargeDecode(layers=8, num_slots=2048, B=256)
     rng = np.random.default_rng(7)
-    picks = [np.sort(rng.choice(wk.B, SAMPLES_PER_LAYER, replace=False)) for _ in range(wk.layers)]
+    # The first and last request of every layer are always among the samples: they sit at
+    # the two ends of the launch grid (blockIdx.x 0 and the last CTAs).
+    picks = [np.sort(np.concatenate([[0, wk.B - 1], 1 + rng.choice(wk.B - 2, SAMPLES_PER_LAYER - 2, replace=False)]))
+             for _ in range(wk.layers)]
     before, untouched = [], []
     for l in range(wk.layers):
         slots = wk.host_steps[l].src_idx[picks[l]]

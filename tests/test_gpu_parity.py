@@ -299,7 +299,7 @@ def test_mismatched_shapes_are_rejected_by_the_binding(torch_cuda):
     ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     with pytest.raises(ValueError):  # a prefill takes one destination per request
         gdn.gdn_prefill_chunked(**{**good, "dst_idx": torch.zeros(32, dtype=torch.int32, device="cuda")},
-                                workspace=ws)
+                                workspace=ws, err_word=torch.zeros(1, dtype=torch.int32, device="cuda"))
     torch.cuda.synchronize()
     assert not bool(pool.any())  # nothing ran
 

@@ -117,6 +117,30 @@ def test_eviction_and_capacity():
     assert np.array_equal(src, dst[:, 0])
 
 
+def test_failing_plan_keeps_evictable_checkpoints():
+    """A plan that needs more fresh slots than free plus evictable ones fails before it
+    takes a slot or evicts a checkpoint: the cached prefix is still a hit afterwards."""
+    c = SlotCache(4)
+    r1, s0, _, _ = c.open([1, 2])
+    c.checkpoint(r1, [1, 2])
+    c.close(r1)  # slot s0 is now held by the tree only: evictable
+    r2 = c.open([3])[0]
+    r3 = c.open([4])[0]
+    before = c.stats()
+    assert before == (1, 1, 2)
+    with pytest.raises(SlotCacheError) as e:  # 4 draft slots wanted, 1 free + 1 evictable
+        c.plan([r2, r3], T=2)
+    assert e.value.status == CAPACITY
+    assert c.stats() == before
+    assert c.refcount(s0) == 1
+    r4, s, matched, needs_init = c.open([1, 2, 9])
+    assert (s, matched, needs_init) == (s0, 2, False)
+    c.close(r4)
+    # one draft each for a single request fits: 1 free + 1 evictable
+    src, cur = c.plan([r2], T=2)
+    assert len(set(cur.ravel())) == 2 and c.stats()[1] == 0
+
+
 def test_invalid_sequences_are_rejected():
     c = SlotCache(8)
     r = c.open([1])[0]

@@ -7,8 +7,8 @@ no-allocation entry point uses an owner map kept in the library's own device mem
 instead.
 
 These tests call it through the C ABI (ctypes on libgdn_b200.so).  Each call's verdict
-must equal the verdict of gdn_check_step, which is given a scratch buffer.  The verdict
-is an integer, so it must match exactly.  Calls come in consecutive pairs, so a second
+must equal both the oracle's brute-force verdict and the verdict of gdn_check_step,
+which is given a scratch buffer.  The verdict is an integer, so it must match exactly.  Calls come in consecutive pairs, so a second
 call would see anything the first one left behind in the shared array.  The file sorts
 last so that a run stopping at the first failure has already run every other test.  It
 also passes when run on its own in a fresh process.
@@ -17,6 +17,8 @@ import ctypes
 
 import numpy as np
 import pytest
+
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -87,7 +89,8 @@ def test_two_calls_in_a_row_match_the_scratch_entry_point(env):
         dst2 = perm[B + B * T:B + 2 * B * T].reshape(B, T).copy()
         calls = [_mutate(src1, dst1, num_slots, kinds[trial % len(kinds)]), (src2, dst2)]
         for n, (src, dst) in enumerate(calls):
-            want = _with_scratch(env, src, dst, num_slots, err)
+            want = oracle.check_step(src, dst, num_slots)
+            assert _with_scratch(env, src, dst, num_slots, err) == want
             got = _noalloc(env, src, dst, num_slots, err)
             assert got == want, (trial, n, src.tolist(), dst.tolist(), got, want)
             if n == 1:
@@ -109,7 +112,7 @@ def test_largest_pool_and_beyond(env):
     for kind in ("ok", "alias"):
         s_, d_ = _mutate(src, dst, limit, kind)
         got = _noalloc(env, s_, d_, limit, err)
-        assert got == _with_scratch(env, s_, d_, limit, err)
+        assert got == _with_scratch(env, s_, d_, limit, err) == oracle.check_step(s_, d_, limit)
         assert got == (gdn.GDN_OK if kind == "ok" else gdn.GDN_ERR_ALIAS)
     src, dst = perm[:4].copy(), perm[4:8].reshape(4, 1).copy()
     s, d = torch.from_numpy(src).cuda(), torch.from_numpy(dst).cuda()
