@@ -770,9 +770,13 @@ def run_prefill(args):
 def measure_configs(cpu: bool) -> dict:
     """The other synthetic workloads beside the headline, each with its oracle baseline."""
     out = {}
-    for name in ("decode_b16", "prefix_cow", "speculative"):
-        out[name] = measure_workload(name, cpu=cpu)
-    out["prefill_chunked"] = measure_prefill(4, 2048, True, cpu=cpu)
+    jobs = [(name, lambda n=name: measure_workload(n, cpu=cpu)) for name in ("decode_b16", "prefix_cow", "speculative")]
+    jobs.append(("prefill_chunked", lambda: measure_prefill(4, 2048, True, cpu=cpu)))
+    for name, job in jobs:
+        try:
+            out[name] = job()
+        except Exception as e:  # one failing entry must not take the headline line with it
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
     return out
 
 

@@ -18,31 +18,25 @@
 //     O   = diag(g) (Q M0) + P E,  P[t][i] = (g_t/g_i)(q_t . k_i), i <= t
 //     M_C = g_C M0 + K^T diag(g_C / g) E                (dk x dv)
 // Kernel 1 builds, for every (request, head, chunk) in parallel, everything that
-// does not depend on the state into the caller's workspace; kernel 2 walks the
-// chunks of each (request, head, column block) in order, carrying M in shared
-// memory.  With bf16 inputs both kernels run their products on the tensor cores
-// (tcgen05, accumulators in TMEM).  An operand that is not a bf16 input is fp32
-// and enters as three bf16 parts (hi + mid + lo carries 24 bits), with every part
-// product formed, which keeps fp32 accuracy.  In that form kernel 1 also computes
-// W = Tb K, so that kernel 2 evaluates the same algebra re-associated:
-//     E = U - W M0,   O = diag(g) (Q M0) + P E,   M_C = g_C M0 + K^T diag(g_C / g) E,
-// all as MMAs.  With fp32 inputs (not exact in bf16) both kernels run on the CUDA
-// cores in the first form.  Ratios g_t / g_i are formed as exp(log g_t - log g_i)
-// <= 1, so nothing overflows; g_t itself may underflow to zero, which is its true
-// value to fp32 precision.
+// does not depend on the state into the caller's workspace; kernel 2 walks each
+// sequence's chunks in order, carrying the state.
 //
-// Workspace record of one (request, head, chunk), bytes.  The first parts are laid
-// out as the shared-memory images the scan copies in (bulk copies, 16-byte granules):
-//   A1  [W_hi; W_mid] then [W_lo; Q] as bf16, two 128 x 128 (dk) tiles in the
-//       no-swizzle K-major core layout of the tensor-core operand, where
-//       W = Tb K is split into three bf16 parts (bf16 inputs only)
-//   A2  K^T as bf16, 128 (dk) rows x 64 tokens, same layout (bf16 inputs only)
-//   PA  [P_hi; P_mid] then [P_lo; P_lo], P split into three bf16 parts, two 128 x 64
-//       operand tiles (bf16 inputs only)
-//   U   four column slabs [4][64][36] fp32 (32 columns + 4 padding each)
-//   TbT [64][64] fp32: Tb transposed, TbT[i][t] = Tb[t][i], zero for t < i (fp32 inputs)
-//   PT  [64][64] fp32: P transposed, PT[i][t] = P[t][i], zero for t < i (fp32 inputs)
-//   G   log g [64]
+// bf16 inputs (tensor cores, tcgen05 with accumulators in TMEM).  Kernel 1 forms
+// [K; Q] K^T as one MMA (exact bf16 products) and solves (I + A) [U | W] =
+// [diag(beta) V | diag(beta g) K] by forward substitution in fp32, W = Tb K, so that
+// kernel 2 evaluates the same algebra re-associated:
+//     E = U - W M0,   O = diag(g) (Q M0) + P E,   M_C = g_C M0 + K^T diag(g_C / g) E,
+// all as MMAs.  Kernel 2 runs one CTA per (request, head) with the whole state: its
+// 128 value rows are the MMA's M dimension and the TMEM lanes.  An operand that is not
+// a bf16 input is fp32 and enters as bf16 parts (hi + mid + lo carries 24 bits); the
+// part products that matter at fp32 precision are formed (the ones left out are named
+// with kernel 2).  With fp32 inputs (not exact in bf16) both kernels run on the CUDA
+// cores in the first form, with T explicit and kernel 2 split into 32-column blocks.
+// Ratios g_t / g_i are formed as exp(log g_t - log g_i) <= 1, so nothing overflows;
+// g_t itself may underflow to zero, which is its true value to fp32 precision.
+//
+// The workspace holds one record per (request, head, chunk); its layouts (one for
+// each input type) are given with the constants below.
 
 #include "gdn_step.h"
 
@@ -60,25 +54,43 @@ constexpr int kNT = 256;        // threads per CTA (both kernels)
 constexpr int kUS = kDVC + 4;   // row stride of the 64 x 32 fp32 tiles (16-byte rows, bank spread)
 constexpr int kPad = 4;         // row padding of [C][D] shared arrays in the fp32 scan kernel
 
-// Workspace record (bytes).
-constexpr size_t kRecA1 = 0;
-constexpr size_t kA1Tile = (size_t)2 * kC * kD * 2;  // one 128 x 128 bf16 operand tile
-constexpr size_t kRecA2 = kRecA1 + 2 * kA1Tile;
-constexpr size_t kA2Tile = (size_t)kD * kC * 2;       // one 128 x 64 bf16 operand tile
-constexpr size_t kRecPA = kRecA2 + kA2Tile;
-constexpr size_t kRecU = kRecPA + 2 * kA2Tile;
+// Workspace record of the fp32-input path (CUDA cores), bytes.
+constexpr size_t kRecU = 0;                             // U in four column slabs [4][64][36] fp32
 constexpr size_t kUSlab = (size_t)kC * kUS * 4;
-constexpr size_t kRecTb = kRecU + kNCB * kUSlab;
-constexpr size_t kRecP = kRecTb + (size_t)kC * kC * 4;
-constexpr size_t kRecG = kRecP + (size_t)kC * kC * 4;
-constexpr size_t kRecBytes = kRecG + (size_t)kC * 4;
-// One scan CTA's small image of a chunk in shared memory: its U slab | log g.
-constexpr uint32_t kImgG = (uint32_t)kUSlab;
-constexpr uint32_t kImgBytes = kImgG + (uint32_t)(kC * 4);
-static_assert(kRecA2 % 16 == 0 && kRecPA % 16 == 0 && kRecU % 16 == 0 && kRecTb % 16 == 0 && kRecP % 16 == 0 &&
-                  kRecBytes % 16 == 0,
+constexpr size_t kRecTb = kRecU + kNCB * kUSlab;        // TbT [64][64] fp32
+constexpr size_t kRecP = kRecTb + (size_t)kC * kC * 4;  // PT [64][64] fp32
+constexpr size_t kRecG = kRecP + (size_t)kC * kC * 4;   // log g [64]
+constexpr size_t kRecF32Bytes = kRecG + (size_t)kC * 4;
+
+// Workspace record of the bf16-input path (tensor cores), bytes: the scan's three
+// shared-memory images, each one contiguous range.
+//   image A  BW  [W_lo | W_mid | W_hi | Q]: 256 rows (tokens, per part) x dk, bf16 parts of
+//                W = T diag(beta g) K and the bf16 Q, K-major no-swizzle operand layout
+//   image B  BK  K^T: dk rows x 64 tokens, same layout
+//            BP  [P_mid | P_hi]: 128 rows (t, per part) x 64 (i), bf16 parts of P
+//   image C  G   g_t [64], g_C / g_t [64], g_C, 3 zero words
+//            UT  U^T [dv][64] fp32: row j holds U[t][j] for the 64 tokens as 16 float4
+//                granules, granule q stored at position q ^ (j & 7) (bank spread)
+constexpr size_t kR2BW = 0;
+constexpr uint32_t kR2BWBytes = 4 * kC * kD * 2;
+constexpr size_t kR2BK = kR2BW + kR2BWBytes;
+constexpr uint32_t kR2BKBytes = kD * kC * 2;
+constexpr size_t kR2BP = kR2BK + kR2BKBytes;
+constexpr uint32_t kR2BPBytes = 2 * kC * kC * 2;
+constexpr size_t kR2G = kR2BP + kR2BPBytes;
+constexpr uint32_t kR2GBytes = (2 * kC + 4) * 4;
+constexpr size_t kR2UT = kR2G + kR2GBytes;
+constexpr uint32_t kR2UTBytes = kD * kC * 4;
+constexpr size_t kR2Bytes = kR2UT + kR2UTBytes;
+constexpr uint32_t kImgA = kR2BWBytes;                 // bytes of image A
+constexpr uint32_t kImgB = kR2BKBytes + kR2BPBytes;    // image B
+constexpr uint32_t kImgC = kR2GBytes + kR2UTBytes;     // image C
+
+constexpr size_t kRecBytes = kR2Bytes > kRecF32Bytes ? kR2Bytes : kRecF32Bytes;
+static_assert(kRecTb % 16 == 0 && kRecP % 16 == 0 && kRecG % 16 == 0 && kR2BK % 16 == 0 && kR2BP % 16 == 0 &&
+                  kR2G % 16 == 0 && kR2UT % 16 == 0 && kRecBytes % 16 == 0,
               "16-byte records");
-static_assert(kUSlab % 16 == 0 && kImgBytes % 16 == 0, "16-byte bulk copies");
+static_assert(kImgA % 16 == 0 && kImgB % 16 == 0 && kImgC % 16 == 0, "16-byte bulk copies");
 
 struct ChunkArgs {
     float* pool;
@@ -260,7 +272,7 @@ __device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& 
 // ---------------------------------------------------------------------------
 
 // Warp 0: log g_t = sum_{i<=t} log alpha_i by a warp scan over two 32-token
-// halves, beta_t, and log g into the record.
+// halves, beta_t, and log g into the record (when Gs is not null).
 __device__ __forceinline__ void gate_scan(const ChunkArgs& a, int b, int h, int t0, int n, int lane, float* lg,
                                           float* bt, float* Gs) {
     float carry = 0.f;
@@ -282,7 +294,7 @@ __device__ __forceinline__ void gate_scan(const ChunkArgs& a, int b, int h, int 
         }
         lg[t] = carry + x;
         bt[t] = be;
-        Gs[t] = carry + x;
+        if (Gs != nullptr) Gs[t] = carry + x;
         carry += __shfl_sync(0xffffffffu, x, 31);
     }
 }
@@ -466,48 +478,38 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 1, tensor-core form (bf16 inputs).  The products with a bf16 input
-// operand run as tcgen05 MMAs with fp32 accumulation in TMEM:
-//   D0 = [K; Q] K^T                    (M = 128, N = 64, K = dk: 8 MMAs, exact products)
-//   D1 = V^T (T diag(beta))^T = U^T    (M = 128 = dv, N = 64, K = 64 tokens; the fp32
-//                                       factor in three bf16 parts: 12 MMAs)
-//   D2 = K^T (T diag(beta g))^T = W^T  (the same with Tb: W = Tb K, 12 MMAs)
-// W is split into three bf16 parts and stored as the scan's A operands
-// [W_hi; W_mid] and [W_lo; Q], so that the scan forms E = U - W M0 and Q M0 on the
-// tensor cores with no triangular product.  The inverse T and the gate scalings
-// stay on the CUDA cores.
+// Kernel 1, tensor-core form (bf16 inputs), one CTA per (request, head, chunk):
+//   D0 = [K; Q] K^T on the tensor cores (M = 128, N = 64, K = dk; exact bf16 products),
+//   read out as A[t][i] = beta_t (g_t / g_i) k_t.k_i (i < t) and P[t][i] =
+//   (g_t / g_i) q_t.k_i (i <= t); then the chunk's unit lower-triangular system
+//   (I + A) [U | W] = [diag(beta) V | diag(beta g) K] solved by forward substitution
+//   in fp32 on the CUDA cores: thread c owns right-hand-side column c (128 columns of
+//   V, 128 of K) and keeps its 64 unknowns in registers, so U and W come out exact to
+//   fp32 rounding with no explicit inverse.  The record receives the scan's operand
+//   images: [W_lo | W_mid | W_hi | Q], K^T and [P_mid | P_hi] as bf16 tensor-core
+//   tiles, the gate factors g_t, g_C / g_t, g_C, and U^T in fp32.
 // ---------------------------------------------------------------------------
 struct SmemP {
     union {
-        unsigned char A1[2 * kC * kD * 2];        // [K; Q] operand of D0 (also B = K)
-        float Y[16][48];                          // scratch of the inverse (after D0)
-        struct {
-            unsigned char VT[kD * kC * 2];        // V^T operand of D1
-            unsigned char Bp[3][kC * kC * 2];     // (T diag(beta)) parts, B of D1
-        } d1;
-        struct {
-            unsigned char KT[kD * kC * 2];        // K^T operand of D2
-            unsigned char Bt[3][kC * kC * 2];     // (T diag(beta g)) parts, B of D2
-        } d2;
-        float W[kC][kD + 4];                      // W staged for its split (row stride spreads banks)
-    } op;
-    union {
-        float A[kC][kC + 1];
-        __nv_bfloat16 R[kC][kD + 2];  // V rows, later K rows (odd word stride for the column gathers)
-    } av;
-    float T[kC][kC + 1];
+        unsigned char KQ[2 * kC * kD * 2];  // [K; Q]: A operand of D0 (rows 0..63 are also its B)
+        __nv_bfloat16 V[kC][kD + 2];        // V rows (right-hand sides), once D0 is complete
+        float W[kC][kD + 4];                // W staged for its split, after the solve
+    } u;
+    __nv_bfloat16 K[kC][kD + 2];            // K rows: right-hand sides and the K^T gather
+    float A[kC][kC + 4];                    // the system's strictly lower part (float4 rows)
     float lg[kC];
     float bt[kC];
+    float gq[kC];                           // g_t
     uint64_t mma;
     uint32_t tmem;
 };
-static_assert(sizeof(SmemP) <= 74 * 1024 + 1024, "three prepare CTAs per SM");
+static_assert(sizeof(SmemP) <= 76 * 1024, "three prepare CTAs per SM");
 
-// Column gather of a bf16 row block R (rows = tokens) into a K-major operand image
-// with kD rows (dk or dv) and kC columns (tokens); optionally also to global memory.
-// Consecutive threads write consecutive 16-byte granules.
-__device__ __forceinline__ void gather_transposed(const __nv_bfloat16 (*R)[kD + 2], unsigned char* img,
-                                                  unsigned char* global_img, int tid) {
+// bf16 row block R (rows = tokens) gathered into a K-major operand image in global
+// memory with kD rows (dk) and kC columns (tokens).  Consecutive threads write
+// consecutive 16-byte granules.
+__device__ __forceinline__ void gather_transposed_global(const __nv_bfloat16 (*R)[kD + 2], unsigned char* img,
+                                                         int tid) {
     for (int e = tid; e < kD * (kC / 8); e += kNT) {
         const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // row j, tokens 8g..8g+7
         uint16_t x[8];
@@ -518,62 +520,52 @@ __device__ __forceinline__ void gather_transposed(const __nv_bfloat16 (*R)[kD + 
         w.y = x[2] | ((uint32_t)x[3] << 16);
         w.z = x[4] | ((uint32_t)x[5] << 16);
         w.w = x[6] | ((uint32_t)x[7] << 16);
-        const uint32_t off = core_off(j, 8 * g, kC);
-        *reinterpret_cast<uint4*>(img + off) = w;
-        if (global_img != nullptr) *reinterpret_cast<uint4*>(global_img + off) = w;
+        *reinterpret_cast<uint4*>(img + core_off(j, 8 * g, kC)) = w;
     }
 }
 
-// B operand (rows t, columns i) = T[t][i] * scale[i], in three bf16 parts.
-__device__ __forceinline__ void split_scaled_T(const float (*T)[kC + 1], const float* scale,
-                                               unsigned char (*parts)[kC * kC * 2], int tid) {
-    for (int e = tid; e < kC * (kC / 8); e += kNT) {
-        const int t = e % kC, g = e / kC;
-        float x[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) x[m] = T[t][8 * g + m] * scale[8 * g + m];
-        uint4 p0, p1, p2;
-        split3x8(x, p0, p1, p2);
-        const uint32_t off = core_off(t, 8 * g, kC);
-        *reinterpret_cast<uint4*>(parts[0] + off) = p0;
-        *reinterpret_cast<uint4*>(parts[1] + off) = p1;
-        *reinterpret_cast<uint4*>(parts[2] + off) = p2;
-    }
+__device__ __forceinline__ void store_row8(__nv_bfloat16* row, const uint4& x) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(row);
+    r[0] = x.x, r[1] = x.y, r[2] = x.z, r[3] = x.w;
 }
 
-__global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
+__global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_p[];
     SmemP& sm = *reinterpret_cast<SmemP*>(smem_p);
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
-    const int c = blockIdx.x % a.nchunks;
-    const int bh = blockIdx.x / a.nchunks;
+    // Chunks in descending order: the records written last are the first ones the scan
+    // reads, so they are still in L2 when it starts.
+    const int nbh = a.B * a.Hv;
+    const int c = a.nchunks - 1 - (int)(blockIdx.x / nbh);
+    const int bh = blockIdx.x % nbh;
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
     const int hk = h / a.G;
     const int t0 = c * kC;
     const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
     unsigned char* rec = record_of(a, bh, c);
-    float* Gs = reinterpret_cast<float*>(rec + kRecG);
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;  // TMEM columns 32*half .. +31 of each accumulator
+    const int half = warp / 4;  // TMEM columns 32*half .. +31 of D0
     constexpr uint32_t kIdesc = umma_idesc(128, kC);
-    constexpr uint32_t kTmemU = 64;  // D1; D0 and then D2 use columns 0..63
 
+    // The scan may be scheduled as soon as every CTA here has started: its CTAs take
+    // whole SMs, so they only land on SMs this grid has left, and wait for it to finish.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         mbar_init(&sm.mma);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
-                     "r"(128)
+                     "r"(64)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-        gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, Gs);
+        gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, nullptr);
     }
-    // k, q, v in 16-byte granules: [K; Q] into the D0 operand image, Q also into the
-    // record's [W_lo; Q] tile (rows 64..127); V stays in registers until the inverse is
-    // done.  Consecutive threads take consecutive granules of the image: token
+    // k, q, v in 16-byte granules: [K; Q] into the D0 operand image, K also into the row
+    // buffer, Q into the record's BW tile (rows 192..255); V stays in registers until D0
+    // is done.  Consecutive threads take consecutive granules of the image: token
     // t = (e & 7) + 8 (e >> 7), group g = (e >> 3) & 15, e = tid + 256 u.
     constexpr int kGr = kC * (kD / 8) / kNT;  // granules per thread
     uint4 vkeep[kGr];
@@ -589,10 +581,10 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             qq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row));
             vv = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + vrow));
         }
-        const uint32_t oq = core_off(kC + t, 8 * g, kD);
-        *reinterpret_cast<uint4*>(sm.op.A1 + core_off(t, 8 * g, kD)) = kq;
-        *reinterpret_cast<uint4*>(sm.op.A1 + oq) = qq;
-        *reinterpret_cast<uint4*>(rec + kRecA1 + kA1Tile + oq) = qq;
+        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(t, 8 * g, kD)) = kq;
+        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(kC + t, 8 * g, kD)) = qq;
+        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(3 * kC + t, 8 * g, kD)) = qq;
+        store_row8(&sm.K[t][8 * g], kq);
         vkeep[u] = vv;
     }
     async_proxy_fence();
@@ -601,16 +593,14 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     if (tid == 0) {
-        const uint32_t a1 = smem_u32(sm.op.A1);
+        const uint32_t kq = smem_u32(sm.u.KQ);
         for (int ks = 0; ks < kD / 16; ++ks)
-            umma_bf16(tmem, umma_desc(a1 + 256 * ks, (kD / 8) * 128), umma_desc(a1 + 256 * ks, (kD / 8) * 128),
+            umma_bf16(tmem, umma_desc(kq + 256 * ks, (kD / 8) * 128), umma_desc(kq + 256 * ks, (kD / 8) * 128),
                       kIdesc, ks != 0 ? 1u : 0u);
         umma_commit(&sm.mma);
     }
-    int waits = 0, issued = 1;
-    bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
+    const bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
     if (ok) {
-        ++waits;
         tc_fence_after();
         // D0 row r < 64: k_r . k_i -> A (scaled); row 64 + t: q_t . k_i -> P (record).
         const int r = (warp % 4) * 32 + lane;
@@ -622,12 +612,17 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             if (r < kC) {
                 const float lt = sm.lg[r], bt = sm.bt[r];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int i = i0 + j;
-                    sm.av.A[r][i] = i < r ? bt * expf(lt - sm.lg[i]) * v[j] : 0.f;
+                for (int j = 0; j < 16; j += 4) {
+                    float x[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int i = i0 + j + m;
+                        x[m] = i < r ? bt * expf(lt - sm.lg[i]) * v[j + m] : 0.f;
+                    }
+                    *reinterpret_cast<float4*>(&sm.A[r][i0 + j]) = make_float4(x[0], x[1], x[2], x[3]);
                 }
             } else {
-                // P row t, columns i0..i0+15, in three bf16 parts: [P_hi; P_mid] and [P_lo; P_lo].
+                // P row t, columns i0..i0+15: its mid and hi bf16 parts into [P_mid | P_hi].
                 const int t = r - kC;
                 const float lt = sm.lg[t];
 #pragma unroll
@@ -640,128 +635,94 @@ __global__ void __launch_bounds__(kNT, 3) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                     }
                     uint4 p0, p1, p2;
                     split3x8(x, p0, p1, p2);
-                    unsigned char* pa = rec + kRecPA;
-                    *reinterpret_cast<uint4*>(pa + core_off(t, i0 + g8, kC)) = p0;
-                    *reinterpret_cast<uint4*>(pa + core_off(kC + t, i0 + g8, kC)) = p1;
-                    *reinterpret_cast<uint4*>(pa + kA2Tile + core_off(t, i0 + g8, kC)) = p2;
-                    *reinterpret_cast<uint4*>(pa + kA2Tile + core_off(kC + t, i0 + g8, kC)) = p2;
+                    unsigned char* bp = rec + kR2BP;
+                    *reinterpret_cast<uint4*>(bp + core_off(t, i0 + g8, kC)) = p1;
+                    *reinterpret_cast<uint4*>(bp + core_off(kC + t, i0 + g8, kC)) = p0;
                 }
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        invert_unit_lower(sm.av.A, sm.T, sm.op.Y, tid);  // the [K; Q] image is dead: D0 is complete
-        // V rows over A (dead after the inverse)
-#pragma unroll
-        for (int u = 0; u < kGr; ++u) {
-            const int e = tid + kNT * u;
-            const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-            uint32_t* vr = reinterpret_cast<uint32_t*>(&sm.av.R[t][8 * g]);
-            vr[0] = vkeep[u].x, vr[1] = vkeep[u].y, vr[2] = vkeep[u].z, vr[3] = vkeep[u].w;
-        }
-        if (tid < kC) sm.lg[tid] = sm.bt[tid] * expf(sm.lg[tid]);  // beta g: log g is in the record already
-        __syncthreads();
-
-        // D1 = U^T: V^T and (T diag(beta)) in parts.
-        gather_transposed(sm.av.R, sm.op.d1.VT, nullptr, tid);
-        split_scaled_T(sm.T, sm.bt, sm.op.d1.Bp, tid);
-        async_proxy_fence();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            const uint32_t vt = smem_u32(sm.op.d1.VT);
-            for (int part = 0; part < 3; ++part)
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem + kTmemU, umma_desc(vt + 256 * ks, (kC / 8) * 128),
-                              umma_desc(smem_u32(sm.op.d1.Bp[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
-                              (part | ks) != 0 ? 1u : 0u);
-            umma_commit(&sm.mma);
-        }
-        ++issued;
-        // K rows again (just read, so from L2) into the row buffer for the K^T image.
-#pragma unroll
-        for (int u = 0; u < kGr; ++u) {
-            const int e = tid + kNT * u;
-            const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-            uint4 kq = make_uint4(0, 0, 0, 0);
-            if (t < n)
-                kq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) +
-                                                          (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD + 8 * g));
-            uint32_t* kr = reinterpret_cast<uint32_t*>(&sm.av.R[t][8 * g]);
-            kr[0] = kq.x, kr[1] = kq.y, kr[2] = kq.z, kr[3] = kq.w;
-        }
-        ok = !__syncthreads_or(wait_parity(&sm.mma, 1) ? 0 : 1);
-        if (ok) {
-            ++waits;
-            tc_fence_after();
-            // D1[j][t] = U[t][j]: lane j of this warp's quadrant, tokens 32*half .. +31.
-            const int j = (warp % 4) * 32 + lane;
-            float* U = reinterpret_cast<float*>(rec + kRecU) + (j / kDVC) * (kC * kUS) + j % kDVC;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                float v[16];
-                const int tb = 32 * half + 16 * part;
-                tmem_ld16(tmem + lane_base + kTmemU + (uint32_t)tb, v);
-#pragma unroll
-                for (int m = 0; m < 16; ++m) U[(tb + m) * kUS] = v[m];
-            }
-            // D2 = W^T: K^T (also the scan's operand, to the record) and (T diag(beta g)) in parts.
-            gather_transposed(sm.av.R, sm.op.d2.KT, rec + kRecA2, tid);
-            split_scaled_T(sm.T, sm.lg, sm.op.d2.Bt, tid);
-            async_proxy_fence();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            if (tid == 0) {
-                const uint32_t kt = smem_u32(sm.op.d2.KT);
-                for (int part = 0; part < 3; ++part)
-                    for (int ks = 0; ks < kC / 16; ++ks)
-                        umma_bf16(tmem, umma_desc(kt + 256 * ks, (kC / 8) * 128),
-                                  umma_desc(smem_u32(sm.op.d2.Bt[part]) + 256 * ks, (kC / 8) * 128), kIdesc,
-                                  (part | ks) != 0 ? 1u : 0u);
-                umma_commit(&sm.mma);
-            }
-            ++issued;
-            ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
-            if (ok) {
-                ++waits;
-                tc_fence_after();
-                // D2[d][t] = W[t][d] -> W staged row-major (the operands of D2 are dead).
-                const int d = (warp % 4) * 32 + lane;
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    float v[16];
-                    const int tb = 32 * half + 16 * part;
-                    tmem_ld16(tmem + lane_base + (uint32_t)tb, v);
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) sm.op.W[tb + m][d] = v[m];
-                }
-                __syncthreads();
-                // [W_hi; W_mid] and [W_lo; (Q, written above)] to the record.
-                for (int e = tid; e < kC * (kD / 8); e += kNT) {
-                    const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-                    const float4 w0 = *reinterpret_cast<const float4*>(&sm.op.W[t][8 * g]);
-                    const float4 w1 = *reinterpret_cast<const float4*>(&sm.op.W[t][8 * g + 4]);
-                    const float x[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                    uint4 p0, p1, p2;
-                    split3x8(x, p0, p1, p2);
-                    *reinterpret_cast<uint4*>(rec + kRecA1 + core_off(t, 8 * g, kD)) = p0;
-                    *reinterpret_cast<uint4*>(rec + kRecA1 + core_off(kC + t, 8 * g, kD)) = p1;
-                    *reinterpret_cast<uint4*>(rec + kRecA1 + kA1Tile + core_off(t, 8 * g, kD)) = p2;
-                }
-            }
-        }
-    }
-    if (!ok && tid == 0) {
+    } else if (tid == 0) {
         record(a.err, GDN_ERR_TIMEOUT);
-        for (; waits < issued; ++waits) wait_parity(&sm.mma, (uint32_t)waits & 1u);
+        wait_parity(&sm.mma, 0);  // one more bounded wait before the accumulator is freed
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64) : "memory");
+    if (!ok) return;
+
+    // V rows over the [K; Q] image (D0 is complete); g_t.
+#pragma unroll
+    for (int u = 0; u < kGr; ++u) {
+        const int e = tid + kNT * u;
+        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+        store_row8(&sm.u.V[t][8 * g], vkeep[u]);
+    }
+    if (tid < kC) sm.gq[tid] = expf(sm.lg[tid]);
+    __syncthreads();
+
+    // Forward substitution, one right-hand-side column per thread: x_r = rhs_r -
+    // sum_{m < r} A[r][m] x_m, rows in order, four partial sums per row.
+    const bool is_u = tid < kD;  // warp-uniform: warps 0..3 solve for U, 4..7 for W
+    const int col = is_u ? tid : tid - kD;
+    float x[kC];
+#pragma unroll
+    for (int r = 0; r < kC; ++r) {
+        const float rhs = is_u ? sm.bt[r] * __bfloat162float(sm.u.V[r][col])
+                               : (sm.bt[r] * sm.gq[r]) * __bfloat162float(sm.K[r][col]);
+        float acc0 = rhs, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+        for (int m = 0; m < (r & ~3); m += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(&sm.A[r][m]);
+            acc0 = fmaf(-a4.x, x[m], acc0);
+            acc1 = fmaf(-a4.y, x[m + 1], acc1);
+            acc2 = fmaf(-a4.z, x[m + 2], acc2);
+            acc3 = fmaf(-a4.w, x[m + 3], acc3);
+        }
+        if (r & 3) {
+            const float4 a4 = *reinterpret_cast<const float4*>(&sm.A[r][r & ~3]);
+            const int m = r & ~3;
+            acc0 = fmaf(-a4.x, x[m], acc0);
+            if ((r & 3) > 1) acc1 = fmaf(-a4.y, x[m + 1], acc1);
+            if ((r & 3) > 2) acc2 = fmaf(-a4.z, x[m + 2], acc2);
+        }
+        x[r] = (acc0 + acc1) + (acc2 + acc3);
+    }
+    __syncthreads();  // every thread is done with V (the union is rewritten next)
+
+    if (is_u) {
+        // U^T row col: 16 float4 granules, granule q at position q ^ (col & 7).
+        float4* ut = reinterpret_cast<float4*>(rec + kR2UT) + col * (kC / 4);
+#pragma unroll
+        for (int q = 0; q < kC / 4; ++q)
+            ut[q ^ (col & 7)] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+    } else {
+#pragma unroll
+        for (int r = 0; r < kC; ++r) sm.u.W[r][col] = x[r];
+    }
+    float* G = reinterpret_cast<float*>(rec + kR2G);
+    if (tid < kC) {
+        G[tid] = sm.gq[tid];
+        G[kC + tid] = expf(sm.lg[kC - 1] - sm.lg[tid]);
+    } else if (tid < kC + 4) {
+        G[kC + tid] = tid == kC ? sm.gq[kC - 1] : 0.f;  // g_C, then zero padding
+    }
+    __syncthreads();
+
+    // W in three bf16 parts into the BW tile: W_lo rows 0..63, W_mid 64..127, W_hi 128..191.
+    for (int e = tid; e < kC * (kD / 8); e += kNT) {
+        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+        const float4 w0 = *reinterpret_cast<const float4*>(&sm.u.W[t][8 * g]);
+        const float4 w1 = *reinterpret_cast<const float4*>(&sm.u.W[t][8 * g + 4]);
+        const float xw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint4 p0, p1, p2;
+        split3x8(xw, p0, p1, p2);
+        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(t, 8 * g, kD)) = p2;
+        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(kC + t, 8 * g, kD)) = p1;
+        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(2 * kC + t, 8 * g, kD)) = p0;
+    }
+    gather_transposed_global(sm.K, rec + kR2BK, tid);
 }
 
 // Reads (src, dst) of request b and classifies it: 0 run, 1 padding (skipped
@@ -967,371 +928,332 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 2, tensor-core form (bf16 inputs).  Per chunk, with the fp32 state block M
-// (128 x 32, held in registers: each thread owns the 16 elements it reads from D2)
-// split into three bf16 parts stacked along N = 3 x 32:
-//   D1a = [W_hi; W_mid] [M_hi M_mid M_lo]   (8 MMAs, K = dk)
-//   D1b = [W_lo; Q]     [M_hi M_mid M_lo]   (8 MMAs)
-//   E   = U - (W_hi + W_mid + W_lo) M       (rows 0..63 of D1a and D1b, rows 64..127 of D1a)
-//   QM  = diag(g) Q M                       (rows 64..127 of D1b)
-//   D2  = K^T [E'_hi E'_mid E'_lo],  E' = diag(g_C / g) E   (4 MMAs, K = 64 tokens)
-//   DOa = [P_hi; P_mid] [E_hi E_mid E_lo],  DOb = [P_lo; P_lo] [E parts]  (4 + 4 MMAs)
-//   O   = QM + (P_hi + P_mid + P_lo) E,     M <- g_C M + D2
-// The sequential chain holds no CUDA-core contraction.  The column groups of each
-// accumulator are added when TMEM is read, and rows that two TMEM quadrants hold
-// are combined through shared memory.  Operands sit in shared memory in the
-// no-swizzle K-major core layout; the accumulators take 3 x 96 of 512 TMEM columns
-// (D1a, then DOa, at 0; D1b, then DOb, at 128; D2 at 256), allocated by warp 0.
-// Thread 0 issues the MMAs, commits them to an mbarrier, and streams the chunk
-// images with cp.async.bulk: the A operands ([W; Q] tiles; K^T with the P tiles;
-// one buffer each, refilled for the next chunk as soon as their MMAs complete) and
-// the small image (U slab, log g; two buffers, two chunks ahead).  Every wait is bounded (2 s); a timeout is
+// Kernel 2, tensor-core form (bf16 inputs): one CTA per (request, head) walks the
+// chunks in order with the whole state in registers, transposed: thread (w, lane)
+// holds S[j][i] = M[i][j] for value row j = 32 (w % 4) + lane and key columns
+// i in [64 (w / 4), +64).  Row j is TMEM lane j of every accumulator, so the thread
+// that reads an accumulator row is the one that owns that row of the state.
+// Per chunk, with S split into three bf16 parts (S = S_hi + S_mid + S_lo) as the A
+// operand (M = 128 value rows, K = dk) and the record's tile [W_lo | W_mid | W_hi | Q]
+// as B (N = 64 tokens per part):
+//   G   = S_hi [W_lo W_mid W_hi Q] + S_mid [W_mid W_hi Q] + S_lo [W_hi]   (TMEM cols 0..255)
+//   E^T = U^T - (G0 + G1 + G2) = (U - W M)^T,    QM^T = G3 (q M per token), scaled by g_t
+// (the part products left out are below 2^-24 of W M, and 2^-16 of Q M, an output-only
+// term).  Then with E' = diag(g_C / g) E split in three parts and E in two as A operands
+// (K = 64 tokens):
+//   D_U = E'^T K              (B = K^T tile; cols 256..383)   ->  S <- g_C S + D_U
+//   D_O = E_hi [P_mid P_hi] + E_mid [P_hi]   (cols 384..511)  ->  o = g Q M + P E
+// The state update is committed first; the chain waits only for it, splits the new
+// state for the next chunk and issues that chunk's first products, and the outputs
+// are read out and stored while those run.  Thread 0 issues the MMAs and streams the
+// three record images with cp.async.bulk: each buffer is refilled for the next chunk
+// as soon as its last reader is done.  Every wait is bounded (2 s); a timeout is
 // recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kBopPart = (uint32_t)kDVC * kD * 2;   // one bf16 part of M^T (32 x 128)
-constexpr uint32_t kBopPartE = (uint32_t)kDVC * kC * 2;  // one bf16 part of E'^T (32 x 64)
+constexpr uint32_t kSPart = (uint32_t)kD * kD * 2;  // one bf16 part of S (128 x 128)
+constexpr uint32_t kEPart = (uint32_t)kD * kC * 2;  // one bf16 part of E^T or E'^T (128 x 64)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemD1b = 128;
-constexpr uint32_t kTmemD2 = 256;
+constexpr uint32_t kTmemDU = 256;
+constexpr uint32_t kTmemDO = 384;
 
-struct SmemTC {
-    unsigned char a1[2 * kA1Tile];      // [W_hi; W_mid] | [W_lo; Q]
-    unsigned char a2[3 * kA2Tile];      // K^T (D2), [P_hi; P_mid] (DOa), [P_lo; P_lo] (DOb)
-    unsigned char img[2][kImgBytes];    // small images, double-buffered
-    unsigned char bop[3 * kBopPart];    // B operand, three stacked parts: M^T, later E'^T
-    unsigned char bopE[3 * kBopPartE];  // B operand of DO: E^T in three stacked parts
-    float S[kC][kUS];                   // rows handed between TMEM quadrants: W_mid M, then QM + P_mid E
-    float QM[kC][kUS];                  // diag(g) Q M
-    uint64_t full[2];                   // small images
-    uint64_t bar_a1, bar_a2, mma;
+struct SmemS {
+    unsigned char aop[3 * kSPart];  // A operands: S parts; then E'^T parts (3) and E^T parts (hi, mid)
+    unsigned char imgA[kImgA];      // [W_lo | W_mid | W_hi | Q]
+    unsigned char imgB[kImgB];      // K^T | [P_mid | P_hi]
+    unsigned char imgC[kImgC];      // g_t, g_C / g_t, g_C | U^T
+    uint64_t bar_a, bar_b, bar_c, mma_g, mma_u, mma_o;
     uint32_t tmem;
     int src, dst, status;
 };
-
-// 8 x 8 transpose of 32-bit values across each group of 8 lanes: on entry lane l
-// (l = lane % 8) holds row l of the block in x[0..7]; on return it holds column l
-// (x[r] = row r's element l).  Three butterfly stages exchange 4 x 4, 2 x 2 and
-// 1 x 1 sub-blocks with the partner lane l ^ s.
-__device__ __forceinline__ void transpose8(float (&x)[8], int lane) {
-#pragma unroll
-    for (int s = 4; s >= 1; s >>= 1) {
-        const bool upper = (lane & s) != 0;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            if (c & s) continue;
-            const float send = upper ? x[c] : x[c + s];
-            const float got = __shfl_xor_sync(0xffffffffu, send, s);
-            if (upper)
-                x[c] = got;
-            else
-                x[c + s] = got;
-        }
-    }
-}
+static_assert(sizeof(SmemS) <= 227 * 1024, "scan shared memory plan exceeds the per-CTA limit");
+static_assert(3 * kEPart + 2 * kEPart <= 3 * kSPart, "E parts overlay the S parts");
 
 __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_tc[];
-    SmemTC& sm = *reinterpret_cast<SmemTC*>(smem_tc);
+    SmemS& sm = *reinterpret_cast<SmemS*>(smem_tc);
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
-    const int cb = blockIdx.x % kNCB;
-    const int bh = blockIdx.x / kNCB;
+    const int bh = blockIdx.x;
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
-    const int col0 = cb * kDVC;
-    constexpr uint32_t kIdesc = umma_idesc(128, 3 * kDVC);
+    const int half = warp / 4;                     // key columns 64*half.., tokens 32*half..
+    const int j = (warp % 4) * 32 + lane;          // value row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const int nch = a.nchunks;
 
-    // Thread 0's copies.  Every barrier completes once per chunk (or once per
-    // use of its buffer), so the parity of the n-th completion is n & 1.
-    auto issue_small = [&](int c) {
-        const unsigned char* rec = record_of(a, bh, c);
-        unsigned char* dst = sm.img[c & 1];
-        uint64_t* bar = &sm.full[c & 1];
-        mbar_expect_tx(bar, kImgBytes);
-        bulk_g2s(dst, rec + kRecU + cb * kUSlab, (uint32_t)kUSlab, bar);
-        bulk_g2s(dst + kImgG, rec + kRecG, (uint32_t)(kC * 4), bar);
+    auto issue_a = [&](int c) {
+        mbar_expect_tx(&sm.bar_a, kImgA);
+        bulk_g2s(sm.imgA, record_of(a, bh, c) + kR2BW, kImgA, &sm.bar_a);
     };
-    auto issue_a1 = [&](int c) {
-        mbar_expect_tx(&sm.bar_a1, (uint32_t)(2 * kA1Tile));
-        bulk_g2s(sm.a1, record_of(a, bh, c) + kRecA1, (uint32_t)(2 * kA1Tile), &sm.bar_a1);
+    auto issue_b = [&](int c) {
+        mbar_expect_tx(&sm.bar_b, kImgB);
+        bulk_g2s(sm.imgB, record_of(a, bh, c) + kR2BK, kImgB, &sm.bar_b);
     };
-    auto issue_a2 = [&](int c) {
-        mbar_expect_tx(&sm.bar_a2, (uint32_t)(3 * kA2Tile));
-        bulk_g2s(sm.a2, record_of(a, bh, c) + kRecA2, (uint32_t)(3 * kA2Tile), &sm.bar_a2);
+    auto issue_c = [&](int c) {
+        mbar_expect_tx(&sm.bar_c, kImgC);
+        bulk_g2s(sm.imgC, record_of(a, bh, c) + kR2G, kImgC, &sm.bar_c);
     };
 
     if (tid == 0) {
-        scan_prologue(a, b, sm.src, sm.dst, sm.status);
-        mbar_init(&sm.full[0]);
-        mbar_init(&sm.full[1]);
-        mbar_init(&sm.bar_a1);
-        mbar_init(&sm.bar_a2);
-        mbar_init(&sm.mma);
+        mbar_init(&sm.bar_a);
+        mbar_init(&sm.bar_b);
+        mbar_init(&sm.bar_c);
+        mbar_init(&sm.mma_g);
+        mbar_init(&sm.mma_u);
+        mbar_init(&sm.mma_o);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (sm.status == 0) {
-            issue_a1(0);
-            issue_a2(0);
-            issue_small(0);
-            if (nch > 1) issue_small(1);
-        }
     }
-    __syncthreads();
-    if (sm.status != 0) return;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;             // TMEM columns half*16 .. +15 of each 32-column group
-    const int row = (warp % 4) * 32 + lane;  // TMEM lane
-    // The state block lives in registers: this thread owns M[row][half*16 .. +15], the
-    // elements it reads from D2 in every state update.
-    float m[16];
-    {
-        const float4* M0 = reinterpret_cast<const float4*>(a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) +
-                                                           (size_t)row * kD + col0 + half * 16);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 v = M0[j];
-            m[4 * j] = v.x, m[4 * j + 1] = v.y, m[4 * j + 2] = v.z, m[4 * j + 3] = v.w;
+    // Launched with programmatic dependent launch behind the prepare kernel: the set-up
+    // above overlaps its tail; the records, indices and pool are read only after it.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) {
+        scan_prologue(a, b, sm.src, sm.dst, sm.status);
+        if (sm.status == 0) {
+            issue_a(0);
+            issue_b(0);
+            issue_c(0);
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    const uint64_t da1 = umma_desc(smem_u32(sm.a1), (kD / 8) * 128);
-    const uint64_t da1b = umma_desc(smem_u32(sm.a1 + kA1Tile), (kD / 8) * 128);
-    const uint64_t da2 = umma_desc(smem_u32(sm.a2), (kC / 8) * 128);
-    const uint64_t dpa = umma_desc(smem_u32(sm.a2 + kA2Tile), (kC / 8) * 128);
-    const uint64_t dpb = umma_desc(smem_u32(sm.a2 + 2 * kA2Tile), (kC / 8) * 128);
+    if (sm.status != 0) {
+        if (warp == 0)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                         : "memory");
+        return;
+    }
+
+    float s[64];  // S[j][64 half + i]
+    {
+        const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) + (size_t)(64 * half) * kD + j;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s[i] = M0[(size_t)i * kD];
+    }
+    // A operand of the first products: S in three bf16 parts, row j, 8 key columns per granule.
+    auto split_s = [&]() {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float x8[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) x8[m] = s[8 * u + m];
+            uint4 p0, p1, p2;
+            split3x8(x8, p0, p1, p2);
+            const uint32_t off = core_off(j, 64 * half + 8 * u, kD);
+            *reinterpret_cast<uint4*>(sm.aop + off) = p0;
+            *reinterpret_cast<uint4*>(sm.aop + kSPart + off) = p1;
+            *reinterpret_cast<uint4*>(sm.aop + 2 * kSPart + off) = p2;
+        }
+        async_proxy_fence();
+    };
+    split_s();
+
+    constexpr uint32_t kIdesc256 = umma_idesc(128, 256), kIdesc192 = umma_idesc(128, 192);
+    constexpr uint32_t kIdesc128 = umma_idesc(128, 128), kIdesc64 = umma_idesc(128, 64);
     bool ok = true;
+    int done_a = 0, done_b = 0, done_c = 0, issued_a = 1, issued_b = 1, issued_c = 1;
+    int waits_g = 0, waits_u = 0, waits_o = 0, issued_g = 0, issued_u = 0, issued_o = 0;
+    float qm[32];   // g_t (q_t M)_j for this thread's 32 tokens of the current chunk
+    int out_t0 = 0, out_n = 0;  // chunk whose outputs are pending
+
+    // Outputs of the chunk whose D_O was last committed: o = g q M + P E.
+    auto store_outputs = [&]() {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const uint32_t col = (uint32_t)(32 * half + 16 * p);
+            uint32_t r0[16], r1[16];
+            tmem_ld16_issue(tmem + lane_base + kTmemDO + col, r0);
+            tmem_ld16_issue(tmem + lane_base + kTmemDO + kC + col, r1);
+            tmem_wait_ld();
+            tie_regs(r0), tie_regs(r1);
+            float* ob = a.out + (((size_t)b * a.L + out_t0) * a.Hv + h) * kD + j;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int t = (int)col + m;
+                if (t < out_n)
+                    ob[(size_t)t * a.Hv * kD] = qm[16 * p + m] + (__uint_as_float(r1[m]) + __uint_as_float(r0[m]));
+            }
+        }
+    };
+
     int c = 0;
-    int waits_mma = 0;   // completed waits per barrier (all threads); thread 0 also
-    int done_a1 = 0, done_a2 = 0, done_small = 0;  // counts what it issued, below
-    int issued_a1 = 1, issued_a2 = 1, issued_small = min(nch, 2), issued_mma = 0;
-
-    // Sum of the three column groups (bf16 parts) of an accumulator, 16 columns at col:
-    // the three loads are in flight together.
-    auto read3 = [&](uint32_t col, float (&v)[16]) {
-        uint32_t r0[16], r1[16], r2[16];
-        tmem_ld16_issue(tmem + lane_base + col, r0);
-        tmem_ld16_issue(tmem + lane_base + col + kDVC, r1);
-        tmem_ld16_issue(tmem + lane_base + col + 2 * kDVC, r2);
-        tmem_wait_ld();
-        tie_regs(r0), tie_regs(r1), tie_regs(r2);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            v[j] = (__uint_as_float(r2[j]) + __uint_as_float(r1[j])) + __uint_as_float(r0[j]);
-    };
-
-    // B of D1: M^T (32 rows x 128) in three bf16 parts, 8 k-values per granule.  Each
-    // group of 8 lanes transposes its 8 rows x 16 columns, so that lane l holds columns
-    // l and 8 + l of those rows: two granules.  The caller fences and synchronises.
-    auto split_m = [&]() {
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            float x[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = m[8 * blk + j];
-            transpose8(x, lane);
-            uint4 p0, p1, p2;
-            split3x8(x, p0, p1, p2);
-            const uint32_t off = core_off(half * 16 + 8 * blk + (lane & 7), row & ~7, kD);
-            *reinterpret_cast<uint4*>(sm.bop + off) = p0;
-            *reinterpret_cast<uint4*>(sm.bop + kBopPart + off) = p1;
-            *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPart + off) = p2;
-        }
-        async_proxy_fence();
-    };
-    split_m();  // the first chunk's; the barrier after the first wait orders it before the MMAs
-
     for (; c < nch; ++c) {
-        const int s = c & 1;
-        bool got = wait_parity(&sm.full[s], (uint32_t)(c >> 1) & 1u);
-        got = wait_parity(&sm.bar_a1, (uint32_t)c & 1u) && got;
+        // --- the chunk's first products: S parts x [W parts | Q]
+        bool got = wait_parity(&sm.bar_a, (uint32_t)c & 1u);
+        async_proxy_fence();
+        tc_fence_before();
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++done_small, ++done_a1;
-        unsigned char* img = sm.img[s];
-        float* U = reinterpret_cast<float*>(img);  // [64][kUS]: U, then E
-        const float* lg = reinterpret_cast<const float*>(img + kImgG);
-        const int t0 = c * kC;
-        const int n = min(kC, a.L - t0);
-
-        // (B of D1, the parts of M, was built after the previous state update.)
+        ++done_a;
+        tc_fence_after();
         if (tid == 0) {
-            const uint64_t db = umma_desc(smem_u32(sm.bop), (kD / 8) * 128);
-            for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(tmem, da1 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
+            const uint32_t aS = smem_u32(sm.aop), bW = smem_u32(sm.imgA);
+            constexpr uint32_t kSbo = (kD / 8) * 128;
             for (int ks = 0; ks < kD / 16; ++ks)
-                umma_bf16(tmem + kTmemD1b, da1b + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
-            umma_commit(&sm.mma);
+                umma_bf16(tmem, umma_desc(aS + 256 * ks, kSbo), umma_desc(bW + 256 * ks, kSbo), kIdesc256,
+                          ks != 0 ? 1u : 0u);
+            for (int ks = 0; ks < kD / 16; ++ks)
+                umma_bf16(tmem + kC, umma_desc(aS + kSPart + 256 * ks, kSbo),
+                          umma_desc(bW + (kC / 8) * kSbo + 256 * ks, kSbo), kIdesc192, 1u);
+            for (int ks = 0; ks < kD / 16; ++ks)
+                umma_bf16(tmem + 2 * kC, umma_desc(aS + 2 * kSPart + 256 * ks, kSbo),
+                          umma_desc(bW + (2 * kC / 8) * kSbo + 256 * ks, kSbo), kIdesc64, 1u);
+            umma_commit(&sm.mma_g);
         }
-        ++issued_mma;
-        // The decision to read TMEM is block-uniform (tcgen05.ld is warp-collective).
-        if (__syncthreads_or(wait_parity(&sm.mma, (uint32_t)waits_mma & 1u) ? 0 : 1)) {
-            ok = false;
-            break;
-        }
-        ++waits_mma;
-        tc_fence_after();
-        if (c + 1 < nch) {  // the [W; Q] buffer is free again
-            if (tid == 0) issue_a1(c + 1);
-            ++issued_a1;
-        }
-        // Rows 64..127: W_mid M (handed over through S) and Q M (scaled by g, to the record).
-        // Rows 0..63: E = U - (W_hi M + W_lo M + W_mid M), in place over U and to the record.
-        {
-            float va[16], vb[16];
-            read3((uint32_t)(half * 16), va);
-            read3(kTmemD1b + (uint32_t)(half * 16), vb);
-            if (row >= kC) {
-                const int t = row - kC;
-                const float g = expf(lg[t]);
-#pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    *reinterpret_cast<float4*>(&sm.S[t][half * 16 + j]) = make_float4(va[j], va[j + 1], va[j + 2], va[j + 3]);
-                    *reinterpret_cast<float4*>(&sm.QM[t][half * 16 + j]) =
-                        make_float4(vb[j] * g, vb[j + 1] * g, vb[j + 2] * g, vb[j + 3] * g);
-                }
-            }
-            tc_fence_before();
-            __syncthreads();
-            if (row < kC) {
-                float* ur = U + row * kUS + half * 16;
-#pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float4 u = *reinterpret_cast<const float4*>(ur + j);
-                    const float4 m = *reinterpret_cast<const float4*>(&sm.S[row][half * 16 + j]);
-                    *reinterpret_cast<float4*>(ur + j) =
-                        make_float4(u.x - ((vb[j] + m.x) + va[j]), u.y - ((vb[j + 1] + m.y) + va[j + 1]),
-                                    u.z - ((vb[j + 2] + m.z) + va[j + 2]), u.w - ((vb[j + 3] + m.w) + va[j + 3]));
-                }
-            }
-        }
-        __syncthreads();
+        ++issued_g;
+        // The previous chunk's outputs, while those products run.
+        if (c > 0) store_outputs();
 
-        // B of D2: E' = diag(g_C / g) E, and B of DO: E, both transposed (32 rows x 64
-        // tokens) in three bf16 parts.
-        {
-            const int jj = tid % kDVC, g = tid / kDVC;  // 32 x 8 granules, one per thread
-            const float lgC = lg[kC - 1];
-            float x[8], y[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                x[j] = U[(8 * g + j) * kUS + jj];
-                y[j] = x[j] * expf(lgC - lg[8 * g + j]);
-            }
-            uint4 p0, p1, p2;
-            const uint32_t off = core_off(jj, 8 * g, kC);
-            split3x8(y, p0, p1, p2);
-            *reinterpret_cast<uint4*>(sm.bop + off) = p0;
-            *reinterpret_cast<uint4*>(sm.bop + kBopPartE + off) = p1;
-            *reinterpret_cast<uint4*>(sm.bop + 2 * kBopPartE + off) = p2;
-            split3x8(x, p0, p1, p2);
-            *reinterpret_cast<uint4*>(sm.bopE + off) = p0;
-            *reinterpret_cast<uint4*>(sm.bopE + kBopPartE + off) = p1;
-            *reinterpret_cast<uint4*>(sm.bopE + 2 * kBopPartE + off) = p2;
-        }
-        got = wait_parity(&sm.bar_a2, (uint32_t)c & 1u);
-        async_proxy_fence();
-        tc_fence_before();
+        got = wait_parity(&sm.mma_g, (uint32_t)waits_g & 1u);
+        got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++done_a2;
+        ++waits_g, ++done_c;
         tc_fence_after();
-        if (tid == 0) {
-            const uint64_t db = umma_desc(smem_u32(sm.bop), (kC / 8) * 128);
-            const uint64_t de = umma_desc(smem_u32(sm.bopE), (kC / 8) * 128);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                umma_bf16(tmem + kTmemD2, da2 + 16 * ks, db + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                umma_bf16(tmem, dpa + 16 * ks, de + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
-            for (int ks = 0; ks < kC / 16; ++ks)
-                umma_bf16(tmem + kTmemD1b, dpb + 16 * ks, de + 16 * ks, kIdesc, ks != 0 ? 1u : 0u);
-            umma_commit(&sm.mma);
+        if (c + 1 < nch) {  // the BW buffer is free again
+            if (tid == 0) issue_a(c + 1);
+            ++issued_a;
         }
-        ++issued_mma;
-
-        if (__syncthreads_or(wait_parity(&sm.mma, (uint32_t)waits_mma & 1u) ? 0 : 1)) {
+        // --- E = U - W M and g Q M for this thread's 32 tokens
+        const float* gq = reinterpret_cast<const float*>(sm.imgC);
+        const float* gk = gq + kC;
+        const float gC = gq[2 * kC];
+        const float4* ut = reinterpret_cast<const float4*>(sm.imgC + kR2GBytes) + j * (kC / 4);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const uint32_t col = (uint32_t)(32 * half + 16 * p);
+            uint32_t r0[16], r1[16], r2[16], r3[16];
+            tmem_ld16_issue(tmem + lane_base + col, r0);
+            tmem_ld16_issue(tmem + lane_base + kC + col, r1);
+            tmem_ld16_issue(tmem + lane_base + 2 * kC + col, r2);
+            tmem_ld16_issue(tmem + lane_base + 3 * kC + col, r3);
+            tmem_wait_ld();
+            tie_regs(r0), tie_regs(r1), tie_regs(r2), tie_regs(r3);
+            float e[16], ep[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int gi = (int)(col / 4) + q4;
+                const float4 uu = ut[gi ^ (j & 7)];
+                const float uv[4] = {uu.x, uu.y, uu.z, uu.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int mm = 4 * q4 + m, t = (int)col + mm;
+                    const float wm = (__uint_as_float(r0[mm]) + __uint_as_float(r1[mm])) + __uint_as_float(r2[mm]);
+                    e[mm] = uv[m] - wm;
+                    ep[mm] = e[mm] * gk[t];
+                    qm[16 * p + mm] = __uint_as_float(r3[mm]) * gq[t];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                float x8[8], y8[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) x8[m] = ep[8 * u + m], y8[m] = e[8 * u + m];
+                uint4 p0, p1, p2;
+                const uint32_t off = core_off(j, (int)col + 8 * u, kC);
+                split3x8(x8, p0, p1, p2);
+                *reinterpret_cast<uint4*>(sm.aop + off) = p0;
+                *reinterpret_cast<uint4*>(sm.aop + kEPart + off) = p1;
+                *reinterpret_cast<uint4*>(sm.aop + 2 * kEPart + off) = p2;
+                split3x8(y8, p0, p1, p2);
+                *reinterpret_cast<uint4*>(sm.aop + 3 * kEPart + off) = p0;
+                *reinterpret_cast<uint4*>(sm.aop + 4 * kEPart + off) = p1;
+            }
+        }
+        out_t0 = c * kC;
+        out_n = min(kC, a.L - out_t0);
+        async_proxy_fence();
+        tc_fence_before();
+        got = wait_parity(&sm.bar_b, (uint32_t)c & 1u);
+        if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++waits_mma;
+        ++done_b;
         tc_fence_after();
-        if (c + 1 < nch) {  // the K^T and P buffer is free again
-            if (tid == 0) issue_a2(c + 1);
-            ++issued_a2;
+        if (c + 1 < nch) {  // U^T and the gate factors are in registers or consumed
+            if (tid == 0) issue_c(c + 1);
+            ++issued_c;
         }
-        // O: rows 64..127 of DOa (P_mid E) plus QM go through S to the warps holding rows
-        // 0..63 of DOa (P_hi E) and DOb (P_lo E), which write the chunk's outputs.
-        {
-            float vo[16];
-            read3((uint32_t)(half * 16), vo);
-            if (row >= kC) {
-                const int t = row - kC;
+        // --- state update first (the chain waits for it), then the outputs' products
+        if (tid == 0) {
+            const uint32_t aE = smem_u32(sm.aop), bK = smem_u32(sm.imgB), bP = bK + kR2BKBytes;
+            constexpr uint32_t kSbo = (kC / 8) * 128;
+            for (int part = 0; part < 3; ++part)
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    umma_bf16(tmem + kTmemDU, umma_desc(aE + part * kEPart + 256 * ks, kSbo),
+                              umma_desc(bK + 256 * ks, kSbo), kIdesc128, (part | ks) != 0 ? 1u : 0u);
+            umma_commit(&sm.mma_u);
+            for (int ks = 0; ks < kC / 16; ++ks)
+                umma_bf16(tmem + kTmemDO, umma_desc(aE + 3 * kEPart + 256 * ks, kSbo), umma_desc(bP + 256 * ks, kSbo),
+                          kIdesc128, ks != 0 ? 1u : 0u);
+            for (int ks = 0; ks < kC / 16; ++ks)
+                umma_bf16(tmem + kTmemDO + kC, umma_desc(aE + 4 * kEPart + 256 * ks, kSbo),
+                          umma_desc(bP + (kC / 8) * kSbo + 256 * ks, kSbo), kIdesc64, 1u);
+            umma_commit(&sm.mma_o);
+        }
+        ++issued_u, ++issued_o;
+        if (__syncthreads_or(wait_parity(&sm.mma_u, (uint32_t)waits_u & 1u) ? 0 : 1)) {
+            ok = false;
+            break;
+        }
+        ++waits_u;
+        tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float4 q = *reinterpret_cast<const float4*>(&sm.QM[t][half * 16 + j]);
-                    *reinterpret_cast<float4*>(&sm.S[t][half * 16 + j]) =
-                        make_float4(q.x + vo[j], q.y + vo[j + 1], q.z + vo[j + 2], q.w + vo[j + 3]);
-                }
+        for (int u = 0; u < 4; u += 2) {
+            uint32_t r0[16], r1[16];
+            tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(64 * half + 16 * u), r0);
+            tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(64 * half + 16 * u + 16), r1);
+            tmem_wait_ld();
+            tie_regs(r0), tie_regs(r1);
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                s[16 * u + m] = fmaf(gC, s[16 * u + m], __uint_as_float(r0[m]));
+                s[16 * u + 16 + m] = fmaf(gC, s[16 * u + 16 + m], __uint_as_float(r1[m]));
             }
-            float vl[16];
-            read3(kTmemD1b + (uint32_t)(half * 16), vl);
-            tc_fence_before();
-            __syncthreads();
-            if (row < n) {
-                float* ob = a.out + (((size_t)b * a.L + t0 + row) * a.Hv + h) * kD + col0 + half * 16;
-#pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float4 sq = *reinterpret_cast<const float4*>(&sm.S[row][half * 16 + j]);
-                    *reinterpret_cast<float4*>(ob + j) =
-                        make_float4(sq.x + (vl[j] + vo[j]), sq.y + (vl[j + 1] + vo[j + 1]),
-                                    sq.z + (vl[j + 2] + vo[j + 2]), sq.w + (vl[j + 3] + vo[j + 3]));
-                }
-            }
         }
-        {
-            float v[16];
-            read3(kTmemD2 + (uint32_t)(half * 16), v);
-            const float gC = expf(lg[kC - 1]);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) m[j] = fmaf(gC, m[j], v[j]);
-        }
-        if (c + 1 < nch) split_m();  // the next chunk's B of D1 (the D2 MMAs, last readers of bop, are done)
-        // Small buffer s (E was written into it) is refilled next by the async proxy.
-        async_proxy_fence();
+        // The outputs' products still read the E parts: the next S parts overwrite them.
+        const bool got_o = wait_parity(&sm.mma_o, (uint32_t)waits_o & 1u);
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(got_o ? 0 : 1)) {
+            ok = false;
+            break;
+        }
+        ++waits_o;
         tc_fence_after();
-        if (c + 2 < nch) {
-            if (tid == 0) issue_small(c + 2);
-            ++issued_small;
+        if (c + 1 < nch) {  // K^T and the P tile are consumed
+            if (tid == 0) issue_b(c + 1);
+            ++issued_b;
+            split_s();
         }
     }
 
     if (ok) {
-        float4* MD = reinterpret_cast<float4*>(a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)row * kD +
-                                               col0 + half * 16);
+        store_outputs();  // the last chunk's
+        float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)(64 * half) * kD + j;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) MD[j] = make_float4(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]);
+        for (int i = 0; i < 64; ++i) MD[(size_t)i * kD] = s[i];
     } else if (tid == 0) {
         // Something never arrived: record it, then give every copy and MMA still
         // outstanding one more bounded wait before shared memory and TMEM go.
         record(a.err, GDN_ERR_TIMEOUT);
-        for (; done_small < issued_small; ++done_small)
-            wait_parity(&sm.full[done_small & 1], (uint32_t)(done_small >> 1) & 1u);
-        for (; done_a1 < issued_a1; ++done_a1) wait_parity(&sm.bar_a1, (uint32_t)done_a1 & 1u);
-        for (; done_a2 < issued_a2; ++done_a2) wait_parity(&sm.bar_a2, (uint32_t)done_a2 & 1u);
-        for (; waits_mma < issued_mma; ++waits_mma) wait_parity(&sm.mma, (uint32_t)waits_mma & 1u);
+        for (; done_a < issued_a; ++done_a) wait_parity(&sm.bar_a, (uint32_t)done_a & 1u);
+        for (; done_b < issued_b; ++done_b) wait_parity(&sm.bar_b, (uint32_t)done_b & 1u);
+        for (; done_c < issued_c; ++done_c) wait_parity(&sm.bar_c, (uint32_t)done_c & 1u);
+        for (; waits_g < issued_g; ++waits_g) wait_parity(&sm.mma_g, (uint32_t)waits_g & 1u);
+        for (; waits_u < issued_u; ++waits_u) wait_parity(&sm.mma_u, (uint32_t)waits_u & 1u);
+        for (; waits_o < issued_o; ++waits_o) wait_parity(&sm.mma_o, (uint32_t)waits_o & 1u);
     }
     tc_fence_before();
     __syncthreads();
@@ -1393,7 +1315,7 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     const ChunkArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, static_cast<unsigned char*>(workspace),
                       err_word, num_slots, B, L, Hk, Hv, Hv / Hk, nchunks};
     const bool bf = qkv_dtype == GDN_BF16;
-    const int s1 = bf ? (int)sizeof(SmemP) : (int)sizeof(Smem1), s2 = bf ? (int)sizeof(SmemTC) : (int)sizeof(Smem2);
+    const int s1 = bf ? (int)sizeof(SmemP) : (int)sizeof(Smem1), s2 = bf ? (int)sizeof(SmemS) : (int)sizeof(Smem2);
     cudaError_t e = bf ? cudaFuncSetAttribute(gdn_chunk_prepare_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1)
                        : cudaFuncSetAttribute(gdn_chunk_prepare_kernel<float>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
@@ -1406,11 +1328,24 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     e = bf ? cudaFuncSetAttribute(gdn_chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s2)
            : cudaFuncSetAttribute(gdn_chunk_scan_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    const unsigned g1 = (unsigned)(B * Hv * nchunks), g2 = (unsigned)(B * Hv * kNCB);
+    const unsigned g1 = (unsigned)(B * Hv * nchunks);
     if (bf) {
         gdn_chunk_prepare_tc_kernel<<<g1, kNT, s1, stream>>>(a);
-        gdn_chunk_scan_tc_kernel<<<g2, kNT, s2, stream>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+        // The scan starts behind the prepare kernel with programmatic dependent launch.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(B * Hv));
+        cfg.blockDim = dim3(kNT);
+        cfg.dynamicSmemBytes = (size_t)s2;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, gdn_chunk_scan_tc_kernel, a) != cudaSuccess) return GDN_ERR_CUDA;
     } else {
+        const unsigned g2 = (unsigned)(B * Hv * kNCB);
         gdn_chunk_prepare_kernel<float><<<g1, kNT, s1, stream>>>(a);
         gdn_chunk_scan_kernel<float><<<g2, kNT, s2, stream>>>(a);
     }

@@ -67,3 +67,18 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
 
     bench.run_reference(A())
     assert not called and capsys.readouterr().out == ""
+
+
+def test_clock_sampler_summarises_the_timed_window():
+    """Samples outside the timed window are ignored; reasons are the union of those inside."""
+    s = bench.ClockSampler()
+    rows = [(0.5, 1200.0, set()), (1.0, 1965.0, set()), (1.1, 1950.0, {"sw_power_cap"}), (1.2, 1965.0, set()),
+            (3.0, 900.0, {"hw_slowdown"})]
+    s.rows = [dict(ts=t, sm=sm, sm_max=1965.0, reasons=r) for t, sm, r in rows]
+    s.mark(0.9, 1.3)
+    c = s.stop()
+    assert c["samples"] == 3 and c["window"] == "timed"
+    assert c["sm_mhz"] == 1965.0 and c["sm_mhz_min"] == 1950.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+    empty = bench.ClockSampler()
+    assert empty.stop() is None

@@ -656,6 +656,36 @@ def test_prefill_chunked_matches_oracle(torch_cuda, shape):
     assert rel_err(out.cpu().numpy(), ref_out) <= TOL_OUT_BF16
 
 
+@pytest.mark.parametrize("L", [200, 700])
+def test_prefill_chunked_slow_decay(torch_cuda, L):
+    """Gates close to one (alpha ~ 0.97, the slow forgetting of trained models): the chunk-start
+    state then reaches every token of a chunk, so the products with the carried state (W M,
+    and the state update) carry the result and their precision is what is tested."""
+    torch = torch_cuda
+    import oracle
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(47 + L)
+    B, Hk, Hv = 2, 1, 2
+    pool = wl.init_pool(rng, 2 * B, Hv, 128, 128)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, 128, 128, wl.BF16)
+    a = np.exp(np.log(a) * np.float32(0.03)).astype(np.float32)
+    src = np.arange(B, dtype=np.int32)
+    dst = np.arange(B, 2 * B, dtype=np.int32)
+    xd = step_to_device(wl.Step(q, k, v, a, b, src, dst.reshape(B, 1)))
+    dev = to_torch(pool)
+    out = torch.full((B, L, Hv, 128), -7.0, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(gdn.gdn_prefill_workspace_bytes(B, L, Hv, 128, 128), dtype=torch.uint8, device="cuda")
+    gdn.gdn_prefill_chunked(dev, xd["src"], to_torch(dst), xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], out,
+                            ws, err_word=err)
+    assert gdn.gdn_get_error(err) == gdn.GDN_OK
+    ref_pool, ref_out = pool.copy(), np.zeros((B, L, Hv, 128), np.float32)
+    assert oracle.prefill(ref_pool, src, dst, q, k, v, a, b, ref_out, nthreads=8) == 0
+    check_pool(dev.cpu().numpy(), ref_pool, pool, dst)
+    assert rel_err(out.cpu().numpy(), ref_out) <= TOL_OUT_BF16
+
+
 def test_prefill_chunked_edge_cases(torch_cuda):
     """Padding rows, an out-of-range slot, a full reset (alpha = 0) and a short workspace."""
     torch = torch_cuda
