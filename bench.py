@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "2749ceb8bdba484ccb2c638bc20fa1bd165c2b17abd6d9fd3899c0caa34bbfaa",
-               "bytes_per_launch": 541164544 + 483485952}
+               "source_sha256": "ce609655212abeb427598841f4281647374eb6246e559fbc6b4601b7fcd12fea",
+               "bytes_per_launch": 541170432 + 483238144}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
@@ -524,14 +524,21 @@ def _time_calls(call, n: int, stream, graph: bool) -> float:
     return 1e3 * ev0.elapsed_time(ev1) / n
 
 
-def _time_cold(call, reps: int, stream) -> float:
-    """Median microseconds of one call right after a write of 256 MiB (twice the L2)."""
+def _time_cold(call, reps: int, stream, clean: bool = False) -> float:
+    """Median microseconds of one call right after a write of 256 MiB (twice the L2).
+
+    The write leaves the L2 full of dirty lines that the timed call then writes back.
+    With ``clean`` the 256 MiB are read instead: the call still finds none of its data
+    in L2, but pays for no one else's write-back."""
     import torch
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(256 << 18, dtype=torch.float32, device="cuda")
     cold = []
     for _ in range(reps):
-        flush.fill_(1)
+        if clean:
+            flush.sum()
+        else:
+            flush.fill_(1)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call()
@@ -594,6 +601,7 @@ def measure_workload(name: str, calls: int = 200, warmup: int = 10, variant: str
     warm_us = _time_calls(call, calls, stream, graph=False)
     graph_us = _time_calls(call, calls, stream, graph=True) if graph_too else None
     cold_us = _time_cold(call, min(calls, cold_reps), stream)
+    cold_clean_us = _time_cold(call, min(calls, cold_reps), stream, clean=True)
     code = gdn.gdn_get_error(err)
     if code != 0:
         raise RuntimeError(f"device error word set: {gdn.status_string(code)}")
@@ -621,6 +629,7 @@ def measure_workload(name: str, calls: int = 200, warmup: int = 10, variant: str
                    "qkv": s.dtype, "state": "f32"},
         "units_per_call": nb["units"], "calls": calls,
         "us_per_call_warm": warm_us, "us_per_call_graph": graph_us, "us_per_call_cold": cold_us,
+        "us_per_call_cold_clean_l2": cold_clean_us,
         "value_warm": nb["units"] / (best_warm / 1e6), "value_cold": nb["units"] / (cold_us / 1e6), "unit": UNIT,
         "bytes_per_call_nominal": nb["nominal"], "bytes_per_call_min": nb["minimum"],
         "gbs_cold_nominal": nb["nominal"] / cold_us / 1e3, "gbs_cold_min": nb["minimum"] / cold_us / 1e3,
@@ -628,7 +637,9 @@ def measure_workload(name: str, calls: int = 200, warmup: int = 10, variant: str
         "frac_cold_nominal": nb["nominal"] / cold_us / 1e3 / hbm_peak,
         "frac_cold_min": nb["minimum"] / cold_us / 1e3 / hbm_peak,
         "peak_gbs": hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
-        "l2": "warm: the call's inputs may sit in L2; cold: after a 256 MiB write",
+        "gbs_cold_clean_nominal": nb["nominal"] / cold_clean_us / 1e3,
+        "l2": "warm: the call's inputs may sit in L2; cold: after a 256 MiB write (the call also writes back "
+              "the dirty lines it evicts); cold_clean_l2: after a 256 MiB read",
         "commit": commit,
     }
     if cpu:

@@ -69,8 +69,9 @@ constexpr size_t kRecF32Bytes = kRecG + (size_t)kC * 4;
 //   image B  BK  K^T: dk rows x 64 tokens, same layout
 //            BP  [P_mid | P_hi]: 128 rows (t, per part) x 64 (i), bf16 parts of P
 //   image C  G   g_t [64], g_C / g_t [64], g_C, 3 zero words
-//            UT  U^T [dv][64] fp32: row j holds U[t][j] for the 64 tokens as 16 float4
-//                granules, granule q stored at position q ^ (j & 7) (bank spread)
+//            UT  U^T fp32 as 16 x 128 float4 granules: granule q of value row j (tokens
+//                4q..4q+3 of U[t][j]) at index q * dv + j, so that 32 consecutive rows
+//                are 512 contiguous bytes for the writer and the reader alike
 constexpr size_t kR2BW = 0;
 constexpr uint32_t kR2BWBytes = 4 * kC * kD * 2;
 constexpr size_t kR2BK = kR2BW + kR2BWBytes;
@@ -248,23 +249,38 @@ __device__ __forceinline__ void tie_regs(uint32_t (&r)[16]) {
                    "+r"(r[15]));
 }
 
-// Eight fp32 values as three 16-byte granules of bf16 parts: x = hi + mid + lo.
-__device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& mid, uint4& lo) {
+// Eight fp32 values as three 16-byte granules of bf16 parts, x = hi + mid + lo up to
+// |x - (hi + mid + lo)| < 2^-23 |x|: hi and mid are the fp32 bit patterns truncated to
+// their upper 16 bits (a byte permute, no rounding, no conversion), lo is rounded.  Each
+// residual is exact in fp32.
+__device__ __forceinline__ void split3x8_fast(const float (&x)[8], uint4& hi, uint4& mid, uint4& lo) {
     uint32_t h[4], m[4], l[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        float a0 = x[2 * j], a1 = x[2 * j + 1];
-        h[j] = pack_bf16x2(a0, a1);
-        a0 -= __uint_as_float(h[j] << 16);
-        a1 -= __uint_as_float(h[j] & 0xffff0000u);
-        m[j] = pack_bf16x2(a0, a1);
-        a0 -= __uint_as_float(m[j] << 16);
-        a1 -= __uint_as_float(m[j] & 0xffff0000u);
-        l[j] = pack_bf16x2(a0, a1);
+        const uint32_t u0 = __float_as_uint(x[2 * j]), u1 = __float_as_uint(x[2 * j + 1]);
+        h[j] = __byte_perm(u0, u1, 0x7632);
+        const float r0 = x[2 * j] - __uint_as_float(u0 & 0xffff0000u);
+        const float r1 = x[2 * j + 1] - __uint_as_float(u1 & 0xffff0000u);
+        const uint32_t v0 = __float_as_uint(r0), v1 = __float_as_uint(r1);
+        m[j] = __byte_perm(v0, v1, 0x7632);
+        l[j] = pack_bf16x2(r0 - __uint_as_float(v0 & 0xffff0000u), r1 - __uint_as_float(v1 & 0xffff0000u));
     }
     hi = make_uint4(h[0], h[1], h[2], h[3]);
     mid = make_uint4(m[0], m[1], m[2], m[3]);
     lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Two parts, hi truncated and mid rounded: |x - (hi + mid)| <= 2^-16 |x|.
+__device__ __forceinline__ void split2x8_fast(const float (&x)[8], uint4& hi, uint4& mid) {
+    uint32_t h[4], m[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t u0 = __float_as_uint(x[2 * j]), u1 = __float_as_uint(x[2 * j + 1]);
+        h[j] = __byte_perm(u0, u1, 0x7632);
+        m[j] = pack_bf16x2(x[2 * j] - __uint_as_float(u0 & 0xffff0000u), x[2 * j + 1] - __uint_as_float(u1 & 0xffff0000u));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    mid = make_uint4(m[0], m[1], m[2], m[3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -272,19 +288,29 @@ __device__ __forceinline__ void split3x8(const float (&x)[8], uint4& hi, uint4& 
 // ---------------------------------------------------------------------------
 
 // Warp 0: log g_t = sum_{i<=t} log alpha_i by a warp scan over two 32-token
-// halves, beta_t, and log g into the record (when Gs is not null).
+// halves, beta_t, and log g into the record (when Gs is not null).  With log2 the
+// logarithms are base 2 (ratios then come from exp2f).
 __device__ __forceinline__ void gate_scan(const ChunkArgs& a, int b, int h, int t0, int n, int lane, float* lg,
-                                          float* bt, float* Gs) {
+                                          float* bt, float* Gs, bool log2 = false) {
+    float al2[2] = {1.f, 1.f}, be2[2] = {0.f, 0.f};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {  // all loads first
+        const int t = half * 32 + lane;
+        if (t < n) {
+            const size_t gi = (((size_t)b * a.L + t0 + t) * a.Hv + h);
+            al2[half] = __ldg(a.alpha + gi);
+            be2[half] = __ldg(a.beta + gi);
+        }
+    }
     float carry = 0.f;
     for (int half = 0; half < 2; ++half) {
         const int t = half * 32 + lane;
-        const size_t gi = (((size_t)b * a.L + t0 + t) * a.Hv + h);
         float la = 0.f, be = 0.f;
         if (t < n) {
             // alpha = 0 (a full reset) would make log g = -inf and the ratios
             // -inf - -inf; e^-80 ~ 2e-35 is zero at fp32 precision instead.
-            la = fmaxf(logf(__ldg(a.alpha + gi)), -80.f);
-            be = __ldg(a.beta + gi);
+            la = log2 ? fmaxf(log2f(al2[half]), -80.f * 1.44269504f) : fmaxf(logf(al2[half]), -80.f);
+            be = be2[half];
         }
         float x = la;
 #pragma unroll
@@ -477,56 +503,131 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_prepare_kernel(ChunkArgs a) 
     }
 }
 
+// T = (I + A)^-1 for the strictly lower 64 x 64 A, in 16 x 16 blocks (all threads;
+// A complete on entry, T complete and zero above its diagonal on return, P scratch of
+// 3 x 16 x 16 floats).  Diagonal blocks by forward substitution (warp I, lane j < 16
+// owns column j of block I); then the blocks below the diagonal, one diagonal distance
+// d at a time: P = sum_{K=J}^{I-1} A_IK T_KJ and T_IJ = -T_II P for J = I - d.  Every
+// step is a set of independent dot products over all 256 threads, unrolled so that the
+// shared-memory loads of a step are in flight together.
+template <int D>
+__device__ __forceinline__ void merge_step(const float (*A)[kC + 4], float (*T)[kC + 4], float* P, int r, int cc) {
+#pragma unroll
+    for (int I = D; I < 4; ++I) {  // P = A_I,[J, I) T_[J, I),J with J = I - D
+        const int J = I - D;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 16 * D; k += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(&A[16 * I + r][16 * J + k]);
+            acc[0] = fmaf(a4.x, T[16 * J + k][16 * J + cc], acc[0]);
+            acc[1] = fmaf(a4.y, T[16 * J + k + 1][16 * J + cc], acc[1]);
+            acc[2] = fmaf(a4.z, T[16 * J + k + 2][16 * J + cc], acc[2]);
+            acc[3] = fmaf(a4.w, T[16 * J + k + 3][16 * J + cc], acc[3]);
+        }
+        P[(I - D) * 256 + r * 16 + cc] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int I = D; I < 4; ++I) {  // T_IJ = -T_II P
+        const int J = I - D;
+        const float* p = P + (I - D) * 256;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 16; m += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(&T[16 * I + r][16 * I + m]);
+            acc[0] = fmaf(t4.x, p[m * 16 + cc], acc[0]);
+            acc[1] = fmaf(t4.y, p[(m + 1) * 16 + cc], acc[1]);
+            acc[2] = fmaf(t4.z, p[(m + 2) * 16 + cc], acc[2]);
+            acc[3] = fmaf(t4.w, p[(m + 3) * 16 + cc], acc[3]);
+        }
+        T[16 * I + r][16 * J + cc] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void invert_blocked(const float (*A)[kC + 4], float (*T)[kC + 4], float* P, int tid) {
+    const int w = tid / 32, lane = tid % 32;
+    if (w < 4) {
+        if (lane < 16) {
+            const int o = 16 * w, j = lane;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc0 = r == j ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < (r & ~3); m += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(&A[o + r][o + m]);
+                    acc0 = fmaf(-a4.x, x[m], acc0);
+                    acc1 = fmaf(-a4.y, x[m + 1], acc1);
+                    acc0 = fmaf(-a4.z, x[m + 2], acc0);
+                    acc1 = fmaf(-a4.w, x[m + 3], acc1);
+                }
+#pragma unroll
+                for (int m = r & ~3; m < r; ++m) acc0 = fmaf(-A[o + r][o + m], x[m], acc0);
+                x[r] = acc0 + acc1;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) T[o + r][o + j] = x[r];
+        }
+    } else {
+        // zero the six blocks above the diagonal
+#pragma unroll
+        for (int e = tid - 128; e < 6 * 256; e += 128) {
+            const int blk = e / 256, r = (e / 16) % 16, cc = e % 16;
+            const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            T[16 * I + r][16 * J + cc] = 0.f;
+        }
+    }
+    __syncthreads();
+    const int r = tid / 16, cc = tid % 16;
+    merge_step<1>(A, T, P, r, cc);
+    merge_step<2>(A, T, P, r, cc);
+    merge_step<3>(A, T, P, r, cc);
+}
+
 // ---------------------------------------------------------------------------
 // Kernel 1, tensor-core form (bf16 inputs), one CTA per (request, head, chunk):
-//   D0 = [K; Q] K^T on the tensor cores (M = 128, N = 64, K = dk; exact bf16 products),
-//   read out as A[t][i] = beta_t (g_t / g_i) k_t.k_i (i < t) and P[t][i] =
-//   (g_t / g_i) q_t.k_i (i <= t); then the chunk's unit lower-triangular system
-//   (I + A) [U | W] = [diag(beta) V | diag(beta g) K] solved by forward substitution
-//   in fp32 on the CUDA cores: thread c owns right-hand-side column c (128 columns of
-//   V, 128 of K) and keeps its 64 unknowns in registers, so U and W come out exact to
-//   fp32 rounding with no explicit inverse.  The record receives the scan's operand
-//   images: [W_lo | W_mid | W_hi | Q], K^T and [P_mid | P_hi] as bf16 tensor-core
-//   tiles, the gate factors g_t, g_C / g_t, g_C, and U^T in fp32.
+//   D0  = [K; Q] K^T on the tensor cores (M = 128, N = 64, K = dk; exact bf16 products),
+//         read out as A[t][i] = beta_t (g_t / g_i) k_t.k_i (i < t) and
+//         P[t][i] = (g_t / g_i) q_t.k_i (i <= t);
+//   T   = (I + A)^-1 in fp32 on the CUDA cores, in 16 x 16 blocks (invert_blocked);
+//   D_U = V^T (T diag(beta))^T = U^T  and  D_W = K^T (T diag(beta g))^T = W^T on the tensor
+//         cores, V and K exact in bf16 and each T factor in three bf16 parts (24 bits).
+// The record receives the scan's operand images: [W_lo | W_mid | W_hi | Q], K^T and
+// [P_mid | P_hi] as bf16 tensor-core tiles, the gate factors g_t, g_C / g_t, g_C, and
+// U^T in fp32.
 // ---------------------------------------------------------------------------
 struct SmemP {
     union {
-        unsigned char KQ[2 * kC * kD * 2];  // [K; Q]: A operand of D0 (rows 0..63 are also its B)
-        __nv_bfloat16 V[kC][kD + 2];        // V rows (right-hand sides), once D0 is complete
-        float W[kC][kD + 4];                // W staged for its split, after the solve
+        unsigned char KQ[2 * kC * kD * 2];   // [K; Q]: A operand of D0 (rows 0..63 are also its B)
+        float P[3 * 16 * 16];                // scratch of the blocked inverse (once D0 is complete)
+        struct {
+            unsigned char after_kq[2 * kC * kD * 2];
+            float A[kC][kC + 4];             // the system's strictly lower part (float4 rows)
+        } ra;
+        unsigned char Bp[2][3][kC * kC * 2]; // B of D_U and D_W: (T diag(beta)), (T diag(beta g)), 3 parts
+                                             // each (over [K; Q] and A, both dead by then)
+        float W[kC][kD + 4];                 // W staged for its split (row stride spreads banks)
     } u;
-    __nv_bfloat16 K[kC][kD + 2];            // K rows: right-hand sides and the K^T gather
-    float A[kC][kC + 4];                    // the system's strictly lower part (float4 rows)
+    float T[kC][kC + 4];                     // (I + A)^-1
+    unsigned char VT[kD * kC * 2];           // V^T: A operand of D_U (dv rows x 64 tokens)
+    unsigned char KT[kD * kC * 2];           // K^T: A operand of D_W, and the record's K^T tile
     float lg[kC];
     float bt[kC];
-    float gq[kC];                           // g_t
+    float bg[kC];                            // beta_t g_t
     uint64_t mma;
     uint32_t tmem;
 };
-static_assert(sizeof(SmemP) <= 76 * 1024, "three prepare CTAs per SM");
+static_assert(sizeof(SmemP) <= 113 * 1024, "two prepare CTAs per SM");
 
-// bf16 row block R (rows = tokens) gathered into a K-major operand image in global
-// memory with kD rows (dk) and kC columns (tokens).  Consecutive threads write
-// consecutive 16-byte granules.
-__device__ __forceinline__ void gather_transposed_global(const __nv_bfloat16 (*R)[kD + 2], unsigned char* img,
-                                                         int tid) {
-    for (int e = tid; e < kD * (kC / 8); e += kNT) {
-        const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // row j, tokens 8g..8g+7
-        uint16_t x[8];
+// The 8 bf16 of a 16-byte granule (one token, 8 consecutive feature indices d0..d0+7)
+// into column t of a K-major operand tile whose rows are the feature index.
+__device__ __forceinline__ void scatter_granule(unsigned char* tile, const uint4& x, int d0, int t) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint16_t*>(&R[8 * g + m][j]);
-        uint4 w;
-        w.x = x[0] | ((uint32_t)x[1] << 16);
-        w.y = x[2] | ((uint32_t)x[3] << 16);
-        w.z = x[4] | ((uint32_t)x[5] << 16);
-        w.w = x[6] | ((uint32_t)x[7] << 16);
-        *reinterpret_cast<uint4*>(img + core_off(j, 8 * g, kC)) = w;
-    }
-}
-
-__device__ __forceinline__ void store_row8(__nv_bfloat16* row, const uint4& x) {
-    uint32_t* r = reinterpret_cast<uint32_t*>(row);
-    r[0] = x.x, r[1] = x.y, r[2] = x.z, r[3] = x.w;
+    for (int m = 0; m < 8; ++m)
+        *reinterpret_cast<uint16_t*>(tile + core_off(d0 + m, t, kC)) = (uint16_t)(w[m >> 1] >> (16 * (m & 1)));
 }
 
 __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
@@ -546,8 +647,9 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     const int n = min(kC, a.L - t0);  // valid tokens; the rest are inert (k = q = v = 0, beta = 0, alpha = 1)
     unsigned char* rec = record_of(a, bh, c);
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const int half = warp / 4;  // TMEM columns 32*half .. +31 of D0
+    const int half = warp / 4;  // TMEM columns 32*half .. +31 of each 64-column accumulator
     constexpr uint32_t kIdesc = umma_idesc(128, kC);
+    constexpr uint32_t kSbo64 = (kC / 8) * 128;
 
     // The scan may be scheduled as soon as every CTA here has started: its CTAs take
     // whole SMs, so they only land on SMs this grid has left, and wait for it to finish.
@@ -558,34 +660,41 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
-                     "r"(64)
+                     "r"(128)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-        gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, nullptr);
     }
-    // k, q, v in 16-byte granules: [K; Q] into the D0 operand image, K also into the row
-    // buffer, Q into the record's BW tile (rows 192..255); V stays in registers until D0
-    // is done.  Consecutive threads take consecutive granules of the image: token
-    // t = (e & 7) + 8 (e >> 7), group g = (e >> 3) & 15, e = tid + 256 u.
+    // k, q, v in 16-byte granules: [K; Q] into the D0 operand image, Q also into the
+    // record's BW tile (rows 192..255), K and V scattered into the K^T and V^T operand
+    // tiles.  Every load is issued before the first store: the record's global stores
+    // could alias the inputs as far as the compiler knows, so interleaving them would
+    // serialise the loads.  Consecutive threads take consecutive granules of the image:
+    // token t = (e & 7) + 8 (e >> 7), group g = (e >> 3) & 15, e = tid + 256 u.
     constexpr int kGr = kC * (kD / 8) / kNT;  // granules per thread
-    uint4 vkeep[kGr];
+    uint4 kq[kGr], qq[kGr], vv[kGr];
 #pragma unroll
     for (int u = 0; u < kGr; ++u) {
         const int e = tid + kNT * u;
         const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-        uint4 kq = make_uint4(0, 0, 0, 0), qq = kq, vv = kq;
+        kq[u] = qq[u] = vv[u] = make_uint4(0, 0, 0, 0);
         if (t < n) {
             const size_t row = (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD + 8 * g;
             const size_t vrow = (((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + 8 * g;
-            kq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + row));
-            qq = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row));
-            vv = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + vrow));
+            kq[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + row));
+            qq[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row));
+            vv[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + vrow));
         }
-        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(t, 8 * g, kD)) = kq;
-        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(kC + t, 8 * g, kD)) = qq;
-        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(3 * kC + t, 8 * g, kD)) = qq;
-        store_row8(&sm.K[t][8 * g], kq);
-        vkeep[u] = vv;
+    }
+    if (warp == 0) gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, nullptr, true);
+#pragma unroll
+    for (int u = 0; u < kGr; ++u) {
+        const int e = tid + kNT * u;
+        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(t, 8 * g, kD)) = kq[u];
+        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(kC + t, 8 * g, kD)) = qq[u];
+        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(3 * kC + t, 8 * g, kD)) = qq[u];
+        scatter_granule(sm.KT, kq[u], 8 * g, t);
+        scatter_granule(sm.VT, vv[u], 8 * g, t);
     }
     async_proxy_fence();
     tc_fence_before();
@@ -599,7 +708,14 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                       kIdesc, ks != 0 ? 1u : 0u);
         umma_commit(&sm.mma);
     }
-    const bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
+    // The K^T tile goes to the record as it is (the scan's B operand of the state update).
+#pragma unroll
+    for (int u = 0; u < (int)(kR2BKBytes / 16) / kNT; ++u) {
+        const int e = tid + kNT * u;
+        *reinterpret_cast<uint4*>(rec + kR2BK + 16 * e) = *reinterpret_cast<const uint4*>(sm.KT + 16 * e);
+    }
+    bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
+    int waits = ok ? 1 : 0, issued = 1;
     if (ok) {
         tc_fence_after();
         // D0 row r < 64: k_r . k_i -> A (scaled); row 64 + t: q_t . k_i -> P (record).
@@ -617,9 +733,9 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         const int i = i0 + j + m;
-                        x[m] = i < r ? bt * expf(lt - sm.lg[i]) * v[j + m] : 0.f;
+                        x[m] = i < r ? bt * exp2f(lt - sm.lg[i]) * v[j + m] : 0.f;
                     }
-                    *reinterpret_cast<float4*>(&sm.A[r][i0 + j]) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(&sm.u.ra.A[r][i0 + j]) = make_float4(x[0], x[1], x[2], x[3]);
                 }
             } else {
                 // P row t, columns i0..i0+15: its mid and hi bf16 parts into [P_mid | P_hi].
@@ -631,84 +747,96 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int i = i0 + g8 + j;
-                        x[j] = i <= t ? expf(lt - sm.lg[i]) * v[g8 + j] : 0.f;
+                        x[j] = i <= t ? exp2f(lt - sm.lg[i]) * v[g8 + j] : 0.f;
                     }
-                    uint4 p0, p1, p2;
-                    split3x8(x, p0, p1, p2);
+                    uint4 p0, p1;
+                    split2x8_fast(x, p0, p1);
                     unsigned char* bp = rec + kR2BP;
                     *reinterpret_cast<uint4*>(bp + core_off(t, i0 + g8, kC)) = p1;
                     *reinterpret_cast<uint4*>(bp + core_off(kC + t, i0 + g8, kC)) = p0;
                 }
             }
         }
-    } else if (tid == 0) {
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        if (tid < kC) sm.bg[tid] = sm.bt[tid] * exp2f(sm.lg[tid]);  // beta_t g_t
+        invert_blocked(sm.u.ra.A, sm.T, sm.u.P, tid);  // ends with a barrier
+        // B operands of D_U and D_W: rows t, columns i, T[t][i] beta_i and T[t][i] beta_i g_i,
+        // each in three bf16 parts.
+        for (int e = tid; e < 2 * kC * (kC / 8); e += kNT) {
+            const int which = e / (kC * (kC / 8)), rem = e % (kC * (kC / 8));
+            const int t = (rem & 7) | ((rem >> 6) << 3), g = (rem >> 3) & 7;
+            const float* sc = which ? sm.bg : sm.bt;
+            const float4 t0v = *reinterpret_cast<const float4*>(&sm.T[t][8 * g]);
+            const float4 t1v = *reinterpret_cast<const float4*>(&sm.T[t][8 * g + 4]);
+            const float xs[8] = {t0v.x * sc[8 * g], t0v.y * sc[8 * g + 1], t0v.z * sc[8 * g + 2], t0v.w * sc[8 * g + 3],
+                                 t1v.x * sc[8 * g + 4], t1v.y * sc[8 * g + 5], t1v.z * sc[8 * g + 6],
+                                 t1v.w * sc[8 * g + 7]};
+            uint4 p0, p1, p2;
+            split3x8_fast(xs, p0, p1, p2);
+            const uint32_t off = core_off(t, 8 * g, kC);
+            *reinterpret_cast<uint4*>(sm.u.Bp[which][0] + off) = p0;
+            *reinterpret_cast<uint4*>(sm.u.Bp[which][1] + off) = p1;
+            *reinterpret_cast<uint4*>(sm.u.Bp[which][2] + off) = p2;
+        }
+        async_proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            const uint32_t vt = smem_u32(sm.VT), kt = smem_u32(sm.KT);
+            for (int p = 0; p < 3; ++p)
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    umma_bf16(tmem, umma_desc(vt + 256 * ks, kSbo64),
+                              umma_desc(smem_u32(sm.u.Bp[0][p]) + 256 * ks, kSbo64), kIdesc, (p | ks) != 0 ? 1u : 0u);
+            for (int p = 0; p < 3; ++p)
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    umma_bf16(tmem + kC, umma_desc(kt + 256 * ks, kSbo64),
+                              umma_desc(smem_u32(sm.u.Bp[1][p]) + 256 * ks, kSbo64), kIdesc, (p | ks) != 0 ? 1u : 0u);
+            umma_commit(&sm.mma);
+        }
+        ++issued;
+        ok = !__syncthreads_or(wait_parity(&sm.mma, 1) ? 0 : 1);
+        if (ok) {
+            ++waits;
+            tc_fence_after();
+            // D_U row j = U^T[j][t] for this warp's 32 tokens -> the record, granule q of row j
+            // at position q ^ (j & 7); D_W row d = W[.][d] -> W staged row-major.
+            const int j = (warp % 4) * 32 + lane;
+            float4* ut = reinterpret_cast<float4*>(rec + kR2UT) + j;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float uv[16], wv[16];
+                const int tb = 32 * half + 16 * part;
+                tmem_ld16(tmem + lane_base + (uint32_t)tb, uv);
+                tmem_ld16(tmem + lane_base + kC + (uint32_t)tb, wv);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    ut[((tb >> 2) + q4) * kD] = make_float4(uv[4 * q4], uv[4 * q4 + 1], uv[4 * q4 + 2], uv[4 * q4 + 3]);
+#pragma unroll
+                for (int m = 0; m < 16; ++m) sm.u.W[tb + m][j] = wv[m];
+            }
+        }
+    }
+    if (!ok && tid == 0) {
         record(a.err, GDN_ERR_TIMEOUT);
-        wait_parity(&sm.mma, 0);  // one more bounded wait before the accumulator is freed
+        for (; waits < issued; ++waits) wait_parity(&sm.mma, (uint32_t)waits & 1u);
+    }
+    float* G = reinterpret_cast<float*>(rec + kR2G);
+    if (tid < kC) {
+        G[tid] = exp2f(sm.lg[tid]);
+        G[kC + tid] = exp2f(sm.lg[kC - 1] - sm.lg[tid]);
+    } else if (tid < kC + 4) {
+        G[kC + tid] = tid == kC ? exp2f(sm.lg[kC - 1]) : 0.f;  // g_C, then zero padding
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
     if (!ok) return;
-
-    // V rows over the [K; Q] image (D0 is complete); g_t.
-#pragma unroll
-    for (int u = 0; u < kGr; ++u) {
-        const int e = tid + kNT * u;
-        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-        store_row8(&sm.u.V[t][8 * g], vkeep[u]);
-    }
-    if (tid < kC) sm.gq[tid] = expf(sm.lg[tid]);
-    __syncthreads();
-
-    // Forward substitution, one right-hand-side column per thread: x_r = rhs_r -
-    // sum_{m < r} A[r][m] x_m, rows in order, four partial sums per row.
-    const bool is_u = tid < kD;  // warp-uniform: warps 0..3 solve for U, 4..7 for W
-    const int col = is_u ? tid : tid - kD;
-    float x[kC];
-#pragma unroll
-    for (int r = 0; r < kC; ++r) {
-        const float rhs = is_u ? sm.bt[r] * __bfloat162float(sm.u.V[r][col])
-                               : (sm.bt[r] * sm.gq[r]) * __bfloat162float(sm.K[r][col]);
-        float acc0 = rhs, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-        for (int m = 0; m < (r & ~3); m += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(&sm.A[r][m]);
-            acc0 = fmaf(-a4.x, x[m], acc0);
-            acc1 = fmaf(-a4.y, x[m + 1], acc1);
-            acc2 = fmaf(-a4.z, x[m + 2], acc2);
-            acc3 = fmaf(-a4.w, x[m + 3], acc3);
-        }
-        if (r & 3) {
-            const float4 a4 = *reinterpret_cast<const float4*>(&sm.A[r][r & ~3]);
-            const int m = r & ~3;
-            acc0 = fmaf(-a4.x, x[m], acc0);
-            if ((r & 3) > 1) acc1 = fmaf(-a4.y, x[m + 1], acc1);
-            if ((r & 3) > 2) acc2 = fmaf(-a4.z, x[m + 2], acc2);
-        }
-        x[r] = (acc0 + acc1) + (acc2 + acc3);
-    }
-    __syncthreads();  // every thread is done with V (the union is rewritten next)
-
-    if (is_u) {
-        // U^T row col: 16 float4 granules, granule q at position q ^ (col & 7).
-        float4* ut = reinterpret_cast<float4*>(rec + kR2UT) + col * (kC / 4);
-#pragma unroll
-        for (int q = 0; q < kC / 4; ++q)
-            ut[q ^ (col & 7)] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-    } else {
-#pragma unroll
-        for (int r = 0; r < kC; ++r) sm.u.W[r][col] = x[r];
-    }
-    float* G = reinterpret_cast<float*>(rec + kR2G);
-    if (tid < kC) {
-        G[tid] = sm.gq[tid];
-        G[kC + tid] = expf(sm.lg[kC - 1] - sm.lg[tid]);
-    } else if (tid < kC + 4) {
-        G[kC + tid] = tid == kC ? sm.gq[kC - 1] : 0.f;  // g_C, then zero padding
-    }
-    __syncthreads();
 
     // W in three bf16 parts into the BW tile: W_lo rows 0..63, W_mid 64..127, W_hi 128..191.
     for (int e = tid; e < kC * (kD / 8); e += kNT) {
@@ -717,12 +845,11 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         const float4 w1 = *reinterpret_cast<const float4*>(&sm.u.W[t][8 * g + 4]);
         const float xw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint4 p0, p1, p2;
-        split3x8(xw, p0, p1, p2);
+        split3x8_fast(xw, p0, p1, p2);
         *reinterpret_cast<uint4*>(rec + kR2BW + core_off(t, 8 * g, kD)) = p2;
         *reinterpret_cast<uint4*>(rec + kR2BW + core_off(kC + t, 8 * g, kD)) = p1;
         *reinterpret_cast<uint4*>(rec + kR2BW + core_off(2 * kC + t, 8 * g, kD)) = p0;
     }
-    gather_transposed_global(sm.K, rec + kR2BK, tid);
 }
 
 // Reads (src, dst) of request b and classifies it: 0 run, 1 padding (skipped
@@ -929,10 +1056,14 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 
 // ---------------------------------------------------------------------------
 // Kernel 2, tensor-core form (bf16 inputs): one CTA per (request, head) walks the
-// chunks in order with the whole state in registers, transposed: thread (w, lane)
-// holds S[j][i] = M[i][j] for value row j = 32 (w % 4) + lane and key columns
-// i in [64 (w / 4), +64).  Row j is TMEM lane j of every accumulator, so the thread
-// that reads an accumulator row is the one that owns that row of the state.
+// chunks in order with the whole state in registers, transposed.  Sixteen compute
+// warps hold it: thread (w, lane), w < 16, owns S[j][i] = M[i][j] for value row
+// j = 32 (w % 4) + lane and key columns i in [32 (w / 4), +32), and handles the
+// chunk's tokens [16 (w / 4), +16).  Row j is TMEM lane j of every accumulator, so
+// the thread that reads an accumulator row is one that owns that row of the state.
+// Thread 0 also issues every MMA and bulk copy; the previous chunk's outputs are
+// stored while the next chunk's first products run (a separate issuing warp would
+// cost registers: a 17-warp CTA is allocated as 20 warps).
 // Per chunk, with S split into three bf16 parts (S = S_hi + S_mid + S_lo) as the A
 // operand (M = 128 value rows, K = dk) and the record's tile [W_lo | W_mid | W_hi | Q]
 // as B (N = 64 tokens per part):
@@ -943,18 +1074,18 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 // (K = 64 tokens):
 //   D_U = E'^T K              (B = K^T tile; cols 256..383)   ->  S <- g_C S + D_U
 //   D_O = E_hi [P_mid P_hi] + E_mid [P_hi]   (cols 384..511)  ->  o = g Q M + P E
-// The state update is committed first; the chain waits only for it, splits the new
-// state for the next chunk and issues that chunk's first products, and the outputs
-// are read out and stored while those run.  Thread 0 issues the MMAs and streams the
-// three record images with cp.async.bulk: each buffer is refilled for the next chunk
-// as soon as its last reader is done.  Every wait is bounded (2 s); a timeout is
-// recorded and the CTA drains and exits.
+// The state update is committed first; the chain waits only for it.  The issuing
+// thread streams the three record images with cp.async.bulk: each buffer is refilled
+// for the next chunk as soon as its last reader is done.  Every wait is bounded (2 s);
+// a timeout is recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kSPart = (uint32_t)kD * kD * 2;  // one bf16 part of S (128 x 128)
 constexpr uint32_t kEPart = (uint32_t)kD * kC * 2;  // one bf16 part of E^T or E'^T (128 x 64)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemDU = 256;
 constexpr uint32_t kTmemDO = 384;
+constexpr int kScanThreads = 512;                   // 16 warps, all of them compute
+constexpr int kIssuer = 0;                          // the thread that also issues MMAs and copies
 
 struct SmemS {
     unsigned char aop[3 * kSPart];  // A operands: S parts; then E'^T parts (3) and E^T parts (hi, mid)
@@ -968,15 +1099,27 @@ struct SmemS {
 static_assert(sizeof(SmemS) <= 227 * 1024, "scan shared memory plan exceeds the per-CTA limit");
 static_assert(3 * kEPart + 2 * kEPart <= 3 * kSPart, "E parts overlay the S parts");
 
-__global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) {
+// 8 consecutive TMEM columns of this warp's 32 lanes (completion awaited separately).
+__device__ __forceinline__ void tmem_ld8_issue(uint32_t addr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void tie_regs8(uint32_t (&r)[8]) {
+    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_tc[];
     SmemS& sm = *reinterpret_cast<SmemS*>(smem_tc);
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
+    constexpr bool compute = true;
+    const bool issuer = tid == kIssuer;
     const int bh = blockIdx.x;
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
-    const int half = warp / 4;                     // key columns 64*half.., tokens 32*half..
+    const int quarter = (warp / 4) & 3;            // key columns 32*quarter.., tokens 16*quarter..
     const int j = (warp % 4) * 32 + lane;          // value row = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const int nch = a.nchunks;
@@ -994,7 +1137,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         bulk_g2s(sm.imgC, record_of(a, bh, c) + kR2G, kImgC, &sm.bar_c);
     };
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(&sm.bar_a);
         mbar_init(&sm.bar_b);
         mbar_init(&sm.bar_c);
@@ -1012,7 +1155,7 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
     // Launched with programmatic dependent launch behind the prepare kernel: the set-up
     // above overlaps its tail; the records, indices and pool are read only after it.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid == 0) {
+    if (issuer) {
         scan_prologue(a, b, sm.src, sm.dst, sm.status);
         if (sm.status == 0) {
             issue_a(0);
@@ -1031,71 +1174,68 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
         return;
     }
 
-    float s[64];  // S[j][64 half + i]
-    {
-        const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) + (size_t)(64 * half) * kD + j;
+    float s[32];  // S[j][32 quarter + i]
+    if (compute) {
+        const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) + (size_t)(32 * quarter) * kD + j;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = M0[(size_t)i * kD];
+        for (int i = 0; i < 32; ++i) s[i] = M0[(size_t)i * kD];
     }
     // A operand of the first products: S in three bf16 parts, row j, 8 key columns per granule.
     auto split_s = [&]() {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 4; ++u) {
             float x8[8];
 #pragma unroll
             for (int m = 0; m < 8; ++m) x8[m] = s[8 * u + m];
             uint4 p0, p1, p2;
-            split3x8(x8, p0, p1, p2);
-            const uint32_t off = core_off(j, 64 * half + 8 * u, kD);
+            split3x8_fast(x8, p0, p1, p2);
+            const uint32_t off = core_off(j, 32 * quarter + 8 * u, kD);
             *reinterpret_cast<uint4*>(sm.aop + off) = p0;
             *reinterpret_cast<uint4*>(sm.aop + kSPart + off) = p1;
             *reinterpret_cast<uint4*>(sm.aop + 2 * kSPart + off) = p2;
         }
-        async_proxy_fence();
     };
-    split_s();
+    if (compute) split_s();
 
     constexpr uint32_t kIdesc256 = umma_idesc(128, 256), kIdesc192 = umma_idesc(128, 192);
     constexpr uint32_t kIdesc128 = umma_idesc(128, 128), kIdesc64 = umma_idesc(128, 64);
     bool ok = true;
+    // The issuer's bookkeeping of what it started and saw complete (for the drain).
     int done_a = 0, done_b = 0, done_c = 0, issued_a = 1, issued_b = 1, issued_c = 1;
     int waits_g = 0, waits_u = 0, waits_o = 0, issued_g = 0, issued_u = 0, issued_o = 0;
-    float qm[32];   // g_t (q_t M)_j for this thread's 32 tokens of the current chunk
+    float qm[16];   // g_t (q_t M)_j for this thread's 16 tokens of the current chunk
     int out_t0 = 0, out_n = 0;  // chunk whose outputs are pending
 
-    // Outputs of the chunk whose D_O was last committed: o = g q M + P E.
+    // Outputs of the chunk whose D_O was last completed: o = g q M + P E.
     auto store_outputs = [&]() {
+        const uint32_t col = (uint32_t)(16 * quarter);
+        uint32_t r0[16], r1[16];
+        tmem_ld16_issue(tmem + lane_base + kTmemDO + col, r0);
+        tmem_ld16_issue(tmem + lane_base + kTmemDO + kC + col, r1);
+        tmem_wait_ld();
+        tie_regs(r0), tie_regs(r1);
+        float* ob = a.out + (((size_t)b * a.L + out_t0) * a.Hv + h) * kD + j;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const uint32_t col = (uint32_t)(32 * half + 16 * p);
-            uint32_t r0[16], r1[16];
-            tmem_ld16_issue(tmem + lane_base + kTmemDO + col, r0);
-            tmem_ld16_issue(tmem + lane_base + kTmemDO + kC + col, r1);
-            tmem_wait_ld();
-            tie_regs(r0), tie_regs(r1);
-            float* ob = a.out + (((size_t)b * a.L + out_t0) * a.Hv + h) * kD + j;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const int t = (int)col + m;
-                if (t < out_n)
-                    ob[(size_t)t * a.Hv * kD] = qm[16 * p + m] + (__uint_as_float(r1[m]) + __uint_as_float(r0[m]));
-            }
+        for (int m = 0; m < 16; ++m) {
+            const int t = (int)col + m;
+            if (t < out_n) ob[(size_t)t * a.Hv * kD] = qm[m] + (__uint_as_float(r1[m]) + __uint_as_float(r0[m]));
         }
     };
 
     int c = 0;
     for (; c < nch; ++c) {
         // --- the chunk's first products: S parts x [W parts | Q]
-        bool got = wait_parity(&sm.bar_a, (uint32_t)c & 1u);
-        async_proxy_fence();
+        bool got = true;
+        if (compute) async_proxy_fence();  // the S parts just written, for the tensor cores
+        if (issuer) got = wait_parity(&sm.bar_a, (uint32_t)c & 1u);
         tc_fence_before();
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++done_a;
         tc_fence_after();
-        if (tid == 0) {
+        if (issuer) {
+            ++done_a;
             const uint32_t aS = smem_u32(sm.aop), bW = smem_u32(sm.imgA);
             constexpr uint32_t kSbo = (kD / 8) * 128;
             for (int ks = 0; ks < kD / 16; ++ks)
@@ -1108,86 +1248,89 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
                 umma_bf16(tmem + 2 * kC, umma_desc(aS + 2 * kSPart + 256 * ks, kSbo),
                           umma_desc(bW + (2 * kC / 8) * kSbo + 256 * ks, kSbo), kIdesc64, 1u);
             umma_commit(&sm.mma_g);
+            ++issued_g;
         }
-        ++issued_g;
         // The previous chunk's outputs, while those products run.
-        if (c > 0) store_outputs();
+        if (compute && c > 0) store_outputs();
 
-        got = wait_parity(&sm.mma_g, (uint32_t)waits_g & 1u);
-        got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
+        got = wait_parity(&sm.mma_g, (uint32_t)c & 1u);
+        if (compute) got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
+        if (issuer && got) {
+            ++waits_g;
+            if (c + 1 < nch) {  // the BW buffer is free again
+                issue_a(c + 1);
+                ++issued_a;
+            }
+        }
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++waits_g, ++done_c;
         tc_fence_after();
-        if (c + 1 < nch) {  // the BW buffer is free again
-            if (tid == 0) issue_a(c + 1);
-            ++issued_a;
-        }
-        // --- E = U - W M and g Q M for this thread's 32 tokens
+        // --- E = U - W M and g Q M for this thread's 16 tokens
         const float* gq = reinterpret_cast<const float*>(sm.imgC);
-        const float* gk = gq + kC;
         const float gC = gq[2 * kC];
-        const float4* ut = reinterpret_cast<const float4*>(sm.imgC + kR2GBytes) + j * (kC / 4);
+        if (compute) {
+            const float* gk = gq + kC;
+            const float4* ut = reinterpret_cast<const float4*>(sm.imgC + kR2GBytes) + j;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const uint32_t col = (uint32_t)(32 * half + 16 * p);
-            uint32_t r0[16], r1[16], r2[16], r3[16];
-            tmem_ld16_issue(tmem + lane_base + col, r0);
-            tmem_ld16_issue(tmem + lane_base + kC + col, r1);
-            tmem_ld16_issue(tmem + lane_base + 2 * kC + col, r2);
-            tmem_ld16_issue(tmem + lane_base + 3 * kC + col, r3);
-            tmem_wait_ld();
-            tie_regs(r0), tie_regs(r1), tie_regs(r2), tie_regs(r3);
-            float e[16], ep[16];
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t col = (uint32_t)(16 * quarter + 8 * p);
+                uint32_t r0[8], r1[8], r2[8], r3[8];
+                tmem_ld8_issue(tmem + lane_base + col, r0);
+                tmem_ld8_issue(tmem + lane_base + kC + col, r1);
+                tmem_ld8_issue(tmem + lane_base + 2 * kC + col, r2);
+                tmem_ld8_issue(tmem + lane_base + 3 * kC + col, r3);
+                tmem_wait_ld();
+                tie_regs8(r0), tie_regs8(r1), tie_regs8(r2), tie_regs8(r3);
+                float e[8], ep[8];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int gi = (int)(col / 4) + q4;
-                const float4 uu = ut[gi ^ (j & 7)];
-                const float uv[4] = {uu.x, uu.y, uu.z, uu.w};
+                for (int q4 = 0; q4 < 2; ++q4) {
+                    const int gi = (int)(col / 4) + q4;
+                    const float4 uu = ut[gi * kD];
+                    const float uv[4] = {uu.x, uu.y, uu.z, uu.w};
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int mm = 4 * q4 + m, t = (int)col + mm;
-                    const float wm = (__uint_as_float(r0[mm]) + __uint_as_float(r1[mm])) + __uint_as_float(r2[mm]);
-                    e[mm] = uv[m] - wm;
-                    ep[mm] = e[mm] * gk[t];
-                    qm[16 * p + mm] = __uint_as_float(r3[mm]) * gq[t];
+                    for (int m = 0; m < 4; ++m) {
+                        const int mm = 4 * q4 + m, t = (int)col + mm;
+                        const float wm =
+                            (__uint_as_float(r0[mm]) + __uint_as_float(r1[mm])) + __uint_as_float(r2[mm]);
+                        e[mm] = uv[m] - wm;
+                        ep[mm] = e[mm] * gk[t];
+                        qm[8 * p + mm] = __uint_as_float(r3[mm]) * gq[t];
+                    }
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float x8[8], y8[8];
-#pragma unroll
-                for (int m = 0; m < 8; ++m) x8[m] = ep[8 * u + m], y8[m] = e[8 * u + m];
                 uint4 p0, p1, p2;
-                const uint32_t off = core_off(j, (int)col + 8 * u, kC);
-                split3x8(x8, p0, p1, p2);
+                const uint32_t off = core_off(j, (int)col, kC);
+                split3x8_fast(ep, p0, p1, p2);
                 *reinterpret_cast<uint4*>(sm.aop + off) = p0;
                 *reinterpret_cast<uint4*>(sm.aop + kEPart + off) = p1;
                 *reinterpret_cast<uint4*>(sm.aop + 2 * kEPart + off) = p2;
-                split3x8(y8, p0, p1, p2);
+                split2x8_fast(e, p0, p1);
                 *reinterpret_cast<uint4*>(sm.aop + 3 * kEPart + off) = p0;
                 *reinterpret_cast<uint4*>(sm.aop + 4 * kEPart + off) = p1;
             }
+            async_proxy_fence();
         }
         out_t0 = c * kC;
         out_n = min(kC, a.L - out_t0);
-        async_proxy_fence();
+        got = true;
+        if (issuer) {
+            ++done_c;
+            got = wait_parity(&sm.bar_b, (uint32_t)c & 1u);
+        }
         tc_fence_before();
-        got = wait_parity(&sm.bar_b, (uint32_t)c & 1u);
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++done_b;
         tc_fence_after();
-        if (c + 1 < nch) {  // U^T and the gate factors are in registers or consumed
-            if (tid == 0) issue_c(c + 1);
-            ++issued_c;
-        }
         // --- state update first (the chain waits for it), then the outputs' products
-        if (tid == 0) {
+        if (issuer) {
+            ++done_b;
+            if (c + 1 < nch) {  // U^T and the gate factors are consumed
+                issue_c(c + 1);
+                ++issued_c;
+            }
             const uint32_t aE = smem_u32(sm.aop), bK = smem_u32(sm.imgB), bP = bK + kR2BKBytes;
             constexpr uint32_t kSbo = (kC / 8) * 128;
             for (int part = 0; part < 3; ++part)
@@ -1202,49 +1345,53 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) 
                 umma_bf16(tmem + kTmemDO + kC, umma_desc(aE + 4 * kEPart + 256 * ks, kSbo),
                           umma_desc(bP + (kC / 8) * kSbo + 256 * ks, kSbo), kIdesc64, 1u);
             umma_commit(&sm.mma_o);
+            ++issued_u, ++issued_o;
         }
-        ++issued_u, ++issued_o;
-        if (__syncthreads_or(wait_parity(&sm.mma_u, (uint32_t)waits_u & 1u) ? 0 : 1)) {
+        got = wait_parity(&sm.mma_u, (uint32_t)c & 1u);
+        if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++waits_u;
+        if (issuer) ++waits_u;
         tc_fence_after();
-#pragma unroll
-        for (int u = 0; u < 4; u += 2) {
+        if (compute) {
             uint32_t r0[16], r1[16];
-            tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(64 * half + 16 * u), r0);
-            tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(64 * half + 16 * u + 16), r1);
+            tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(32 * quarter), r0);
+            tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(32 * quarter + 16), r1);
             tmem_wait_ld();
             tie_regs(r0), tie_regs(r1);
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
-                s[16 * u + m] = fmaf(gC, s[16 * u + m], __uint_as_float(r0[m]));
-                s[16 * u + 16 + m] = fmaf(gC, s[16 * u + 16 + m], __uint_as_float(r1[m]));
+                s[m] = fmaf(gC, s[m], __uint_as_float(r0[m]));
+                s[16 + m] = fmaf(gC, s[16 + m], __uint_as_float(r1[m]));
             }
         }
         // The outputs' products still read the E parts: the next S parts overwrite them.
-        const bool got_o = wait_parity(&sm.mma_o, (uint32_t)waits_o & 1u);
+        got = wait_parity(&sm.mma_o, (uint32_t)c & 1u);
         tc_fence_before();
-        if (__syncthreads_or(got_o ? 0 : 1)) {
+        if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
-        ++waits_o;
         tc_fence_after();
-        if (c + 1 < nch) {  // K^T and the P tile are consumed
-            if (tid == 0) issue_b(c + 1);
-            ++issued_b;
-            split_s();
+        if (issuer) {
+            ++waits_o;
+            if (c + 1 < nch) {  // K^T and the P tile are consumed
+                issue_b(c + 1);
+                ++issued_b;
+            }
         }
+        if (compute && c + 1 < nch) split_s();
     }
 
     if (ok) {
-        store_outputs();  // the last chunk's
-        float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)(64 * half) * kD + j;
+        if (compute) {
+            store_outputs();  // the last chunk's
+            float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)(32 * quarter) * kD + j;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) MD[(size_t)i * kD] = s[i];
-    } else if (tid == 0) {
+            for (int i = 0; i < 32; ++i) MD[(size_t)i * kD] = s[i];
+        }
+    } else if (issuer) {
         // Something never arrived: record it, then give every copy and MMA still
         // outstanding one more bounded wait before shared memory and TMEM go.
         record(a.err, GDN_ERR_TIMEOUT);
@@ -1335,7 +1482,7 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
         // The scan starts behind the prepare kernel with programmatic dependent launch.
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(B * Hv));
-        cfg.blockDim = dim3(kNT);
+        cfg.blockDim = dim3(kScanThreads);
         cfg.dynamicSmemBytes = (size_t)s2;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];

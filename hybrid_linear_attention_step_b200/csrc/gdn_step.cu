@@ -82,6 +82,9 @@ __device__ __forceinline__ float load_in<__nv_bfloat16>(const void* base, size_t
     return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(base) + idx));
 }
 
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
 // Request status: kRun when src and all T destination slots of request b lie
 // inside the pool; kPad when src is the padding sentinel GDN_SLOT_NONE (the
 // request is skipped silently, its destinations are not looked at); kBad
@@ -530,6 +533,157 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             // The other buffer was last read during token t-1, before this token's barrier.
             stage(cb ^ 1, kx, qx, vx, ax, bx, dx);
             __syncthreads();
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Multi-token form for short drafts (2 <= T <= kStageT = 4, no fused prologue): every
+// token's inputs are requested together with the state tile at kernel start and
+// staged in shared memory (in their input type), so the token loop waits on no
+// global load and takes one barrier per token (the reduction buffers alternate by
+// token parity; a buffer is rewritten two tokens later, after every thread has
+// passed the barrier in between).  Same thread layout and the same per-token
+// arithmetic in the same order as gdn_tile1_kernel and gdn_tile_kernel: identical
+// bits.
+// ---------------------------------------------------------------------------
+constexpr int kStageT = 4;
+
+template <int DK, int DV, int DVC, int NT, int MINB, typename InT>
+__global__ void __launch_bounds__(NT, MINB) gdn_tileT_kernel(StepArgs a) {
+    constexpr int CG = DVC / 4;
+    static_assert(DV % DVC == 0 && DVC % 4 == 0 && NT % CG == 0 && NT >= DK && NT >= DVC, "tile shape");
+    constexpr int RG = NT / CG;
+    static_assert(DK % RG == 0, "tile shape");
+    constexpr int RPT = DK / RG;
+    constexpr int NC = DV / DVC;
+
+    __shared__ InT ks[kStageT][DK];
+    __shared__ InT qs[kStageT][DK];
+    __shared__ InT vs[kStageT][DVC];
+    __shared__ float gates[kStageT][2];
+    __shared__ int dst_s[kStageT];
+    __shared__ float4 red_u[2][RG][CG];
+    __shared__ float4 red_w[2][RG][CG];
+    __shared__ float kq_s[2];
+
+    const int tid = threadIdx.x;
+    const int cg = tid % CG;
+    const int rg = tid / CG;
+    const int chunk = blockIdx.x % NC;
+    const int unit = blockIdx.x / NC;
+    const int h = unit % a.Hv;
+    const int b = unit / a.Hv;
+    const int T = a.T;
+
+    grid_dependency_wait();
+    int src, dst0 = 0;
+    const int status = request_status(a, b, T, src, dst0);
+    if (status != kRun) {
+        if (status == kBad && tid == 0) record_error(a.err, GDN_ERR_INDEX);
+        return;
+    }
+    const int col4 = chunk * CG + cg;
+    const int toff = rg * (DV / 4) + col4;
+    constexpr int kRowStep = RG * (DV / 4);
+    const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV)) + toff;
+    float4 s[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+    allow_dependent_launch();
+
+    const int hk = h / a.G;
+    const InT* kin = static_cast<const InT*>(a.k);
+    const InT* qin = static_cast<const InT*>(a.q);
+    const InT* vin = static_cast<const InT*>(a.v);
+    // Every token's loads are in flight together before any of them is staged.
+    InT kr[kStageT], qr[kStageT], vr[kStageT];
+#pragma unroll
+    for (int t = 0; t < kStageT; ++t) {
+        if (t < T) {
+            const size_t tok = (size_t)b * T + t;
+            if (tid < DK) {
+                kr[t] = kin[(tok * a.Hk + hk) * DK + tid];
+                qr[t] = qin[(tok * a.Hk + hk) * DK + tid];
+            }
+            if (tid < DVC) vr[t] = vin[(tok * a.Hv + h) * DV + (size_t)chunk * DVC + tid];
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kStageT; ++t) {
+        if (t < T) {
+            if (tid < DK) {
+                ks[t][tid] = kr[t];
+                qs[t][tid] = qr[t];
+            }
+            if (tid < DVC) vs[t][tid] = vr[t];
+        }
+    }
+    if (tid < T) {
+        const size_t tok = (size_t)b * T + tid;
+        gates[tid][0] = __ldg(a.alpha + tok * a.Hv + h);
+        gates[tid][1] = __ldg(a.beta + tok * a.Hv + h);
+        dst_s[tid] = tid == 0 ? dst0 : __ldg(a.dst_idx + tok);
+    }
+    __syncthreads();
+
+    for (int t = 0; t < T; ++t) {
+        const int cb = t & 1;
+        float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const int i = m * RG + rg;
+            fma4(pu, s[m], to_f32(ks[t][i]));
+            fma4(pw, s[m], to_f32(qs[t][i]));
+        }
+        red_u[cb][rg][cg] = pu;
+        red_w[cb][rg][cg] = pw;
+        if (tid < 32) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = tid; i < DK; i += 32) acc = fmaf(to_f32(ks[t][i]), to_f32(qs[t][i]), acc);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+            if (tid == 0) kq_s[cb] = acc;
+        }
+        __syncthreads();
+
+        float4 u = red_u[cb][0][cg];
+        float4 w = red_w[cb][0][cg];
+#pragma unroll
+        for (int r = 1; r < RG; ++r) {
+            add4_rn(u, red_u[cb][r][cg]);
+            add4_rn(w, red_w[cb][r][cg]);
+        }
+        const float al = gates[t][0];
+        const float be = gates[t][1];
+        const float4 vv = make_float4(to_f32(vs[t][4 * cg]), to_f32(vs[t][4 * cg + 1]), to_f32(vs[t][4 * cg + 2]),
+                                      to_f32(vs[t][4 * cg + 3]));
+        float4 c;
+        c.x = __fmul_rn(be, fmaf(-al, u.x, vv.x));
+        c.y = __fmul_rn(be, fmaf(-al, u.y, vv.y));
+        c.z = __fmul_rn(be, fmaf(-al, u.z, vv.z));
+        c.w = __fmul_rn(be, fmaf(-al, u.w, vv.w));
+        const size_t gh = ((size_t)b * T + t) * a.Hv + h;
+        if (rg == 0) {
+            const float kq = kq_s[cb];
+            float4 o;
+            o.x = fmaf(c.x, kq, __fmul_rn(al, w.x));
+            o.y = fmaf(c.y, kq, __fmul_rn(al, w.y));
+            o.z = fmaf(c.z, kq, __fmul_rn(al, w.z));
+            o.w = fmaf(c.w, kq, __fmul_rn(al, w.w));
+            __stcs(reinterpret_cast<float4*>(a.out + gh * DV) + col4, o);
+        }
+        float4* D = reinterpret_cast<float4*>(a.pool + ((size_t)dst_s[t] * a.Hv + h) * (DK * DV)) + toff;
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const float ki = to_f32(ks[t][m * RG + rg]);
+            s[m].x = fmaf(ki, c.x, __fmul_rn(al, s[m].x));
+            s[m].y = fmaf(ki, c.y, __fmul_rn(al, s[m].y));
+            s[m].z = fmaf(ki, c.z, __fmul_rn(al, s[m].z));
+            s[m].w = fmaf(ki, c.w, __fmul_rn(al, s[m].w));
+            __stcs(D + m * kRowStep, s[m]);
         }
     }
 }
@@ -998,6 +1152,9 @@ gdn_status launch_tile_impl(const StepArgs& a, int32_t dtype, cudaStream_t strea
     if (a.T == 1) {
         e = bf ? launch_pdl(gdn_tile1_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16, FUSE>, grid, NT, stream, a)
                : launch_pdl(gdn_tile1_kernel<DK, DV, DVC, NT, MINB, float, FUSE>, grid, NT, stream, a);
+    } else if (!FUSE && !a.prefill && a.T <= kStageT) {
+        e = bf ? launch_pdl(gdn_tileT_kernel<DK, DV, DVC, NT, MINB, __nv_bfloat16>, grid, NT, stream, a)
+               : launch_pdl(gdn_tileT_kernel<DK, DV, DVC, NT, MINB, float>, grid, NT, stream, a);
     } else {
         // The fused multi-token form needs a few more registers than 5 CTAs/SM allow.
         constexpr int MINB_T = (FUSE && MINB > 1) ? MINB - 1 : MINB;
