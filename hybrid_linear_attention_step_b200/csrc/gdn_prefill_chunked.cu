@@ -621,14 +621,34 @@ struct SmemP {
 };
 static_assert(sizeof(SmemP) <= 113 * 1024, "two prepare CTAs per SM");
 
-// The 8 bf16 of a 16-byte granule (one token, 8 consecutive feature indices d0..d0+7)
-// into column t of a K-major operand tile whose rows are the feature index.
-__device__ __forceinline__ void scatter_granule(unsigned char* tile, const uint4& x, int d0, int t) {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+// bf16 row block R (rows = tokens, row stride kD + 2: an odd number of 32-bit words, so
+// the column reads below are conflict-free) gathered into a K-major operand tile with kD
+// rows (the feature index) and kC columns (tokens), in shared memory and, when global_img
+// is not null, in global memory too.  Consecutive threads write consecutive 16-byte granules.
+__device__ __forceinline__ void gather_transposed(const __nv_bfloat16* R, unsigned char* img,
+                                                  unsigned char* global_img, int tid) {
+    for (int e = tid; e < kD * (kC / 8); e += kNT) {
+        const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // row j, tokens 8g..8g+7
+        uint16_t x[8];
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-        *reinterpret_cast<uint16_t*>(tile + core_off(d0 + m, t, kC)) = (uint16_t)(w[m >> 1] >> (16 * (m & 1)));
+        for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint16_t*>(R + (8 * g + m) * (kD + 2) + j);
+        uint4 w;
+        w.x = x[0] | ((uint32_t)x[1] << 16);
+        w.y = x[2] | ((uint32_t)x[3] << 16);
+        w.z = x[4] | ((uint32_t)x[5] << 16);
+        w.w = x[6] | ((uint32_t)x[7] << 16);
+        const uint32_t off = core_off(j, 8 * g, kC);
+        *reinterpret_cast<uint4*>(img + off) = w;
+        if (global_img != nullptr) *reinterpret_cast<uint4*>(global_img + off) = w;
+    }
 }
+
+__device__ __forceinline__ void store_row8(__nv_bfloat16* row, const uint4& x) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(row);
+    r[0] = x.x, r[1] = x.y, r[2] = x.z, r[3] = x.w;
+}
+
+static_assert(kC * (kD + 2) * 2 <= kC * (kC + 4) * 4, "a bf16 row block fits in an A or T array");
 
 __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_p[];
@@ -686,6 +706,10 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         }
     }
     if (warp == 0) gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, nullptr, true);
+    // K and V rows go to row buffers in the T and A arrays (both written only after D0),
+    // to be gathered into the K^T and V^T operand tiles.
+    __nv_bfloat16* krows = reinterpret_cast<__nv_bfloat16*>(&sm.T[0][0]);
+    __nv_bfloat16* vrows = reinterpret_cast<__nv_bfloat16*>(&sm.u.ra.A[0][0]);
 #pragma unroll
     for (int u = 0; u < kGr; ++u) {
         const int e = tid + kNT * u;
@@ -693,8 +717,8 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         *reinterpret_cast<uint4*>(sm.u.KQ + core_off(t, 8 * g, kD)) = kq[u];
         *reinterpret_cast<uint4*>(sm.u.KQ + core_off(kC + t, 8 * g, kD)) = qq[u];
         *reinterpret_cast<uint4*>(rec + kR2BW + core_off(3 * kC + t, 8 * g, kD)) = qq[u];
-        scatter_granule(sm.KT, kq[u], 8 * g, t);
-        scatter_granule(sm.VT, vv[u], 8 * g, t);
+        store_row8(krows + t * (kD + 2) + 8 * g, kq[u]);
+        store_row8(vrows + t * (kD + 2) + 8 * g, vv[u]);
     }
     async_proxy_fence();
     tc_fence_before();
@@ -708,12 +732,10 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                       kIdesc, ks != 0 ? 1u : 0u);
         umma_commit(&sm.mma);
     }
-    // The K^T tile goes to the record as it is (the scan's B operand of the state update).
-#pragma unroll
-    for (int u = 0; u < (int)(kR2BKBytes / 16) / kNT; ++u) {
-        const int e = tid + kNT * u;
-        *reinterpret_cast<uint4*>(rec + kR2BK + 16 * e) = *reinterpret_cast<const uint4*>(sm.KT + 16 * e);
-    }
+    // K^T (also the record's tile: the scan's B operand of the state update) and V^T,
+    // while D0 runs.
+    gather_transposed(krows, sm.KT, rec + kR2BK, tid);
+    gather_transposed(vrows, sm.VT, nullptr, tid);
     bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
     int waits = ok ? 1 : 0, issued = 1;
     if (ok) {
@@ -1206,19 +1228,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(Chun
     float qm[16];   // g_t (q_t M)_j for this thread's 16 tokens of the current chunk
     int out_t0 = 0, out_n = 0;  // chunk whose outputs are pending
 
-    // Outputs of the chunk whose D_O was last completed: o = g q M + P E.
-    auto store_outputs = [&]() {
-        const uint32_t col = (uint32_t)(16 * quarter);
-        uint32_t r0[16], r1[16];
-        tmem_ld16_issue(tmem + lane_base + kTmemDO + col, r0);
-        tmem_ld16_issue(tmem + lane_base + kTmemDO + kC + col, r1);
+    // Outputs of the chunk whose D_O was last completed, o = g q M + P E: tokens
+    // 16 quarter + 8 part .. +8 of this thread's value row (warp-collective TMEM reads).
+    auto store_outputs = [&](int part) {
+        const uint32_t col = (uint32_t)(16 * quarter + 8 * part);
+        uint32_t r0[8], r1[8];
+        tmem_ld8_issue(tmem + lane_base + kTmemDO + col, r0);
+        tmem_ld8_issue(tmem + lane_base + kTmemDO + kC + col, r1);
         tmem_wait_ld();
-        tie_regs(r0), tie_regs(r1);
+        tie_regs8(r0), tie_regs8(r1);
         float* ob = a.out + (((size_t)b * a.L + out_t0) * a.Hv + h) * kD + j;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
+        for (int m = 0; m < 8; ++m) {
             const int t = (int)col + m;
-            if (t < out_n) ob[(size_t)t * a.Hv * kD] = qm[m] + (__uint_as_float(r1[m]) + __uint_as_float(r0[m]));
+            if (t < out_n)
+                ob[(size_t)t * a.Hv * kD] = qm[8 * part + m] + (__uint_as_float(r1[m]) + __uint_as_float(r0[m]));
         }
     };
 
@@ -1234,24 +1258,39 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(Chun
             break;
         }
         tc_fence_after();
-        if (issuer) {
-            ++done_a;
-            const uint32_t aS = smem_u32(sm.aop), bW = smem_u32(sm.imgA);
-            constexpr uint32_t kSbo = (kD / 8) * 128;
-            for (int ks = 0; ks < kD / 16; ++ks)
-                umma_bf16(tmem, umma_desc(aS + 256 * ks, kSbo), umma_desc(bW + 256 * ks, kSbo), kIdesc256,
-                          ks != 0 ? 1u : 0u);
-            for (int ks = 0; ks < kD / 16; ++ks)
-                umma_bf16(tmem + kC, umma_desc(aS + kSPart + 256 * ks, kSbo),
-                          umma_desc(bW + (kC / 8) * kSbo + 256 * ks, kSbo), kIdesc192, 1u);
-            for (int ks = 0; ks < kD / 16; ++ks)
-                umma_bf16(tmem + 2 * kC, umma_desc(aS + 2 * kSPart + 256 * ks, kSbo),
-                          umma_desc(bW + (2 * kC / 8) * kSbo + 256 * ks, kSbo), kIdesc64, 1u);
-            umma_commit(&sm.mma_g);
-            ++issued_g;
+        // The chunk's first products, issued by thread 0 in three batches (one per S
+        // part) with its warp's share of the previous chunk's outputs stored in between;
+        // the other warps store theirs while the products run.
+        const uint32_t aS = smem_u32(sm.aop), bW = smem_u32(sm.imgA);
+        constexpr uint32_t kSboG = (kD / 8) * 128;
+        if (warp == 0) {
+            if (issuer) {
+                ++done_a;
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    umma_bf16(tmem, umma_desc(aS + 256 * ks, kSboG), umma_desc(bW + 256 * ks, kSboG), kIdesc256,
+                              ks != 0 ? 1u : 0u);
+            }
+            __syncwarp();
+            if (c > 0) store_outputs(0);
+            if (issuer) {
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    umma_bf16(tmem + kC, umma_desc(aS + kSPart + 256 * ks, kSboG),
+                              umma_desc(bW + (kC / 8) * kSboG + 256 * ks, kSboG), kIdesc192, 1u);
+            }
+            __syncwarp();
+            if (c > 0) store_outputs(1);
+            if (issuer) {
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    umma_bf16(tmem + 2 * kC, umma_desc(aS + 2 * kSPart + 256 * ks, kSboG),
+                              umma_desc(bW + (2 * kC / 8) * kSboG + 256 * ks, kSboG), kIdesc64, 1u);
+                umma_commit(&sm.mma_g);
+                ++issued_g;
+            }
+            __syncwarp();
+        } else if (c > 0) {
+            store_outputs(0);
+            store_outputs(1);
         }
-        // The previous chunk's outputs, while those products run.
-        if (compute && c > 0) store_outputs();
 
         got = wait_parity(&sm.mma_g, (uint32_t)c & 1u);
         if (compute) got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
@@ -1386,7 +1425,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(Chun
 
     if (ok) {
         if (compute) {
-            store_outputs();  // the last chunk's
+            store_outputs(0);  // the last chunk's
+            store_outputs(1);
             float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)(32 * quarter) * kD + j;
 #pragma unroll
             for (int i = 0; i < 32; ++i) MD[(size_t)i * kD] = s[i];
