@@ -40,6 +40,7 @@
 
 #include "gdn_step.h"
 
+#include <cuda.h>  // CUtensorMap and its encoder's types (the encoder comes from the runtime)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -62,36 +63,40 @@ constexpr size_t kRecP = kRecTb + (size_t)kC * kC * 4;  // PT [64][64] fp32
 constexpr size_t kRecG = kRecP + (size_t)kC * kC * 4;   // log g [64]
 constexpr size_t kRecF32Bytes = kRecG + (size_t)kC * 4;
 
-// Workspace record of the bf16-input path (tensor cores), bytes: the scan's three
-// shared-memory images, each one contiguous range.
-//   image A  BW  [W_lo | W_mid | W_hi | Q]: 256 rows (tokens, per part) x dk, bf16 parts of
-//                W = T diag(beta g) K and the bf16 Q, K-major no-swizzle operand layout
-//   image B  BK  K^T: dk rows x 64 tokens, same layout
-//            BP  [P_mid | P_hi]: 128 rows (t, per part) x 64 (i), bf16 parts of P
-//   image C  G   g_t [64], g_C / g_t [64], g_C, 3 zero words
-//            UT  U^T fp32 as 16 x 128 float4 granules: granule q of value row j (tokens
-//                4q..4q+3 of U[t][j]) at index q * dv + j, so that 32 consecutive rows
-//                are 512 contiguous bytes for the writer and the reader alike
-constexpr size_t kR2BW = 0;
-constexpr uint32_t kR2BWBytes = 4 * kC * kD * 2;
-constexpr size_t kR2BK = kR2BW + kR2BWBytes;
-constexpr uint32_t kR2BKBytes = kD * kC * 2;
-constexpr size_t kR2BP = kR2BK + kR2BKBytes;
-constexpr uint32_t kR2BPBytes = 2 * kC * kC * 2;
-constexpr size_t kR2G = kR2BP + kR2BPBytes;
+// Workspace record of the bf16-input path (tensor cores), bytes.  The tiles the scan
+// gives the tensor cores straight from the inputs (Q, K) are not in it: it loads them
+// itself.
+//   W   [W_lo | W_mid | W_hi] for dk 0..63, then the same for dk 64..127: six tiles of
+//       64 tokens x 64 features (bf16 parts of W = T diag(beta g) K), each in the
+//       128-byte-swizzled K-major layout a tensor copy writes (row t at 128 t, its
+//       16-byte granule q at position q ^ (t & 7))
+//   P   [P_mid | P_hi]: 128 rows (t, per part) x 64 (i), bf16 parts of P, K-major
+//       no-swizzle core-matrix layout
+//   G   g_t [64], g_C / g_t [64], g_C, 3 zero words
+//   UT  U^T fp32 as 16 x 128 float4 granules: granule q of value row j (tokens 4q..4q+3
+//       of U[t][j]) at index q * dv + j, so that 32 consecutive rows are 512 contiguous
+//       bytes for the writer and the reader alike
+// G and UT are one contiguous range (the scan copies them together).
+constexpr uint32_t kSwTile = kC * 64 * 2;              // one 64 x 64 bf16 swizzled tile
+constexpr size_t kR2W = 0;
+constexpr uint32_t kR2WBytes = 6 * kSwTile;
+constexpr size_t kR2P = kR2W + kR2WBytes;
+constexpr uint32_t kR2PBytes = 2 * kC * kC * 2;
+constexpr size_t kR2G = kR2P + kR2PBytes;
 constexpr uint32_t kR2GBytes = (2 * kC + 4) * 4;
 constexpr size_t kR2UT = kR2G + kR2GBytes;
 constexpr uint32_t kR2UTBytes = kD * kC * 4;
 constexpr size_t kR2Bytes = kR2UT + kR2UTBytes;
-constexpr uint32_t kImgA = kR2BWBytes;                 // bytes of image A
-constexpr uint32_t kImgB = kR2BKBytes + kR2BPBytes;    // image B
-constexpr uint32_t kImgC = kR2GBytes + kR2UTBytes;     // image C
+constexpr uint32_t kImgA = 8 * kSwTile;                // [W_lo W_mid W_hi Q] x two feature halves
+constexpr uint32_t kImgB = 2 * kSwTile + kR2PBytes;    // K (two feature halves) | P parts
+constexpr uint32_t kImgC = kR2GBytes + kR2UTBytes;     // G | UT
 
-constexpr size_t kRecBytes = kR2Bytes > kRecF32Bytes ? kR2Bytes : kRecF32Bytes;
-static_assert(kRecTb % 16 == 0 && kRecP % 16 == 0 && kRecG % 16 == 0 && kR2BK % 16 == 0 && kR2BP % 16 == 0 &&
-                  kR2G % 16 == 0 && kR2UT % 16 == 0 && kRecBytes % 16 == 0,
-              "16-byte records");
-static_assert(kImgA % 16 == 0 && kImgB % 16 == 0 && kImgC % 16 == 0, "16-byte bulk copies");
+constexpr size_t kRecMax = kR2Bytes > kRecF32Bytes ? kR2Bytes : kRecF32Bytes;
+constexpr size_t kRecBytes = (kRecMax + 255) / 256 * 256;
+static_assert(kRecTb % 16 == 0 && kRecP % 16 == 0 && kRecG % 16 == 0 && kR2P % 16 == 0 && kR2G % 16 == 0 &&
+                  kR2UT % 16 == 0,
+              "16-byte record fields");
+static_assert(kImgC % 16 == 0 && kR2PBytes % 16 == 0 && (3 * kSwTile) % 16 == 0, "16-byte bulk copies");
 
 struct ChunkArgs {
     float* pool;
@@ -161,6 +166,50 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t sbo) {
 // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, both K-major.
 __host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand (layout type 2, version 1),
+// in the canonical forms of the tcgen05 shared-memory descriptor:
+//   K-major:  rows 128 B apart, 8-row atoms (1024 B) `sbo` apart; the 32-byte step of one
+//             MMA along K is added to the start address (lbo is not used: 16)
+//   MN-major: 64 consecutive M (or N) elements per 128-byte row, one row per K index,
+//             8-row atoms `sbo` apart along K, 64-element blocks `lbo` apart along M (N)
+// The tiles start on 1024-byte boundaries, where the swizzle pattern starts.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+constexpr uint32_t kIdescAmn = 1u << 15;  // instruction descriptor: A is MN-major
+constexpr uint32_t kIdescBmn = 1u << 16;  // B is MN-major
+
+// The k, q and v tensors as 4-d tensor maps {feature, head, token, request} with a box
+// of 64 features x 1 head x 64 tokens, 128-byte swizzle: one load is one 8 KB operand
+// tile of a chunk; tokens past L read as zero.
+struct TileMaps {
+    CUtensorMap k, q, v;
+};
+
+// One tile load (no multicast) completing on `bar` with its byte count.
+__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, int feat, int head, int tok, int req,
+                                         uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(feat), "r"(head), "r"(tok), "r"(req), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Dynamic shared memory rounded up to the next 1024-byte boundary (kernels that hold
+// swizzled tiles allocate 1 KB more than their plan).
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+    const uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// Byte offset of the 16-byte granule q (features 8q..8q+7) of row t in a 128-byte-swizzled
+// 64-row tile.
+__host__ __device__ constexpr uint32_t sw128_off(int t, int q) {
+    return (uint32_t)(t * 128 + ((q ^ (t & 7)) << 4));
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
@@ -588,71 +637,45 @@ __device__ __forceinline__ void invert_blocked(const float (*A)[kC + 4], float (
 
 // ---------------------------------------------------------------------------
 // Kernel 1, tensor-core form (bf16 inputs), one CTA per (request, head, chunk):
+//   the chunk's k, q and v tiles arrive by tensor copies in the 128-byte-swizzled layout;
 //   D0  = [K; Q] K^T on the tensor cores (M = 128, N = 64, K = dk; exact bf16 products),
 //         read out as A[t][i] = beta_t (g_t / g_i) k_t.k_i (i < t) and
 //         P[t][i] = (g_t / g_i) q_t.k_i (i <= t);
 //   T   = (I + A)^-1 in fp32 on the CUDA cores, in 16 x 16 blocks (invert_blocked);
 //   D_U = V^T (T diag(beta))^T = U^T  and  D_W = K^T (T diag(beta g))^T = W^T on the tensor
-//         cores, V and K exact in bf16 and each T factor in three bf16 parts (24 bits).
-// The record receives the scan's operand images: [W_lo | W_mid | W_hi | Q], K^T and
-// [P_mid | P_hi] as bf16 tensor-core tiles, the gate factors g_t, g_C / g_t, g_C, and
-// U^T in fp32.
+//         cores, V^T and K^T read from the same tiles as MN-major operands (exact in bf16),
+//         each T factor in three bf16 parts (24 bits).
+// The record receives the scan's operands that are not inputs: W in bf16 parts,
+// [P_mid | P_hi], the gate factors g_t, g_C / g_t, g_C, and U^T in fp32.
 // ---------------------------------------------------------------------------
 struct SmemP {
+    // [K lo | Q lo | K hi | Q hi] (lo, hi: features 0..63, 64..127), 128-byte swizzled:
+    // A operand of D0 (K rows also its B), K^T of D_W; once D0 is complete the two Q
+    // tiles hold the first two bf16 parts of D_W's B operand.
+    unsigned char KQ[4 * kSwTile];
+    unsigned char V[2 * kSwTile];            // [V lo | V hi]: V^T of D_U
     union {
-        unsigned char KQ[2 * kC * kD * 2];   // [K; Q]: A operand of D0 (rows 0..63 are also its B)
-        float P[3 * 16 * 16];                // scratch of the blocked inverse (once D0 is complete)
         struct {
-            unsigned char after_kq[2 * kC * kD * 2];
             float A[kC][kC + 4];             // the system's strictly lower part (float4 rows)
+            float P[3 * 16 * 16];            // scratch of the blocked inverse
         } ra;
-        unsigned char Bp[2][3][kC * kC * 2]; // B of D_U and D_W: (T diag(beta)), (T diag(beta g)), 3 parts
-                                             // each (over [K; Q] and A, both dead by then)
+        unsigned char Bp[4][kC * kC * 2];    // B of D_U: T diag(beta) in 3 parts; D_W's third part
         float W[kC][kD + 4];                 // W staged for its split (row stride spreads banks)
     } u;
     float T[kC][kC + 4];                     // (I + A)^-1
-    unsigned char VT[kD * kC * 2];           // V^T: A operand of D_U (dv rows x 64 tokens)
-    unsigned char KT[kD * kC * 2];           // K^T: A operand of D_W, and the record's K^T tile
     float lg[kC];
     float bt[kC];
     float bg[kC];                            // beta_t g_t
-    uint64_t mma;
+    uint64_t mma, ld;
     uint32_t tmem;
 };
-static_assert(sizeof(SmemP) <= 113 * 1024, "two prepare CTAs per SM");
+constexpr int kSmemP = (int)sizeof(SmemP) + 1024;  // + alignment slack
+static_assert(kSmemP <= 112 * 1024, "two prepare CTAs per SM");
 
-// bf16 row block R (rows = tokens, row stride kD + 2: an odd number of 32-bit words, so
-// the column reads below are conflict-free) gathered into a K-major operand tile with kD
-// rows (the feature index) and kC columns (tokens), in shared memory and, when global_img
-// is not null, in global memory too.  Consecutive threads write consecutive 16-byte granules.
-__device__ __forceinline__ void gather_transposed(const __nv_bfloat16* R, unsigned char* img,
-                                                  unsigned char* global_img, int tid) {
-    for (int e = tid; e < kD * (kC / 8); e += kNT) {
-        const int j = (e & 7) | ((e >> 6) << 3), g = (e >> 3) & 7;  // row j, tokens 8g..8g+7
-        uint16_t x[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) x[m] = *reinterpret_cast<const uint16_t*>(R + (8 * g + m) * (kD + 2) + j);
-        uint4 w;
-        w.x = x[0] | ((uint32_t)x[1] << 16);
-        w.y = x[2] | ((uint32_t)x[3] << 16);
-        w.z = x[4] | ((uint32_t)x[5] << 16);
-        w.w = x[6] | ((uint32_t)x[7] << 16);
-        const uint32_t off = core_off(j, 8 * g, kC);
-        *reinterpret_cast<uint4*>(img + off) = w;
-        if (global_img != nullptr) *reinterpret_cast<uint4*>(global_img + off) = w;
-    }
-}
-
-__device__ __forceinline__ void store_row8(__nv_bfloat16* row, const uint4& x) {
-    uint32_t* r = reinterpret_cast<uint32_t*>(row);
-    r[0] = x.x, r[1] = x.y, r[2] = x.z, r[3] = x.w;
-}
-
-static_assert(kC * (kD + 2) * 2 <= kC * (kC + 4) * 4, "a bf16 row block fits in an A or T array");
-
-__global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs a) {
+__global__ void __launch_bounds__(kNT, 2)
+    gdn_chunk_prepare_tc_kernel(ChunkArgs a, const __grid_constant__ TileMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem_p[];
-    SmemP& sm = *reinterpret_cast<SmemP*>(smem_p);
+    SmemP& sm = *reinterpret_cast<SmemP*>(align1024(smem_p));
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
     // Chunks in descending order: the records written last are the first ones the scan
@@ -676,7 +699,15 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         mbar_init(&sm.mma);
+        mbar_init(&sm.ld);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_expect_tx(&sm.ld, 6 * kSwTile);
+        tma_tile(sm.KQ, &maps.k, 0, hk, t0, b, &sm.ld);
+        tma_tile(sm.KQ + kSwTile, &maps.q, 0, hk, t0, b, &sm.ld);
+        tma_tile(sm.KQ + 2 * kSwTile, &maps.k, 64, hk, t0, b, &sm.ld);
+        tma_tile(sm.KQ + 3 * kSwTile, &maps.q, 64, hk, t0, b, &sm.ld);
+        tma_tile(sm.V, &maps.v, 0, h, t0, b, &sm.ld);
+        tma_tile(sm.V + kSwTile, &maps.v, 64, h, t0, b, &sm.ld);
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
@@ -684,60 +715,33 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // k, q, v in 16-byte granules: [K; Q] into the D0 operand image, Q also into the
-    // record's BW tile (rows 192..255), K and V scattered into the K^T and V^T operand
-    // tiles.  Every load is issued before the first store: the record's global stores
-    // could alias the inputs as far as the compiler knows, so interleaving them would
-    // serialise the loads.  Consecutive threads take consecutive granules of the image:
-    // token t = (e & 7) + 8 (e >> 7), group g = (e >> 3) & 15, e = tid + 256 u.
-    constexpr int kGr = kC * (kD / 8) / kNT;  // granules per thread
-    uint4 kq[kGr], qq[kGr], vv[kGr];
-#pragma unroll
-    for (int u = 0; u < kGr; ++u) {
-        const int e = tid + kNT * u;
-        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-        kq[u] = qq[u] = vv[u] = make_uint4(0, 0, 0, 0);
-        if (t < n) {
-            const size_t row = (((size_t)b * a.L + t0 + t) * a.Hk + hk) * kD + 8 * g;
-            const size_t vrow = (((size_t)b * a.L + t0 + t) * a.Hv + h) * kD + 8 * g;
-            kq[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + row));
-            qq[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row));
-            vv[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + vrow));
-        }
-    }
-    if (warp == 0) gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, nullptr, true);
-    // K and V rows go to row buffers in the T and A arrays (both written only after D0),
-    // to be gathered into the K^T and V^T operand tiles.
-    __nv_bfloat16* krows = reinterpret_cast<__nv_bfloat16*>(&sm.T[0][0]);
-    __nv_bfloat16* vrows = reinterpret_cast<__nv_bfloat16*>(&sm.u.ra.A[0][0]);
-#pragma unroll
-    for (int u = 0; u < kGr; ++u) {
-        const int e = tid + kNT * u;
-        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
-        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(t, 8 * g, kD)) = kq[u];
-        *reinterpret_cast<uint4*>(sm.u.KQ + core_off(kC + t, 8 * g, kD)) = qq[u];
-        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(3 * kC + t, 8 * g, kD)) = qq[u];
-        store_row8(krows + t * (kD + 2) + 8 * g, kq[u]);
-        store_row8(vrows + t * (kD + 2) + 8 * g, vv[u]);
-    }
-    async_proxy_fence();
+    if (warp == 1) gate_scan(a, b, h, t0, n, lane, sm.lg, sm.bt, nullptr, true);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
+    const uint32_t kq = smem_u32(sm.KQ), vt = smem_u32(sm.V);
+    bool got = true, ld_done = false;
     if (tid == 0) {
-        const uint32_t kq = smem_u32(sm.u.KQ);
-        for (int ks = 0; ks < kD / 16; ++ks)
-            umma_bf16(tmem, umma_desc(kq + 256 * ks, (kD / 8) * 128), umma_desc(kq + 256 * ks, (kD / 8) * 128),
-                      kIdesc, ks != 0 ? 1u : 0u);
-        umma_commit(&sm.mma);
+        got = ld_done = wait_parity(&sm.ld, 0);
+        if (got) {
+            tc_fence_after();
+            // D0: K-steps of 16 features, 32 bytes apart within a tile, the second
+            // feature half two tiles on.
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                const uint32_t at = kq + (ks < 4 ? 32u * ks : 2 * kSwTile + 32u * (ks - 4));
+                umma_bf16(tmem, umma_desc_sw128(at, 16, 1024), umma_desc_sw128(at, 16, 1024), kIdesc,
+                          ks != 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.mma);
+        }
     }
-    // K^T (also the record's tile: the scan's B operand of the state update) and V^T,
-    // while D0 runs.
-    gather_transposed(krows, sm.KT, rec + kR2BK, tid);
-    gather_transposed(vrows, sm.VT, nullptr, tid);
-    bool ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
-    int waits = ok ? 1 : 0, issued = 1;
+    int waits = 0, issued = got ? 1 : 0;
+    bool ok = !__syncthreads_or(got ? 0 : 1);
+    if (ok) {
+        ok = !__syncthreads_or(wait_parity(&sm.mma, 0) ? 0 : 1);
+        if (ok) ++waits;
+    }
     if (ok) {
         tc_fence_after();
         // D0 row r < 64: k_r . k_i -> A (scaled); row 64 + t: q_t . k_i -> P (record).
@@ -773,7 +777,7 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
                     }
                     uint4 p0, p1;
                     split2x8_fast(x, p0, p1);
-                    unsigned char* bp = rec + kR2BP;
+                    unsigned char* bp = rec + kR2P;
                     *reinterpret_cast<uint4*>(bp + core_off(t, i0 + g8, kC)) = p1;
                     *reinterpret_cast<uint4*>(bp + core_off(kC + t, i0 + g8, kC)) = p0;
                 }
@@ -784,9 +788,12 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         tc_fence_after();
 
         if (tid < kC) sm.bg[tid] = sm.bt[tid] * exp2f(sm.lg[tid]);  // beta_t g_t
-        invert_blocked(sm.u.ra.A, sm.T, sm.u.P, tid);  // ends with a barrier
+        invert_blocked(sm.u.ra.A, sm.T, sm.u.ra.P, tid);  // ends with a barrier
         // B operands of D_U and D_W: rows t, columns i, T[t][i] beta_i and T[t][i] beta_i g_i,
-        // each in three bf16 parts.
+        // each in three bf16 parts; D_W's first two parts go to the Q tiles, free since D0.
+        auto bpart = [&](int which, int p) -> unsigned char* {
+            return which == 0 ? sm.u.Bp[p] : (p == 0 ? sm.KQ + kSwTile : p == 1 ? sm.KQ + 3 * kSwTile : sm.u.Bp[3]);
+        };
         for (int e = tid; e < 2 * kC * (kC / 8); e += kNT) {
             const int which = e / (kC * (kC / 8)), rem = e % (kC * (kC / 8));
             const int t = (rem & 7) | ((rem >> 6) << 3), g = (rem >> 3) & 7;
@@ -799,24 +806,26 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             uint4 p0, p1, p2;
             split3x8_fast(xs, p0, p1, p2);
             const uint32_t off = core_off(t, 8 * g, kC);
-            *reinterpret_cast<uint4*>(sm.u.Bp[which][0] + off) = p0;
-            *reinterpret_cast<uint4*>(sm.u.Bp[which][1] + off) = p1;
-            *reinterpret_cast<uint4*>(sm.u.Bp[which][2] + off) = p2;
+            *reinterpret_cast<uint4*>(bpart(which, 0) + off) = p0;
+            *reinterpret_cast<uint4*>(bpart(which, 1) + off) = p1;
+            *reinterpret_cast<uint4*>(bpart(which, 2) + off) = p2;
         }
         async_proxy_fence();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            const uint32_t vt = smem_u32(sm.VT), kt = smem_u32(sm.KT);
+            // A = V^T and K^T, MN-major: features 64 to a row, tokens one row each
+            // (16 tokens per MMA: 2048 bytes), the second feature half lbo bytes on.
+            constexpr uint32_t kIdescMN = kIdesc | kIdescAmn;
             for (int p = 0; p < 3; ++p)
                 for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem, umma_desc(vt + 256 * ks, kSbo64),
-                              umma_desc(smem_u32(sm.u.Bp[0][p]) + 256 * ks, kSbo64), kIdesc, (p | ks) != 0 ? 1u : 0u);
+                    umma_bf16(tmem, umma_desc_sw128(vt + 2048u * ks, kSwTile, 1024),
+                              umma_desc(smem_u32(bpart(0, p)) + 256 * ks, kSbo64), kIdescMN, (p | ks) != 0 ? 1u : 0u);
             for (int p = 0; p < 3; ++p)
                 for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem + kC, umma_desc(kt + 256 * ks, kSbo64),
-                              umma_desc(smem_u32(sm.u.Bp[1][p]) + 256 * ks, kSbo64), kIdesc, (p | ks) != 0 ? 1u : 0u);
+                    umma_bf16(tmem + kC, umma_desc_sw128(kq + 2048u * ks, 2 * kSwTile, 1024),
+                              umma_desc(smem_u32(bpart(1, p)) + 256 * ks, kSbo64), kIdescMN, (p | ks) != 0 ? 1u : 0u);
             umma_commit(&sm.mma);
         }
         ++issued;
@@ -825,7 +834,7 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
             ++waits;
             tc_fence_after();
             // D_U row j = U^T[j][t] for this warp's 32 tokens -> the record, granule q of row j
-            // at position q ^ (j & 7); D_W row d = W[.][d] -> W staged row-major.
+            // at index q * dv + j; D_W row d = W[.][d] -> W staged row-major.
             const int j = (warp % 4) * 32 + lane;
             float4* ut = reinterpret_cast<float4*>(rec + kR2UT) + j;
 #pragma unroll
@@ -844,6 +853,7 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
     }
     if (!ok && tid == 0) {
         record(a.err, GDN_ERR_TIMEOUT);
+        if (!ld_done) wait_parity(&sm.ld, 0);
         for (; waits < issued; ++waits) wait_parity(&sm.mma, (uint32_t)waits & 1u);
     }
     float* G = reinterpret_cast<float*>(rec + kR2G);
@@ -860,17 +870,19 @@ __global__ void __launch_bounds__(kNT, 2) gdn_chunk_prepare_tc_kernel(ChunkArgs 
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
     if (!ok) return;
 
-    // W in three bf16 parts into the BW tile: W_lo rows 0..63, W_mid 64..127, W_hi 128..191.
+    // W in three bf16 parts into the record's six swizzled tiles: for each feature half,
+    // W_lo, W_mid, W_hi.  Consecutive threads take consecutive granules of a row.
     for (int e = tid; e < kC * (kD / 8); e += kNT) {
-        const int t = (e & 7) | ((e >> 7) << 3), g = (e >> 3) & 15;
+        const int t = e >> 4, g = e & 15;
         const float4 w0 = *reinterpret_cast<const float4*>(&sm.u.W[t][8 * g]);
         const float4 w1 = *reinterpret_cast<const float4*>(&sm.u.W[t][8 * g + 4]);
         const float xw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint4 p0, p1, p2;
         split3x8_fast(xw, p0, p1, p2);
-        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(t, 8 * g, kD)) = p2;
-        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(kC + t, 8 * g, kD)) = p1;
-        *reinterpret_cast<uint4*>(rec + kR2BW + core_off(2 * kC + t, 8 * g, kD)) = p0;
+        unsigned char* wt = rec + kR2W + (size_t)(g >> 3) * 3 * kSwTile + sw128_off(t, g & 7);
+        *reinterpret_cast<uint4*>(wt) = p2;
+        *reinterpret_cast<uint4*>(wt + kSwTile) = p1;
+        *reinterpret_cast<uint4*>(wt + 2 * kSwTile) = p0;
     }
 }
 
@@ -1087,18 +1099,19 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 // stored while the next chunk's first products run (a separate issuing warp would
 // cost registers: a 17-warp CTA is allocated as 20 warps).
 // Per chunk, with S split into three bf16 parts (S = S_hi + S_mid + S_lo) as the A
-// operand (M = 128 value rows, K = dk) and the record's tile [W_lo | W_mid | W_hi | Q]
-// as B (N = 64 tokens per part):
+// operand (M = 128 value rows, K = dk) and [W_lo | W_mid | W_hi | Q] as B (N = 64 tokens
+// per part; the record's W parts and the chunk's Q tiles, all 128-byte swizzled):
 //   G   = S_hi [W_lo W_mid W_hi Q] + S_mid [W_mid W_hi Q] + S_lo [W_hi]   (TMEM cols 0..255)
 //   E^T = U^T - (G0 + G1 + G2) = (U - W M)^T,    QM^T = G3 (q M per token), scaled by g_t
 // (the part products left out are below 2^-24 of W M, and 2^-16 of Q M, an output-only
 // term).  Then with E' = diag(g_C / g) E split in three parts and E in two as A operands
 // (K = 64 tokens):
-//   D_U = E'^T K              (B = K^T tile; cols 256..383)   ->  S <- g_C S + D_U
+//   D_U = E'^T K              (B = the K tiles, MN-major; cols 256..383) ->  S <- g_C S + D_U
 //   D_O = E_hi [P_mid P_hi] + E_mid [P_hi]   (cols 384..511)  ->  o = g Q M + P E
 // The state update is committed first; the chain waits only for it.  The issuing
-// thread streams the three record images with cp.async.bulk: each buffer is refilled
-// for the next chunk as soon as its last reader is done.  Every wait is bounded (2 s);
+// thread streams three shared-memory images, record fields by cp.async.bulk and the
+// chunk's Q and K tiles by tensor copies: each buffer is refilled for the next chunk as
+// soon as its last reader is done.  Every wait is bounded (2 s);
 // a timeout is recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kSPart = (uint32_t)kD * kD * 2;  // one bf16 part of S (128 x 128)
@@ -1111,14 +1124,16 @@ constexpr int kIssuer = 0;                          // the thread that also issu
 
 struct SmemS {
     unsigned char aop[3 * kSPart];  // A operands: S parts; then E'^T parts (3) and E^T parts (hi, mid)
-    unsigned char imgA[kImgA];      // [W_lo | W_mid | W_hi | Q]
-    unsigned char imgB[kImgB];      // K^T | [P_mid | P_hi]
+    unsigned char imgA[kImgA];      // [W_lo W_mid W_hi Q] for features 0..63, then 64..127
+    unsigned char imgB[kImgB];      // [K lo | K hi] | [P_mid | P_hi]
     unsigned char imgC[kImgC];      // g_t, g_C / g_t, g_C | U^T
     uint64_t bar_a, bar_b, bar_c, mma_g, mma_u, mma_o;
     uint32_t tmem;
     int src, dst, status;
 };
-static_assert(sizeof(SmemS) <= 227 * 1024, "scan shared memory plan exceeds the per-CTA limit");
+constexpr int kSmemS = (int)sizeof(SmemS) + 1024;  // + alignment slack
+static_assert(kSmemS <= 227 * 1024, "scan shared memory plan exceeds the per-CTA limit");
+static_assert(3 * kSPart % 1024 == 0 && kImgA % 1024 == 0, "swizzled images start on 1024-byte boundaries");
 static_assert(3 * kEPart + 2 * kEPart <= 3 * kSPart, "E parts overlay the S parts");
 
 // 8 consecutive TMEM columns of this warp's 32 lanes (completion awaited separately).
@@ -1131,9 +1146,10 @@ __device__ __forceinline__ void tie_regs8(uint32_t (&r)[8]) {
     asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
 }
 
-__global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(ChunkArgs a) {
+__global__ void __launch_bounds__(kScanThreads, 1)
+    gdn_chunk_scan_tc_kernel(ChunkArgs a, const __grid_constant__ TileMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem_tc[];
-    SmemS& sm = *reinterpret_cast<SmemS*>(smem_tc);
+    SmemS& sm = *reinterpret_cast<SmemS*>(align1024(smem_tc));
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
     constexpr bool compute = true;
@@ -1141,18 +1157,25 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(Chun
     const int bh = blockIdx.x;
     const int h = bh % a.Hv;
     const int b = bh / a.Hv;
+    const int hk = h / a.G;
     const int quarter = (warp / 4) & 3;            // key columns 32*quarter.., tokens 16*quarter..
     const int j = (warp % 4) * 32 + lane;          // value row = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const int nch = a.nchunks;
 
     auto issue_a = [&](int c) {
+        const unsigned char* w = record_of(a, bh, c) + kR2W;
         mbar_expect_tx(&sm.bar_a, kImgA);
-        bulk_g2s(sm.imgA, record_of(a, bh, c) + kR2BW, kImgA, &sm.bar_a);
+        bulk_g2s(sm.imgA, w, 3 * kSwTile, &sm.bar_a);
+        bulk_g2s(sm.imgA + 4 * kSwTile, w + 3 * kSwTile, 3 * kSwTile, &sm.bar_a);
+        tma_tile(sm.imgA + 3 * kSwTile, &maps.q, 0, hk, c * kC, b, &sm.bar_a);
+        tma_tile(sm.imgA + 7 * kSwTile, &maps.q, 64, hk, c * kC, b, &sm.bar_a);
     };
     auto issue_b = [&](int c) {
         mbar_expect_tx(&sm.bar_b, kImgB);
-        bulk_g2s(sm.imgB, record_of(a, bh, c) + kR2BK, kImgB, &sm.bar_b);
+        tma_tile(sm.imgB, &maps.k, 0, hk, c * kC, b, &sm.bar_b);
+        tma_tile(sm.imgB + kSwTile, &maps.k, 64, hk, c * kC, b, &sm.bar_b);
+        bulk_g2s(sm.imgB + 2 * kSwTile, record_of(a, bh, c) + kR2P, kR2PBytes, &sm.bar_b);
     };
     auto issue_c = [&](int c) {
         mbar_expect_tx(&sm.bar_c, kImgC);
@@ -1261,28 +1284,31 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(Chun
         // The chunk's first products, issued by thread 0 in three batches (one per S
         // part) with its warp's share of the previous chunk's outputs stored in between;
         // the other warps store theirs while the products run.
+        // B: K-steps of 16 features 32 bytes apart within a tile, the second feature half
+        // four tiles on; each batch starts one tile (64 token rows) further in.
         const uint32_t aS = smem_u32(sm.aop), bW = smem_u32(sm.imgA);
         constexpr uint32_t kSboG = (kD / 8) * 128;
+        auto bdesc = [&](int part, int ks) {
+            return umma_desc_sw128(bW + part * kSwTile + (ks < 4 ? 32u * ks : 4 * kSwTile + 32u * (ks - 4)), 16, 1024);
+        };
         if (warp == 0) {
             if (issuer) {
                 ++done_a;
                 for (int ks = 0; ks < kD / 16; ++ks)
-                    umma_bf16(tmem, umma_desc(aS + 256 * ks, kSboG), umma_desc(bW + 256 * ks, kSboG), kIdesc256,
-                              ks != 0 ? 1u : 0u);
+                    umma_bf16(tmem, umma_desc(aS + 256 * ks, kSboG), bdesc(0, ks), kIdesc256, ks != 0 ? 1u : 0u);
             }
             __syncwarp();
             if (c > 0) store_outputs(0);
             if (issuer) {
                 for (int ks = 0; ks < kD / 16; ++ks)
-                    umma_bf16(tmem + kC, umma_desc(aS + kSPart + 256 * ks, kSboG),
-                              umma_desc(bW + (kC / 8) * kSboG + 256 * ks, kSboG), kIdesc192, 1u);
+                    umma_bf16(tmem + kC, umma_desc(aS + kSPart + 256 * ks, kSboG), bdesc(1, ks), kIdesc192, 1u);
             }
             __syncwarp();
             if (c > 0) store_outputs(1);
             if (issuer) {
                 for (int ks = 0; ks < kD / 16; ++ks)
-                    umma_bf16(tmem + 2 * kC, umma_desc(aS + 2 * kSPart + 256 * ks, kSboG),
-                              umma_desc(bW + (2 * kC / 8) * kSboG + 256 * ks, kSboG), kIdesc64, 1u);
+                    umma_bf16(tmem + 2 * kC, umma_desc(aS + 2 * kSPart + 256 * ks, kSboG), bdesc(2, ks), kIdesc64,
+                              1u);
                 umma_commit(&sm.mma_g);
                 ++issued_g;
             }
@@ -1370,12 +1396,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_chunk_scan_tc_kernel(Chun
                 issue_c(c + 1);
                 ++issued_c;
             }
-            const uint32_t aE = smem_u32(sm.aop), bK = smem_u32(sm.imgB), bP = bK + kR2BKBytes;
+            // B = K, MN-major: features 64 to a row, tokens one row each (16 tokens per
+            // MMA: 2048 bytes), the second feature half one tile on.
+            const uint32_t aE = smem_u32(sm.aop), bK = smem_u32(sm.imgB), bP = bK + 2 * kSwTile;
             constexpr uint32_t kSbo = (kC / 8) * 128;
             for (int part = 0; part < 3; ++part)
                 for (int ks = 0; ks < kC / 16; ++ks)
                     umma_bf16(tmem + kTmemDU, umma_desc(aE + part * kEPart + 256 * ks, kSbo),
-                              umma_desc(bK + 256 * ks, kSbo), kIdesc128, (part | ks) != 0 ? 1u : 0u);
+                              umma_desc_sw128(bK + 2048u * ks, kSwTile, 1024), kIdesc128 | kIdescBmn,
+                              (part | ks) != 0 ? 1u : 0u);
             umma_commit(&sm.mma_u);
             for (int ks = 0; ks < kC / 16; ++ks)
                 umma_bf16(tmem + kTmemDO, umma_desc(aE + 3 * kEPart + 256 * ks, kSbo), umma_desc(bP + 256 * ks, kSbo),
@@ -1470,6 +1499,43 @@ extern "C" gdn_status gdn_wait_selftest(uint64_t limit_ns, int32_t* err_word, cu
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// The driver's tensor-map encoder, looked up once through the runtime (no link to the
+// driver library); null if the driver does not export it.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn tensor_map_encoder() {
+    static const EncodeTiledFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+// Tensor maps of k, q ([B][L][Hk][dk]) and v ([B][L][Hv][dv]), bf16: dims {feature, head,
+// token, request}, box 64 x 1 x 64 x 1, 128-byte swizzle, zero fill past L.  The
+// addresses are 16-byte aligned and every stride a multiple of 256 bytes (checked by
+// the caller), which is what the encoder asks for.
+static gdn_status encode_tile_maps(TileMaps& m, const ChunkArgs& a) {
+    const EncodeTiledFn enc = tensor_map_encoder();
+    if (enc == nullptr) return GDN_ERR_CUDA;
+    auto one = [&](CUtensorMap* map, const void* base, int H) {
+        const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)a.L, (cuuint64_t)a.B};
+        const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)a.L * H * kD * 2};
+        const cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+        const cuuint32_t step[4] = {1, 1, 1, 1};
+        return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, step,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!one(&m.k, a.k, a.Hk) || !one(&m.q, a.q, a.Hk) || !one(&m.v, a.v, a.Hv)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
 extern "C" size_t gdn_prefill_workspace_bytes(int32_t B, int32_t L, int32_t Hv, int32_t dk, int32_t dv) {
     if (B < 0 || L < 1 || Hv < 1 || dk != kD || dv != kD) return 0;
     const size_t nchunks = ((size_t)L + kC - 1) / kC;
@@ -1502,12 +1568,17 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     const ChunkArgs a{pool, src_idx, dst_idx, q, k, v, alpha, beta, out, static_cast<unsigned char*>(workspace),
                       err_word, num_slots, B, L, Hk, Hv, Hv / Hk, nchunks};
     const bool bf = qkv_dtype == GDN_BF16;
-    const int s1 = bf ? (int)sizeof(SmemP) : (int)sizeof(Smem1), s2 = bf ? (int)sizeof(SmemS) : (int)sizeof(Smem2);
+    const int s1 = bf ? kSmemP : (int)sizeof(Smem1), s2 = bf ? kSmemS : (int)sizeof(Smem2);
+    TileMaps maps;
+    if (bf) {
+        const gdn_status st = encode_tile_maps(maps, a);
+        if (st != GDN_OK) return st;
+    }
     cudaError_t e = bf ? cudaFuncSetAttribute(gdn_chunk_prepare_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1)
                        : cudaFuncSetAttribute(gdn_chunk_prepare_kernel<float>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    if (bf) {  // three prepare CTAs per SM need the largest shared-memory carveout
+    if (bf) {  // two prepare CTAs per SM need the largest shared-memory carveout
         e = cudaFuncSetAttribute(gdn_chunk_prepare_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return GDN_ERR_CUDA;
@@ -1517,7 +1588,7 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     const unsigned g1 = (unsigned)(B * Hv * nchunks);
     if (bf) {
-        gdn_chunk_prepare_tc_kernel<<<g1, kNT, s1, stream>>>(a);
+        gdn_chunk_prepare_tc_kernel<<<g1, kNT, s1, stream>>>(a, maps);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
         // The scan starts behind the prepare kernel with programmatic dependent launch.
         cudaLaunchConfig_t cfg = {};
@@ -1530,7 +1601,7 @@ extern "C" gdn_status gdn_prefill_chunked(float* pool, int32_t num_slots, const 
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, gdn_chunk_scan_tc_kernel, a) != cudaSuccess) return GDN_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, gdn_chunk_scan_tc_kernel, a, maps) != cudaSuccess) return GDN_ERR_CUDA;
     } else {
         const unsigned g2 = (unsigned)(B * Hv * kNCB);
         gdn_chunk_prepare_kernel<float><<<g1, kNT, s1, stream>>>(a);
