@@ -152,6 +152,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------------------
 // tcgen05 / bulk-copy helpers (sm_100a PTX).
 // ---------------------------------------------------------------------------
+// 2^x by the ex2.approx.ftz instruction (PTX ISA: relative error about 2^-22, subnormal
+// results flushed to zero), for the 8192 gate ratios g_t / g_i <= 1 of a chunk.  A ratio
+// below 2^-126 multiplies a dot product of unit-norm vectors, so flushing it is below fp32
+// precision of the sums it enters.
+__device__ __forceinline__ float ex2a(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -746,11 +755,17 @@ __global__ void __launch_bounds__(kNT, 2)
         tc_fence_after();
         // D0 row r < 64: k_r . k_i -> A (scaled); row 64 + t: q_t . k_i -> P (record).
         const int r = (warp % 4) * 32 + lane;
+        uint32_t d0r[2][16];  // both halves of this thread's D0 row, one completion wait
+        tmem_ld16_issue(tmem + lane_base + (uint32_t)(32 * half), d0r[0]);
+        tmem_ld16_issue(tmem + lane_base + (uint32_t)(32 * half + 16), d0r[1]);
+        tmem_wait_ld();
+        tie_regs(d0r[0]), tie_regs(d0r[1]);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
             float v[16];
             const int i0 = 32 * half + 16 * part;
-            tmem_ld16(tmem + lane_base + (uint32_t)i0, v);
+#pragma unroll
+            for (int m = 0; m < 16; ++m) v[m] = __uint_as_float(d0r[part][m]);
             if (r < kC) {
                 const float lt = sm.lg[r], bt = sm.bt[r];
 #pragma unroll
@@ -759,7 +774,7 @@ __global__ void __launch_bounds__(kNT, 2)
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         const int i = i0 + j + m;
-                        x[m] = i < r ? bt * exp2f(lt - sm.lg[i]) * v[j + m] : 0.f;
+                        x[m] = i < r ? bt * ex2a(lt - sm.lg[i]) * v[j + m] : 0.f;
                     }
                     *reinterpret_cast<float4*>(&sm.u.ra.A[r][i0 + j]) = make_float4(x[0], x[1], x[2], x[3]);
                 }
@@ -773,7 +788,7 @@ __global__ void __launch_bounds__(kNT, 2)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int i = i0 + g8 + j;
-                        x[j] = i <= t ? exp2f(lt - sm.lg[i]) * v[g8 + j] : 0.f;
+                        x[j] = i <= t ? ex2a(lt - sm.lg[i]) * v[g8 + j] : 0.f;
                     }
                     uint4 p0, p1;
                     split2x8_fast(x, p0, p1);
