@@ -197,8 +197,10 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     constexpr int kRowStep = RG * (DV / 4);
     const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV)) + toff;
     float4 s[RPT];
+    // Default L2 priority, not evict-first: a prefix checkpoint shared by several requests
+    // then stays in L2 for its other readers (the stores below are the streaming ones).
 #pragma unroll
-    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+    for (int m = 0; m < RPT; ++m) s[m] = __ldg(S + m * kRowStep);
     allow_dependent_launch();
 
     const size_t gh = (size_t)b * a.Hv + h;  // token index = b for a single token
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV)) + toff;
     float4 s[RPT];
 #pragma unroll
-    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+    for (int m = 0; m < RPT; ++m) s[m] = __ldg(S + m * kRowStep);  // default L2 priority (see gdn_tile1_kernel)
     allow_dependent_launch();
 
     const int hk = h / a.G;
@@ -589,7 +591,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tileT_kernel(StepArgs a) {
     const float4* S = reinterpret_cast<const float4*>(a.pool + ((size_t)src * a.Hv + h) * (DK * DV)) + toff;
     float4 s[RPT];
 #pragma unroll
-    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(S + m * kRowStep);
+    for (int m = 0; m < RPT; ++m) s[m] = __ldg(S + m * kRowStep);  // default L2 priority (see gdn_tile1_kernel)
     allow_dependent_launch();
 
     const int hk = h / a.G;
