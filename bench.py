@@ -599,6 +599,10 @@ def measure_workload(name: str, calls: int = 200, warmup: int = 10, variant: str
         call()
     torch.cuda.synchronize()
     warm_us = _time_calls(call, calls, stream, graph=False)
+    # The same call through the prepared form (buffers checked once, stream bound).
+    prepared = gdn.PreparedDecodeStep(pool, x["src_idx"], dst, x["q"], x["k"], x["v"], x["alpha"], x["beta"], out,
+                                      err_word=err, variant=None if variant == "auto" else variant, stream=stream)
+    prepared_us = _time_calls(prepared, calls, stream, graph=False)
     graph_us = _time_calls(call, calls, stream, graph=True) if graph_too else None
     cold_us = _time_cold(call, min(calls, cold_reps), stream)
     cold_clean_us = _time_cold(call, min(calls, cold_reps), stream, clean=True)
@@ -628,7 +632,8 @@ def measure_workload(name: str, calls: int = 200, warmup: int = 10, variant: str
         "config": {"B": s.B, "T": s.T, "Hk": s.Hk, "Hv": s.Hv, "dk": s.dk, "dv": s.dv, "slots": w.num_slots,
                    "qkv": s.dtype, "state": "f32"},
         "units_per_call": nb["units"], "calls": calls,
-        "us_per_call_warm": warm_us, "us_per_call_graph": graph_us, "us_per_call_cold": cold_us,
+        "us_per_call_warm": warm_us, "us_per_call_prepared": prepared_us, "us_per_call_graph": graph_us,
+        "us_per_call_cold": cold_us,
         "us_per_call_cold_clean_l2": cold_clean_us,
         "value_warm": nb["units"] / (best_warm / 1e6), "value_cold": nb["units"] / (cold_us / 1e6), "unit": UNIT,
         "bytes_per_call_nominal": nb["nominal"], "bytes_per_call_min": nb["minimum"],

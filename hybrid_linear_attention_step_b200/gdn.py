@@ -157,6 +157,46 @@ def gdn_decode_step(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Te
     return status
 
 
+class PreparedDecodeStep:
+    """gdn_decode_step on buffers checked once: for a serving loop that reuses the same
+    tensors every step (as a CUDA graph does), each call then only passes the pointers.
+
+    The tensors must stay alive and keep their storage while the object is used; their
+    contents may change between calls (new inputs, indices, gates).  ``variant`` is None for
+    gdn_decode_step or a GDN_VARIANT_* value or name for gdn_decode_step_variant.  A
+    ``stream`` given here is used by every call that names none (looking up torch's current
+    stream costs about as much host time as the launch); without one, each call enqueues on
+    the current stream, which is what stream capture into a CUDA graph needs.
+    """
+
+    def __init__(self, pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
+                 q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
+                 err_word: Optional[torch.Tensor] = None, variant=None, stream=None):
+        lib = load_library()
+        args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out) + (_ptr_or_null(err_word, "err_word"),)
+        if variant is None:
+            self._fn, self._name = lib.gdn_decode_step, "gdn_decode_step"
+        else:
+            if isinstance(variant, str):
+                variant = VARIANTS[variant]
+            self._fn, self._name = lib.gdn_decode_step_variant, "gdn_decode_step_variant"
+            args = args + (int(variant),)
+        self._args = args
+        self._stream = None if stream is None else _stream_handle(stream)
+        self._keep = (pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word, stream)
+
+    def __call__(self, stream=None, check: bool = True) -> int:
+        if stream is None and self._stream is not None:
+            handle = self._stream
+        else:
+            handle = _stream_handle(stream)
+        status = self._fn(*self._args, handle)
+        if check and status != GDN_OK:
+            raise GdnError(status, self._name)
+        return status
+
+
 def gdn_decode_step_variant(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
                             q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                             alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor, variant,

@@ -181,3 +181,23 @@ def test_stream_variant_requires_the_error_word(lib):
     args = [16, 8, 16, 16, 16, 16, 16, 16, 16, 16, 4, 1, 1, 1, 128, 128, 1]
     assert f(*args, None, 1, None) == 1      # GDN_VARIANT_STREAM, no error word
     assert f(*args, None, 9, None) == 1      # no such variant
+
+
+def test_prepared_decode_step_checks_its_buffers_once():
+    """The prepared decode call validates shapes and devices when it is made (no GPU needed:
+    the checks come before any call into the library)."""
+    import torch
+
+    from hybrid_linear_attention_step_b200 import gdn
+
+    B, T, Hk, Hv, d = 2, 1, 1, 2, 128
+    pool = torch.zeros((4, Hv, d, d))
+    q = torch.zeros((B, T, Hk, d), dtype=torch.bfloat16)
+    v = torch.zeros((B, T, Hv, d), dtype=torch.bfloat16)
+    gates = torch.zeros((B, T, Hv))
+    idx = torch.zeros(B, dtype=torch.int32)
+    out = torch.zeros((B, T, Hv, d))
+    with pytest.raises(ValueError):
+        gdn.PreparedDecodeStep(pool, idx, idx, q, q, v, gates, gates, torch.zeros((B, T, Hv, d + 1)))
+    with pytest.raises(TypeError):
+        gdn.PreparedDecodeStep(pool, idx, idx, q, q, v, gates, gates, out)  # host tensors

@@ -740,3 +740,51 @@ def test_bounded_wait_runs_out_and_reports_timeout(torch_cuda):
     assert gdn.gdn_get_error(err) == gdn.GDN_OK
     check_pool(dev.cpu().numpy(), ref_pool, w.pool, w.steps[0].dst_idx)
     assert rel_err(out, ref_out) <= TOL_OUT_BF16
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_prepared_decode_step_equals_the_checked_call(torch_cuda, T):
+    """The prepared form (buffers checked once, stream bound or not) enqueues the same call:
+    bit for bit the checked call's results, and the oracle's; its buffers' contents change
+    between calls (new inputs and slot tables) while their storage stays."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(300 + T)
+    B, Hk, Hv, d = 6, 2, 4, 128
+    num_slots = B * (T + 1) + 2
+    pool_np = wl.init_pool(rng, num_slots, Hv, d, d)
+    dev_a, dev_b = to_torch(pool_np), to_torch(pool_np)
+    q, k, v, a, b = (to_torch(x) for x in wl.random_step_inputs(rng, B, T, Hk, Hv, d, d, wl.BF16))
+    src = torch.zeros(B, dtype=torch.int32, device="cuda")
+    dst = torch.zeros((B, T), dtype=torch.int32, device="cuda")
+    out_a = torch.zeros((B, T, Hv, d), device="cuda")
+    out_b = torch.zeros((B, T, Hv, d), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bound = gdn.PreparedDecodeStep(dev_b, src, dst, q, k, v, a, b, out_b, err_word=err,
+                                   stream=torch.cuda.current_stream())
+    unbound = gdn.PreparedDecodeStep(dev_b, src, dst, q, k, v, a, b, out_b, err_word=err)
+    ref = pool_np.copy()
+    for it, call in enumerate((bound, unbound, bound)):
+        perm = rng.permutation(num_slots).astype(np.int32)
+        src_np = perm[:B].copy()
+        dst_np = (src_np.reshape(B, 1).copy() if T == 1 else perm[B:B + B * T].reshape(B, T).copy())
+        src.copy_(torch.from_numpy(src_np))
+        dst.copy_(torch.from_numpy(dst_np))
+        hq, hk_, hv, ha, hb = wl.random_step_inputs(rng, B, T, Hk, Hv, d, d, wl.BF16)
+        for t_dev, x in ((q, hq), (k, hk_), (v, hv), (a, ha), (b, hb)):
+            t_dev.copy_(to_torch(x))
+        gdn.gdn_decode_step(dev_a, src, dst, q, k, v, a, b, out_a, err_word=err)
+        call()
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_error(err) == gdn.GDN_OK
+        got_a, got_b = dev_a.cpu().numpy(), dev_b.cpu().numpy()
+        assert np.array_equal(got_a.view(np.uint32), got_b.view(np.uint32)), it
+        assert np.array_equal(out_a.cpu().numpy().view(np.uint32), out_b.cpu().numpy().view(np.uint32)), it
+        s = wl.Step(hq, hk_, hv, ha, hb, src_np, dst_np)
+        before = ref.copy()
+        ref, ref_out, skipped = run_oracle(ref, s)
+        assert skipped == 0
+        check_pool(got_b, ref, before, dst_np)
+        assert rel_err(out_b.cpu().numpy(), ref_out) <= TOL_OUT_BF16
+        ref = got_b.copy()  # carry the device state on, so that each call is checked alone
