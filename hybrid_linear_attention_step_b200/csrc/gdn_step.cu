@@ -52,9 +52,18 @@ struct StepArgs {
     float* out;
     int32_t* err;
     int num_slots, B, T, Hk, Hv, dk, dv, G;
-    int flags;    // GDN_FUSE_* bits (gdn_decode_step_fused); 0 for plain calls
+    int flags;    // GDN_FUSE_* and GDN_SHARED_SOURCES bits (gdn_decode_step_fused); 0 for plain calls
     int prefill;  // 1 (gdn_prefill): dst_idx is [B], only the state after the last token is stored
 };
+
+// The flags that change the arithmetic (and pick the fused kernels).
+constexpr int kFuseFlags = GDN_FUSE_GATES | GDN_FUSE_QK_NORM;
+
+// unit_order: the register-tile kernels number their CTAs (request, head, column block)
+// request-major, so that consecutive CTAs walk one slot's contiguous 2 MiB (the faster
+// order when every request has a state of its own).  With GDN_SHARED_SOURCES they go
+// head-major: every request of one value head within a fraction of a wave, so that a
+// source tile that several requests share is read from HBM once and then from L2.
 
 // Fused prologue (gdn_decode_step_fused).  alpha = exp(-softplus(x)) equals
 // 1 / (1 + e^x) exactly, and beta = sigmoid(y) = 1 / (1 + e^-y); both limits
@@ -177,8 +186,9 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile1_kernel(StepArgs a) {
     const int rg = tid / CG;
     const int chunk = blockIdx.x % NC;
     const int unit = blockIdx.x / NC;
-    const int h = unit % a.Hv;
-    const int b = unit / a.Hv;
+    const bool by_head = (a.flags & GDN_SHARED_SOURCES) != 0;  // see unit_order
+    const int h = by_head ? unit / a.B : unit % a.Hv;
+    const int b = by_head ? unit % a.B : unit / a.Hv;
 
     // With programmatic dependent launch this grid may start while the previous
     // kernel in the stream is finishing: wait for it before touching memory.
@@ -358,8 +368,9 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     const int rg = tid / CG;
     const int chunk = blockIdx.x % NC;
     const int unit = blockIdx.x / NC;
-    const int h = unit % a.Hv;
-    const int b = unit / a.Hv;
+    const bool by_head = (a.flags & GDN_SHARED_SOURCES) != 0;  // see unit_order
+    const int h = by_head ? unit / a.B : unit % a.Hv;
+    const int b = by_head ? unit % a.B : unit / a.Hv;
     const int T = MULTI ? a.T : 1;
 
     grid_dependency_wait();  // launched with programmatic dependent launch, as gdn_tile1_kernel
@@ -574,8 +585,9 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tileT_kernel(StepArgs a) {
     const int rg = tid / CG;
     const int chunk = blockIdx.x % NC;
     const int unit = blockIdx.x / NC;
-    const int h = unit % a.Hv;
-    const int b = unit / a.Hv;
+    const bool by_head = (a.flags & GDN_SHARED_SOURCES) != 0;  // see unit_order
+    const int h = by_head ? unit / a.B : unit % a.Hv;
+    const int b = by_head ? unit % a.B : unit / a.Hv;
     const int T = a.T;
 
     grid_dependency_wait();
@@ -1169,7 +1181,8 @@ gdn_status launch_tile_impl(const StepArgs& a, int32_t dtype, cudaStream_t strea
 
 template <int DK, int DV>
 gdn_status launch_tile(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
-    return a.flags ? launch_tile_impl<DK, DV, true>(a, dtype, stream) : launch_tile_impl<DK, DV, false>(a, dtype, stream);
+    return (a.flags & kFuseFlags) ? launch_tile_impl<DK, DV, true>(a, dtype, stream)
+                                  : launch_tile_impl<DK, DV, false>(a, dtype, stream);
 }
 
 gdn_status launch_column(const StepArgs& a, int32_t dtype, cudaStream_t stream) {
@@ -1221,7 +1234,7 @@ gdn_status launch_stream(const StepArgs& a, cudaStream_t stream) {
 // a compiled tile shape and 16-byte aligned pool/out; the column kernel takes
 // anything.
 bool stream_ok(const StepArgs& a) {
-    return a.flags == 0 && a.T == 1 && a.dk == 128 && a.dv == 128 && ((int64_t)a.B * a.Hv) % 4 == 0 && aligned16(a.pool) &&
+    return (a.flags & kFuseFlags) == 0 && a.T == 1 && a.dk == 128 && a.dv == 128 && ((int64_t)a.B * a.Hv) % 4 == 0 && aligned16(a.pool) &&
            aligned16(a.out) && aligned16(a.q) && aligned16(a.k) && aligned16(a.v) && aligned16(a.alpha) &&
            aligned16(a.beta);
 }
@@ -1290,7 +1303,7 @@ extern "C" gdn_status gdn_decode_step_fused(float* pool, int32_t num_slots, cons
     if (B < 0 || T < 1 || Hk < 1 || Hv < 1 || dk < 1 || dv < 1 || num_slots < 1) return GDN_ERR_INVALID_ARG;
     if (Hv % Hk != 0 || dk > kMaxDk) return GDN_ERR_INVALID_ARG;
     if (qkv_dtype != GDN_F32 && qkv_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
-    if ((flags & ~(GDN_FUSE_GATES | GDN_FUSE_QK_NORM)) != 0) return GDN_ERR_INVALID_ARG;
+    if ((flags & ~(kFuseFlags | GDN_SHARED_SOURCES)) != 0) return GDN_ERR_INVALID_ARG;
     if ((int64_t)B * Hv * 4 >= (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;
     if (B == 0) return GDN_OK;
     if (!pool || !src_idx || !dst_idx || !q || !k || !v || !alpha_or_x || !beta_or_y || !out)

@@ -26,6 +26,7 @@ GDN_SLOT_NONE = -1
 
 GDN_FUSE_GATES = 1
 GDN_FUSE_QK_NORM = 2
+GDN_SHARED_SOURCES = 4  # scheduling hint: many requests share source slots (same results)
 
 GDN_F32 = 0
 GDN_BF16 = 1
@@ -162,26 +163,35 @@ class PreparedDecodeStep:
     tensors every step (as a CUDA graph does), each call then only passes the pointers.
 
     The tensors must stay alive and keep their storage while the object is used; their
-    contents may change between calls (new inputs, indices, gates).  ``variant`` is None for
-    gdn_decode_step or a GDN_VARIANT_* value or name for gdn_decode_step_variant.  A
-    ``stream`` given here is used by every call that names none (looking up torch's current
-    stream costs about as much host time as the launch); without one, each call enqueues on
-    the current stream, which is what stream capture into a CUDA graph needs.
+    contents may change between calls (new inputs, indices, gates).  ``variant`` is None
+    for the automatic kernel choice or a GDN_VARIANT_* value or name (then the call is
+    gdn_decode_step_variant); nonzero ``flags`` (GDN_FUSE_*, GDN_SHARED_SOURCES) make it
+    gdn_decode_step_fused, with the automatic choice.  A ``stream`` given here is used by
+    every call that names none (looking up torch's current stream costs about as much host
+    time as the launch); without one, each call enqueues on the current stream, which is
+    what stream capture into a CUDA graph needs.
     """
 
     def __init__(self, pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
                  q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
-                 err_word: Optional[torch.Tensor] = None, variant=None, stream=None):
+                 err_word: Optional[torch.Tensor] = None, variant=None, stream=None, flags: int = 0):
         lib = load_library()
-        args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out) + (_ptr_or_null(err_word, "err_word"),)
-        if variant is None:
+        args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+        err = _ptr_or_null(err_word, "err_word")
+        if flags and variant is not None:
+            raise ValueError("flags go with the automatic kernel choice: pass variant=None")
+        if flags:
+            self._fn, self._name = lib.gdn_decode_step_fused, "gdn_decode_step_fused"
+            args = args + (int(flags), err)
+        elif variant is None:
             self._fn, self._name = lib.gdn_decode_step, "gdn_decode_step"
+            args = args + (err,)
         else:
             if isinstance(variant, str):
                 variant = VARIANTS[variant]
             self._fn, self._name = lib.gdn_decode_step_variant, "gdn_decode_step_variant"
-            args = args + (int(variant),)
+            args = args + (err, int(variant))
         self._args = args
         self._stream = None if stream is None else _stream_handle(stream)
         self._keep = (pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word, stream)
@@ -219,7 +229,8 @@ def gdn_decode_step_fused(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: to
                           err_word: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> int:
     """gdn_decode_step with the input prologue folded in (see gdn_decode_step_fused in
     include/gdn_step.h): GDN_FUSE_GATES makes alpha_or_x / beta_or_y the raw x, y;
-    GDN_FUSE_QK_NORM L2-normalises q and k inside the kernel."""
+    GDN_FUSE_QK_NORM L2-normalises q and k inside the kernel; GDN_SHARED_SOURCES tells the
+    kernels that many requests share source slots (an ordering hint, same results)."""
     args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha_or_x, beta_or_y, out)
     status = load_library().gdn_decode_step_fused(*args, int(flags), _ptr_or_null(err_word, "err_word"),
                                                   _stream_handle(stream))

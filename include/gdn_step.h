@@ -158,6 +158,7 @@ gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t
 /* Flags of gdn_decode_step_fused. */
 #define GDN_FUSE_GATES 1   /* alpha/beta arguments are raw x, y: alpha = exp(-softplus(x)), beta = sigmoid(y) */
 #define GDN_FUSE_QK_NORM 2 /* q and k are L2-normalised per (token, key head): x / sqrt(sum x^2 + 1e-6) */
+#define GDN_SHARED_SOURCES 4 /* scheduling hint, no arithmetic: many requests share source slots */
 
 /*
  * gdn_decode_step_fused -- gdn_decode_step with its input prologue folded in.
@@ -172,6 +173,15 @@ gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t
  *                             if it has one, is applied by the caller.
  *   flags & GDN_FUSE_QK_NORM: q and k are used as q / sqrt(|q|^2 + 1e-6) and
  *                             k / sqrt(|k|^2 + 1e-6), per (token, key head).
+ *   flags & GDN_SHARED_SOURCES: a hint that many of the batch's requests share
+ *                             source slots (prefix-checkpoint hits; a caller that
+ *                             plans with gdn_slot_cache_plan sees it as repeated
+ *                             src entries).  The register-tile kernels then visit
+ *                             every request of one value head before the next
+ *                             head, so a shared tile is read from HBM once and then
+ *                             from L2.  The result is bit for bit the same with or
+ *                             without it; without sharing it only costs bandwidth
+ *                             (request-major order keeps each slot's 2 MiB together).
  * Without flags the call is gdn_decode_step.  Same layouts, preconditions, errors
  * and bytes moved as gdn_decode_step; unknown flag bits return GDN_ERR_INVALID_ARG.
  * Served by the register-tile kernels (column kernel for other shapes/alignments).

@@ -201,3 +201,17 @@ def test_prepared_decode_step_checks_its_buffers_once():
         gdn.PreparedDecodeStep(pool, idx, idx, q, q, v, gates, gates, torch.zeros((B, T, Hv, d + 1)))
     with pytest.raises(TypeError):
         gdn.PreparedDecodeStep(pool, idx, idx, q, q, v, gates, gates, out)  # host tensors
+
+
+def test_fused_flags_are_checked_on_the_host(lib):
+    """gdn_decode_step_fused accepts GDN_FUSE_GATES, GDN_FUSE_QK_NORM and the
+    GDN_SHARED_SOURCES hint, and refuses any other bit before doing anything."""
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    f = lib.gdn_decode_step_fused
+    f.restype = i32
+    f.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    args = [16, 8, 16, 16, 16, 16, 16, 16, 16, 16, 0, 1, 1, 1, 128, 128, 1]  # B = 0: a no-op when valid
+    for flags in (0, 1, 2, 3, 4, 5, 7):
+        assert f(*args, flags, None, None) == 0, flags
+    for flags in (8, 16, 12, -1):
+        assert f(*args, flags, None, None) == 1, flags

@@ -526,7 +526,7 @@ def test_fused_without_flags_equals_plain_bitwise(torch_cuda):
         pools.append(dev.cpu().numpy())
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(pools[0].view(np.uint32), pools[1].view(np.uint32))
     with pytest.raises(gdn.GdnError):
-        gdn.gdn_decode_step_fused(*args, 4)
+        gdn.gdn_decode_step_fused(*args, 8)  # no such flag
 
 
 PREFILL_SHAPES = [
@@ -788,3 +788,44 @@ def test_prepared_decode_step_equals_the_checked_call(torch_cuda, T):
         check_pool(got_b, ref, before, dst_np)
         assert rel_err(out_b.cpu().numpy(), ref_out) <= TOL_OUT_BF16
         ref = got_b.copy()  # carry the device state on, so that each call is checked alone
+
+
+@pytest.mark.parametrize("T,d,fuse", [(1, 128, 0), (3, 128, 0), (6, 128, 0), (1, 64, 0), (2, 128, 1), (1, 128, 3)],
+                         ids=["T1", "T3", "T6", "d64", "T2gates", "T1fused"])
+def test_shared_sources_hint_changes_no_bit(torch_cuda, T, d, fuse):
+    """GDN_SHARED_SOURCES only reorders the register-tile kernels' CTAs (head-major): with
+    a batch whose requests share source slots, every state and output equals the call
+    without the hint bit for bit, and the oracle's within tolerance."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(400 + 10 * T + d + fuse)
+    B, Hk, Hv = 12, 2, 4
+    num_slots = 4 + B * T + 2
+    pool_np = wl.init_pool(rng, num_slots, Hv, d, d)
+    q, k, v, a, b = wl.random_step_inputs(rng, B, T, Hk, Hv, d, d, wl.BF16)
+    src = rng.integers(0, 4, size=B).astype(np.int32)          # 12 requests over 4 shared checkpoints
+    dst = (4 + np.arange(B * T, dtype=np.int32)).reshape(B, T)  # fresh slots, copy-on-write
+    s = wl.Step(q, k, v, a, b, src, dst)
+    x = step_to_device(s)
+    results = []
+    for flags in (fuse, fuse | gdn.GDN_SHARED_SOURCES):
+        dev = to_torch(pool_np)
+        out = torch.full((B, T, Hv, d), -7.0, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        args = (dev, x["src"], x["dst"], x["q"], x["k"], x["v"], x["alpha"], x["beta"], out)
+        if flags:
+            gdn.gdn_decode_step_fused(*args, flags, err_word=err)
+        else:
+            gdn.gdn_decode_step(*args, err_word=err)
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_error(err) == gdn.GDN_OK
+        results.append((dev.cpu().numpy(), out.cpu().numpy()))
+    (p0, o0), (p1, o1) = results
+    assert np.array_equal(p0.view(np.uint32), p1.view(np.uint32))
+    assert np.array_equal(o0.view(np.uint32), o1.view(np.uint32))
+    if fuse == 0:
+        ref_pool, ref_out, skipped = run_oracle(pool_np, s)
+        assert skipped == 0
+        check_pool(p1, ref_pool, pool_np, dst)
+        assert rel_err(o1, ref_out) <= TOL_OUT_BF16
