@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "baba2a34a6488c4d30ff77c39a2dea4ec6059f58a577b12337b57db7e9ad8b14",
-               "bytes_per_launch": 541154816 + 485277952}
+               "source_sha256": "653e380a65bed55bdf5c11fb0841a0f3c2185c346aa9937013636690656a7732",
+               "bytes_per_launch": 541175040 + 483651584}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
