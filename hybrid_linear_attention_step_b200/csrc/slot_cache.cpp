@@ -117,9 +117,13 @@ struct gdn_slot_cache {
         return (int64_t)slots.size();
     }
 
-    // A free slot with reference count 1, evicting if needed; -1 if none.
+    // A free slot with reference count 1, evicting if needed; -1 if none.  One eviction
+    // frees nothing when another checkpoint names the same slot, so evict until a slot is
+    // free.  Every evictable checkpoint's slot is held by checkpoints only, so the loop
+    // ends with a free slot whenever evictable_slots() > 0, and evicts nothing otherwise.
     int32_t alloc() {
-        if (free_list.empty() && !evict_one()) return -1;
+        while (free_list.empty())
+            if (!evict_one()) return -1;
         const int32_t s = free_list.back();
         free_list.pop_back();
         ref[s] = 1;

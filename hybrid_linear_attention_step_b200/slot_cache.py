@@ -76,7 +76,10 @@ class SlotCache:
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            _lib().gdn_slot_cache_destroy(h)
+            try:
+                _lib().gdn_slot_cache_destroy(h)
+            except TypeError:  # interpreter shutdown: the module's globals are already gone
+                return
             self._h = None
 
     def open(self, tokens) -> Tuple[int, int, int, bool]:

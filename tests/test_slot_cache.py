@@ -188,6 +188,10 @@ def test_random_operations_keep_invariants_and_preconditions():
                 r = int(rng.choice(list(open_reqs)))
                 if open_reqs[r]:
                     c.checkpoint(r, open_reqs[r])
+                    if rng.random() < 0.3:
+                        # one state under a second, shorter prefix too: several checkpoints
+                        # then name one slot, which the bookkeeping must still count right
+                        c.checkpoint(r, open_reqs[r][: rng.integers(1, len(open_reqs[r]) + 1)])
             elif op == 8:
                 r = int(rng.choice(list(open_reqs)))
                 c.close(r)
@@ -204,3 +208,39 @@ def test_random_operations_keep_invariants_and_preconditions():
         c.close(r)
     c.evict(num_slots)
     assert c.stats() == (num_slots, 0, 0)
+
+
+def test_slot_named_by_several_checkpoints_is_freed_before_reuse():
+    """Two checkpoints of one request name the same slot.  With no free slot left, a new
+    request must get that slot only after both checkpoints are evicted: evicting one of
+    them frees nothing, and handing the slot out then would let the request overwrite a
+    cached prefix state."""
+    c = SlotCache(1)
+    req, s0, _, _ = c.open([1, 2, 3])
+    assert c.checkpoint(req, [1, 2]) == s0 and c.checkpoint(req, [1, 2, 3]) == s0
+    c.close(req)
+    assert c.stats() == (0, 2, 0) and c.refcount(s0) == 2
+    r2, s2, matched, needs_init = c.open([9])
+    assert (s2, matched, needs_init) == (s0, 0, True)
+    assert c.stats() == (0, 0, 1) and c.refcount(s0) == 1   # both checkpoints gone, slot owned once
+    c.close(r2)
+    _, _, matched, needs_init = c.open([1, 2, 3])              # the prefix is no longer cached
+    assert matched == 0 and needs_init
+
+
+def test_capacity_failure_with_shared_checkpoint_slot_changes_nothing():
+    """Slot 0 is held by a request and a checkpoint; slot 1 by two checkpoints of another
+    request.  A plan that needs two fresh slots fails (one evictable slot), and the
+    evictable checkpoints survive the failure."""
+    c = SlotCache(2)
+    a, sa, _, _ = c.open([1])
+    c.checkpoint(a, [1])
+    b, sb, _, _ = c.open([5, 6])
+    c.checkpoint(b, [5])
+    c.checkpoint(b, [5, 6])
+    c.close(b)
+    assert c.stats() == (0, 3, 1)
+    with pytest.raises(SlotCacheError) as e:
+        c.plan([a], T=2)  # the checkpointed source needs T = 2 fresh slots; one can be made
+    assert e.value.status == CAPACITY
+    assert c.stats() == (0, 3, 1) and c.refcount(sb) == 2
