@@ -224,7 +224,9 @@ gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, c
  * dependencies reduce to a unit lower-triangular system (I + A) E = R whose inverse
  * depends only on the chunk's keys and gates; a first kernel builds it for all
  * chunks in parallel, a second walks each sequence's chunks in order carrying the
- * state.  Supports dk = dv = 128.
+ * state.  Supports dk = dv = 128.  With bf16 inputs both kernels run their products on
+ * the tensor cores; with fp32 inputs they run on the CUDA cores and, on B200, take
+ * longer than gdn_prefill's token steps, which is then the faster call.
  *
  *   workspace        device memory of at least gdn_prefill_workspace_bytes(B, L, Hv,
  *                    dk, dv) bytes, 16-byte aligned, caller-owned; contents on entry
@@ -232,8 +234,8 @@ gdn_status gdn_prefill(float* pool, int32_t num_slots, const int32_t* src_idx, c
  *                    workspace must not overlap.
  *   err_word         device int32, required here (unlike gdn_prefill): besides index
  *                    errors, a copy or tensor-core wait that runs out (2 s) records
- *                    GDN_ERR_TIMEOUT, and the affected requests' checkpoints and
- *                    outputs are then left unwritten.
+ *                    GDN_ERR_TIMEOUT; the affected requests' checkpoints are then left
+ *                    unwritten and their outputs are unspecified.
  * Unsupported shapes, a missing or short workspace, a NULL err_word, or a workspace,
  * pool, out, q, k or v that is not 16-byte aligned return GDN_ERR_INVALID_ARG.
  */
