@@ -21,10 +21,11 @@
 // does not depend on the state into the caller's workspace; kernel 2 walks each
 // sequence's chunks in order, carrying the state.
 //
-// bf16 inputs (tensor cores, tcgen05 with accumulators in TMEM).  Kernel 1 forms
-// [K; Q] K^T as one MMA (exact bf16 products) and solves (I + A) [U | W] =
-// [diag(beta) V | diag(beta g) K] by forward substitution in fp32, W = Tb K, so that
-// kernel 2 evaluates the same algebra re-associated:
+// bf16 inputs (tensor cores, tcgen05 with accumulators in TMEM; k, q, v tiles brought
+// by tensor copies).  Kernel 1 forms [K; Q] K^T as one MMA (exact bf16 products),
+// inverts I + A in fp32 by 16 x 16 blocks, and forms U = T diag(beta) V and
+// W = T diag(beta g) K = Tb K as MMAs, so that kernel 2 evaluates the same algebra
+// re-associated:
 //     E = U - W M0,   O = diag(g) (Q M0) + P E,   M_C = g_C M0 + K^T diag(g_C / g) E,
 // all as MMAs.  Kernel 2 runs one CTA per (request, head) with the whole state: its
 // 128 value rows are the MMA's M dimension and the TMEM lanes.  An operand that is not
