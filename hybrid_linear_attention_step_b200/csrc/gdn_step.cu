@@ -393,14 +393,15 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
 
     const int hk = h / a.G;
     // Token t's inputs: thread j < DK fetches k_j and q_j, thread j < DVC its v
-    // column, thread 0 the gates.
-    auto fetch = [&](int t, float& kx, float& qx, float& vx, float& ax, float& bx, int& dx) {
+    // column, thread 0 the gates.  They stay in their input type until staged: a
+    // conversion right after the load would wait for it ahead of this token's stores.
+    auto fetch = [&](int t, InT& kx, InT& qx, InT& vx, float& ax, float& bx, int& dx) {
         const size_t tok = (size_t)b * T + t;
         if (tid < DK) {
-            kx = load_in<InT>(a.k, (tok * a.Hk + hk) * DK + tid);
-            qx = load_in<InT>(a.q, (tok * a.Hk + hk) * DK + tid);
+            kx = __ldg(static_cast<const InT*>(a.k) + (tok * a.Hk + hk) * DK + tid);
+            qx = __ldg(static_cast<const InT*>(a.q) + (tok * a.Hk + hk) * DK + tid);
         }
-        if (tid < DVC) vx = load_in<InT>(a.v, (tok * a.Hv + h) * DV + (size_t)chunk * DVC + tid);
+        if (tid < DVC) vx = __ldg(static_cast<const InT*>(a.v) + (tok * a.Hv + h) * DV + (size_t)chunk * DVC + tid);
         if (tid == 0) {
             const float x = __ldg(a.alpha + tok * a.Hv + h), y = __ldg(a.beta + tok * a.Hv + h);
             const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
@@ -412,12 +413,12 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     // The destination slot goes through shared memory as well: re-reading it
     // from global memory at store time would put a cache miss in front of the
     // stores, and holding it in a register costs occupancy.
-    auto stage = [&](int buf, float kx, float qx, float vx, float ax, float bx, int dx) {
+    auto stage = [&](int buf, InT kx, InT qx, InT vx, float ax, float bx, int dx) {
         if (tid < DK) {
-            ks[buf][tid] = kx;
-            qs[buf][tid] = qx;
+            ks[buf][tid] = to_f32(kx);
+            qs[buf][tid] = to_f32(qx);
         }
-        if (tid < DVC) vs[buf][tid] = vx;
+        if (tid < DVC) vs[buf][tid] = to_f32(vx);
         if (tid == 0) {
             gates[buf][0] = ax;
             gates[buf][1] = bx;
@@ -426,7 +427,8 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     };
     static_assert(NT >= DK || !MULTI, "one thread per k/q element when staging tokens");
     {
-        float kx = 0.f, qx = 0.f, vx = 0.f, ax = 0.f, bx = 0.f;
+        InT kx = InT(0.f), qx = InT(0.f), vx = InT(0.f);
+        float ax = 0.f, bx = 0.f;
         int dx = 0;
         if (NT >= DK) {
             fetch(0, kx, qx, vx, ax, bx, dx);
@@ -438,7 +440,7 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
                 qs[0][i] = load_in<InT>(a.q, kbase + i);
             }
             fetch(0, kx, qx, vx, ax, bx, dx);
-            if (tid < DVC) vs[0][tid] = vx;
+            if (tid < DVC) vs[0][tid] = to_f32(vx);
             if (tid == 0) {
                 gates[0][0] = ax;
                 gates[0][1] = bx;
@@ -490,7 +492,8 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
         __syncthreads();
 
         // Next token's inputs are requested now; their latency hides behind this token's stores.
-        float kx = 0.f, qx = 0.f, vx = 0.f, ax = 0.f, bx = 0.f;
+        InT kx = InT(0.f), qx = InT(0.f), vx = InT(0.f);
+        float ax = 0.f, bx = 0.f;
         int dx = 0;
         if (MULTI && t + 1 < T) fetch(t + 1, kx, qx, vx, ax, bx, dx);
 
