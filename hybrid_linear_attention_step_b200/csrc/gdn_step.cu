@@ -403,10 +403,8 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
         }
         if (tid < DVC) vx = __ldg(static_cast<const InT*>(a.v) + (tok * a.Hv + h) * DV + (size_t)chunk * DVC + tid);
         if (tid == 0) {
-            const float x = __ldg(a.alpha + tok * a.Hv + h), y = __ldg(a.beta + tok * a.Hv + h);
-            const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
-            ax = raw ? alpha_from_raw(x) : x;
-            bx = raw ? beta_from_raw(y) : y;
+            ax = __ldg(a.alpha + tok * a.Hv + h);  // raw x, y with GDN_FUSE_GATES: mapped when staged
+            bx = __ldg(a.beta + tok * a.Hv + h);
             dx = (t == 0 || a.prefill) ? dst0 : __ldg(a.dst_idx + tok);
         }
     };
@@ -420,8 +418,9 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
         }
         if (tid < DVC) vs[buf][tid] = to_f32(vx);
         if (tid == 0) {
-            gates[buf][0] = ax;
-            gates[buf][1] = bx;
+            const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
+            gates[buf][0] = raw ? alpha_from_raw(ax) : ax;
+            gates[buf][1] = raw ? beta_from_raw(bx) : bx;
             dst_s[buf] = dx;
         }
     };
@@ -442,8 +441,9 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
             fetch(0, kx, qx, vx, ax, bx, dx);
             if (tid < DVC) vs[0][tid] = to_f32(vx);
             if (tid == 0) {
-                gates[0][0] = ax;
-                gates[0][1] = bx;
+                const bool raw = FUSE && (a.flags & GDN_FUSE_GATES);
+                gates[0][0] = raw ? alpha_from_raw(ax) : ax;
+                gates[0][1] = raw ? beta_from_raw(bx) : bx;
                 dst_s[0] = dx;
             }
         }
