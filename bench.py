@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "653e380a65bed55bdf5c11fb0841a0f3c2185c346aa9937013636690656a7732",
-               "bytes_per_launch": 541175040 + 483651584}
+               "source_sha256": "040fb3c3fc68f6c4b273d43468d268aa8392de62a54a64e2a8ec1fa799181537",
+               "bytes_per_launch": 541153280 + 483076608}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
