@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "040fb3c3fc68f6c4b273d43468d268aa8392de62a54a64e2a8ec1fa799181537",
+               "source_sha256": "2827aedbcf7c211ac4e2f41f69a398f46b47640b8b33449e134845a6607594e3",
                "bytes_per_launch": 541153280 + 483076608}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the

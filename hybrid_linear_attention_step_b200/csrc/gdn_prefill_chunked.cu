@@ -199,7 +199,7 @@ struct TileMaps {
     CUtensorMap k, q, v;
 };
 
-// One tile load (no multicast) completing on `bar` with its byte count.
+// One tile load into this CTA's shared memory, completing on `bar` with its byte count.
 __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, int feat, int head, int tok, int req,
                                          uint64_t* bar) {
     asm volatile(

@@ -786,9 +786,9 @@ __global__ void gdn_column_kernel(StepArgs a) {
 
 // ---------------------------------------------------------------------------
 // Bulk-copy helpers (sm_90+ PTX, used on sm_100a): mbarrier transaction
-// counting and one-dimensional cp.async.bulk global -> shared copies.  No
-// multicast and no tensor maps: every copy is a contiguous, 16-byte aligned
-// range of this GPU's own memory.
+// counting and one-dimensional cp.async.bulk global -> shared copies into this
+// CTA's own shared memory, without tensor maps: every copy is a contiguous,
+// 16-byte aligned range of this GPU's own memory.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
