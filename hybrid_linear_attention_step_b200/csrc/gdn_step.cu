@@ -61,9 +61,11 @@ constexpr int kFuseFlags = GDN_FUSE_GATES | GDN_FUSE_QK_NORM;
 
 // unit_order: the register-tile kernels number their CTAs (request, head, column block)
 // request-major, so that consecutive CTAs walk one slot's contiguous 2 MiB (the faster
-// order when every request has a state of its own).  With GDN_SHARED_SOURCES they go
-// head-major: every request of one value head within a fraction of a wave, so that a
-// source tile that several requests share is read from HBM once and then from L2.
+// order when every request has a state of its own).  With GDN_SHARED_SOURCES the
+// single-token kernel goes head-major: every request of one value head within a fraction
+// of a wave, so that a source tile that several requests share is read from HBM once and
+// then from L2.  (The multi-token kernels keep request-major order: the extra index
+// arithmetic cost them registers and time, and prefix sharing is a single-token case.)
 
 // Fused prologue (gdn_decode_step_fused).  alpha = exp(-softplus(x)) equals
 // 1 / (1 + e^x) exactly, and beta = sigmoid(y) = 1 / (1 + e^-y); both limits
@@ -368,9 +370,8 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tile_kernel(StepArgs a) {
     const int rg = tid / CG;
     const int chunk = blockIdx.x % NC;
     const int unit = blockIdx.x / NC;
-    const bool by_head = (a.flags & GDN_SHARED_SOURCES) != 0;  // see unit_order
-    const int h = by_head ? unit / a.B : unit % a.Hv;
-    const int b = by_head ? unit % a.B : unit / a.Hv;
+    const int h = unit % a.Hv;  // request-major (the ordering hint serves single-token calls)
+    const int b = unit / a.Hv;
     const int T = MULTI ? a.T : 1;
 
     grid_dependency_wait();  // launched with programmatic dependent launch, as gdn_tile1_kernel
@@ -588,9 +589,8 @@ __global__ void __launch_bounds__(NT, MINB) gdn_tileT_kernel(StepArgs a) {
     const int rg = tid / CG;
     const int chunk = blockIdx.x % NC;
     const int unit = blockIdx.x / NC;
-    const bool by_head = (a.flags & GDN_SHARED_SOURCES) != 0;  // see unit_order
-    const int h = by_head ? unit / a.B : unit % a.Hv;
-    const int b = by_head ? unit % a.B : unit / a.Hv;
+    const int h = unit % a.Hv;  // request-major (the ordering hint serves single-token calls)
+    const int b = unit / a.Hv;
     const int T = a.T;
 
     grid_dependency_wait();

@@ -176,10 +176,10 @@ gdn_status gdn_decode_step_variant(float* pool, int32_t num_slots, const int32_t
  *   flags & GDN_SHARED_SOURCES: a hint that many of the batch's requests share
  *                             source slots (prefix-checkpoint hits; a caller that
  *                             plans with gdn_slot_cache_plan sees it as repeated
- *                             src entries).  The register-tile kernels then visit
- *                             every request of one value head before the next
- *                             head, so a shared tile is read from HBM once and then
- *                             from L2.  The result is bit for bit the same with or
+ *                             src entries).  The single-token register-tile kernel
+ *                             then visits every request of one value head before
+ *                             the next head, so a shared tile is read from HBM once
+ *                             and then from L2; other kernels ignore the hint.  The result is bit for bit the same with or
  *                             without it; without sharing it only costs bandwidth
  *                             (request-major order keeps each slot's 2 MiB together).
  * Without flags the call is gdn_decode_step.  Same layouts, preconditions, errors
