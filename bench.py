@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "2827aedbcf7c211ac4e2f41f69a398f46b47640b8b33449e134845a6607594e3",
-               "bytes_per_launch": 541153280 + 483076608}
+               "source_sha256": "0984bccc532caada70117c89e186038080876014904470c22dd5bdd2f1c75da4",
+               "bytes_per_launch": 541174528 + 483733504}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).
