@@ -656,11 +656,12 @@ def test_prefill_chunked_matches_oracle(torch_cuda, shape):
     assert rel_err(out.cpu().numpy(), ref_out) <= TOL_OUT_BF16
 
 
-@pytest.mark.parametrize("L", [200, 700])
+@pytest.mark.parametrize("L", [200, 700, 4096])
 def test_prefill_chunked_slow_decay(torch_cuda, L):
     """Gates close to one (alpha ~ 0.97, the slow forgetting of trained models): the chunk-start
     state then reaches every token of a chunk, so the products with the carried state (W M,
-    and the state update) carry the result and their precision is what is tested."""
+    and the state update) carry the result and their precision is what is tested.  L = 4096
+    carries the state through 64 chunks, where a part product left out would accumulate."""
     torch = torch_cuda
     import oracle
     from hybrid_linear_attention_step_b200 import gdn
