@@ -830,3 +830,52 @@ def test_shared_sources_hint_changes_no_bit(torch_cuda, T, d, fuse):
         assert skipped == 0
         check_pool(p1, ref_pool, pool_np, dst)
         assert rel_err(o1, ref_out) <= TOL_OUT_BF16
+
+
+def test_prefill_chunked_replays_from_a_cuda_graph(torch_cuda):
+    """The chunked prefill captured once in a CUDA graph (its tensor maps are kernel
+    arguments, its second kernel a programmatic dependent launch) and replayed with new
+    inputs written into the captured buffers: every replay equals an eager call bit for bit."""
+    torch = torch_cuda
+    from hybrid_linear_attention_step_b200 import gdn
+
+    rng = np.random.default_rng(71)
+    B, L, Hk, Hv = 2, 200, 2, 4
+    pool0 = wl.init_pool(rng, 2 * B, Hv, 128, 128)
+    src = to_torch(np.arange(B, dtype=np.int32))
+    dst = to_torch(np.arange(B, 2 * B, dtype=np.int32))
+
+    def inputs():
+        q, k, v, a, b = wl.random_step_inputs(rng, B, L, Hk, Hv, 128, 128, wl.BF16)
+        return [to_torch(x) for x in (q, k, v, a, b)]
+
+    bufs = inputs()
+    pool = to_torch(pool0)
+    out = torch.zeros((B, L, Hv, 128), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(gdn.gdn_prefill_workspace_bytes(B, L, Hv, 128, 128), dtype=torch.uint8, device="cuda")
+    call = lambda: gdn.gdn_prefill_chunked(pool, src, dst, *bufs, out, ws, err_word=err)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for _ in range(3):
+        for t_dev, x in zip(bufs, inputs()):
+            t_dev.copy_(x)
+        pool.copy_(to_torch(pool0))
+        graph.replay()
+        torch.cuda.synchronize()
+        got_pool, got_out = pool.cpu().numpy(), out.cpu().numpy()
+        pool.copy_(to_torch(pool0))
+        out.zero_()
+        call()
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_error(err) == gdn.GDN_OK
+        assert np.array_equal(got_pool.view(np.uint32), pool.cpu().numpy().view(np.uint32))
+        assert np.array_equal(got_out.view(np.uint32), out.cpu().numpy().view(np.uint32))
+        assert np.isfinite(got_out).all()
