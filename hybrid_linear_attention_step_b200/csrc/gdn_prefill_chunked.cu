@@ -230,6 +230,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t
         : "memory");
 }
 
+// The same with A in TMEM: row m of A on lane m, its 16 K-elements packed two to a 32-bit
+// column (the lower K index in the low half) over 8 columns from tmem_a.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                             uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
@@ -1121,17 +1132,19 @@ __global__ void __launch_bounds__(kNT, 1) gdn_chunk_scan_kernel(ChunkArgs a) {
 //   E^T = U^T - (G0 + G1 + G2) = (U - W M)^T,    QM^T = G3 (q M per token), scaled by g_t
 // (the part products left out are below 2^-24 of W M, and 2^-16 of Q M, an output-only
 // term).  Then with E' = diag(g_C / g) E split in three parts and E in two as A operands
-// (K = 64 tokens):
+// (K = 64 tokens), held in TMEM: each thread writes its parts over columns of G it has
+// already read (8 columns per part and 16 tokens, see the E phase), so they take neither
+// shared memory nor its bandwidth:
 //   D_U = E'^T K              (B = the K tiles, MN-major; cols 256..383) ->  S <- g_C S + D_U
 //   D_O = E_hi [P_mid P_hi] + E_mid [P_hi]   (cols 384..511)  ->  o = g Q M + P E
-// The state update is committed first; the chain waits only for it.  The issuing
+// The state update is committed first; the chain waits only for it, and the next S parts
+// are written while the outputs' products run.  The issuing
 // thread streams three shared-memory images, record fields by cp.async.bulk and the
 // chunk's Q and K tiles by tensor copies: each buffer is refilled for the next chunk as
 // soon as its last reader is done.  Every wait is bounded (2 s);
 // a timeout is recorded and the CTA drains and exits.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kSPart = (uint32_t)kD * kD * 2;  // one bf16 part of S (128 x 128)
-constexpr uint32_t kEPart = (uint32_t)kD * kC * 2;  // one bf16 part of E^T or E'^T (128 x 64)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemDU = 256;
 constexpr uint32_t kTmemDO = 384;
@@ -1139,7 +1152,7 @@ constexpr int kScanThreads = 512;                   // 16 warps, all of them com
 constexpr int kIssuer = 0;                          // the thread that also issues MMAs and copies
 
 struct SmemS {
-    unsigned char aop[3 * kSPart];  // A operands: S parts; then E'^T parts (3) and E^T parts (hi, mid)
+    unsigned char aop[3 * kSPart];  // A operands of the first products: S parts
     unsigned char imgA[kImgA];      // [W_lo W_mid W_hi Q] for features 0..63, then 64..127
     unsigned char imgB[kImgB];      // [K lo | K hi] | [P_mid | P_hi]
     unsigned char imgC[kImgC];      // g_t, g_C / g_t, g_C | U^T
@@ -1150,7 +1163,6 @@ struct SmemS {
 constexpr int kSmemS = (int)sizeof(SmemS) + 1024;  // + alignment slack
 static_assert(kSmemS <= 227 * 1024, "scan shared memory plan exceeds the per-CTA limit");
 static_assert(3 * kSPart % 1024 == 0 && kImgA % 1024 == 0, "swizzled images start on 1024-byte boundaries");
-static_assert(3 * kEPart + 2 * kEPart <= 3 * kSPart, "E parts overlay the S parts");
 
 // 8 consecutive TMEM columns of this warp's 32 lanes (completion awaited separately).
 __device__ __forceinline__ void tmem_ld8_issue(uint32_t addr, uint32_t (&r)[8]) {
@@ -1161,6 +1173,18 @@ __device__ __forceinline__ void tmem_ld8_issue(uint32_t addr, uint32_t (&r)[8]) 
 __device__ __forceinline__ void tie_regs8(uint32_t (&r)[8]) {
     asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
 }
+// 4 or 8 consecutive TMEM columns of this warp's 32 lanes, from registers.
+__device__ __forceinline__ void tmem_st4(uint32_t addr, const uint4& v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t addr, const uint4& v, const uint4& w) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(addr), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kScanThreads, 1)
     gdn_chunk_scan_tc_kernel(ChunkArgs a, const __grid_constant__ TileMaps maps) {
@@ -1354,6 +1378,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         if (compute) {
             const float* gk = gq + kC;
             const float4* ut = reinterpret_cast<const float4*>(sm.imgC + kR2GBytes) + j;
+            uint4 emid0;  // E_mid of the first 8 tokens (stored with the second 8)
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
                 const uint32_t col = (uint32_t)(16 * quarter + 8 * p);
@@ -1380,17 +1405,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                         qm[8 * p + mm] = __uint_as_float(r3[mm]) * gq[t];
                     }
                 }
-                uint4 p0, p1, p2;
-                const uint32_t off = core_off(j, (int)col, kC);
+                // Parts 0..3 over columns 4p.. of the first 8 of this thread's 16 columns of
+                // G block 0..3 (read in pass 0); part 4 after pass 1, over the last 8 of block 0.
+                uint4 p0, p1, p2, p3, p4;
                 split3x8_fast(ep, p0, p1, p2);
-                *reinterpret_cast<uint4*>(sm.aop + off) = p0;
-                *reinterpret_cast<uint4*>(sm.aop + kEPart + off) = p1;
-                *reinterpret_cast<uint4*>(sm.aop + 2 * kEPart + off) = p2;
-                split2x8_fast(e, p0, p1);
-                *reinterpret_cast<uint4*>(sm.aop + 3 * kEPart + off) = p0;
-                *reinterpret_cast<uint4*>(sm.aop + 4 * kEPart + off) = p1;
+                split2x8_fast(e, p3, p4);
+                const uint32_t gb = tmem + lane_base + (uint32_t)(16 * quarter);
+                tmem_st4(gb + 4 * p, p0);
+                tmem_st4(gb + kC + 4 * p, p1);
+                tmem_st4(gb + 2 * kC + 4 * p, p2);
+                tmem_st4(gb + 3 * kC + 4 * p, p3);
+                if (p == 0)
+                    emid0 = p4;
+                else
+                    tmem_st8(gb + 8, emid0, p4);
             }
-            async_proxy_fence();
+            tmem_wait_st();
         }
         out_t0 = c * kC;
         out_n = min(kC, a.L - out_t0);
@@ -1414,20 +1444,23 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             }
             // B = K, MN-major: features 64 to a row, tokens one row each (16 tokens per
             // MMA: 2048 bytes), the second feature half one tile on.
-            const uint32_t aE = smem_u32(sm.aop), bK = smem_u32(sm.imgB), bP = bK + 2 * kSwTile;
+            const uint32_t bK = smem_u32(sm.imgB), bP = bK + 2 * kSwTile;
             constexpr uint32_t kSbo = (kC / 8) * 128;
+            // A: E part p of the 16 tokens of K-step ks, in TMEM (written by token quarter ks).
+            auto epart = [&](int p, int ks) -> uint32_t {
+                return tmem + (uint32_t)(16 * ks) + (p < 4 ? (uint32_t)(p * kC) : 8u);
+            };
             for (int part = 0; part < 3; ++part)
                 for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16(tmem + kTmemDU, umma_desc(aE + part * kEPart + 256 * ks, kSbo),
-                              umma_desc_sw128(bK + 2048u * ks, kSwTile, 1024), kIdesc128 | kIdescBmn,
-                              (part | ks) != 0 ? 1u : 0u);
+                    umma_bf16_ta(tmem + kTmemDU, epart(part, ks), umma_desc_sw128(bK + 2048u * ks, kSwTile, 1024),
+                                 kIdesc128 | kIdescBmn, (part | ks) != 0 ? 1u : 0u);
             umma_commit(&sm.mma_u);
             for (int ks = 0; ks < kC / 16; ++ks)
-                umma_bf16(tmem + kTmemDO, umma_desc(aE + 3 * kEPart + 256 * ks, kSbo), umma_desc(bP + 256 * ks, kSbo),
-                          kIdesc128, ks != 0 ? 1u : 0u);
+                umma_bf16_ta(tmem + kTmemDO, epart(3, ks), umma_desc(bP + 256 * ks, kSbo), kIdesc128,
+                             ks != 0 ? 1u : 0u);
             for (int ks = 0; ks < kC / 16; ++ks)
-                umma_bf16(tmem + kTmemDO + kC, umma_desc(aE + 4 * kEPart + 256 * ks, kSbo),
-                          umma_desc(bP + (kC / 8) * kSbo + 256 * ks, kSbo), kIdesc64, 1u);
+                umma_bf16_ta(tmem + kTmemDO + kC, epart(4, ks), umma_desc(bP + (kC / 8) * kSbo + 256 * ks, kSbo),
+                             kIdesc64, 1u);
             umma_commit(&sm.mma_o);
             ++issued_u, ++issued_o;
         }
@@ -1450,7 +1483,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 s[16 + m] = fmaf(gC, s[16 + m], __uint_as_float(r1[m]));
             }
         }
-        // The outputs' products still read the E parts: the next S parts overwrite them.
+        // The next S parts (the first products are complete: the state update's commit
+        // covers them), written while the outputs' products run.
+        if (compute && c + 1 < nch) split_s();
+        // The outputs' products read the E parts in TMEM, which the next first products
+        // overwrite.
         got = wait_parity(&sm.mma_o, (uint32_t)c & 1u);
         tc_fence_before();
         if (__syncthreads_or(got ? 0 : 1)) {
@@ -1465,7 +1502,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 ++issued_b;
             }
         }
-        if (compute && c + 1 < nch) split_s();
     }
 
     if (ok) {
