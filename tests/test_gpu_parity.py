@@ -623,6 +623,7 @@ CHUNKED_SHAPES = [
     (1, 1000, 1, 2, wl.BF16, True),
     (4, 130, 2, 2, wl.BF16, False),   # one value head per key head, ragged last chunk
     (2, 96, 1, 4, wl.BF16, True),     # four value heads per key head, in place
+    (10, 130, 16, 32, wl.BF16, False),  # 320 scan CTAs: more (request, head) chains than SMs
 ]
 
 
