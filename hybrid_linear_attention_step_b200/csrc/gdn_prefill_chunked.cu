@@ -1192,7 +1192,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     SmemS& sm = *reinterpret_cast<SmemS*>(align1024(smem_tc));
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
-    constexpr bool compute = true;
     const bool issuer = tid == kIssuer;
     const int bh = blockIdx.x;
     const int h = bh % a.Hv;
@@ -1260,7 +1259,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
 
     float s[32];  // S[j][32 quarter + i]
-    if (compute) {
+    {
         const float* M0 = a.pool + ((size_t)sm.src * a.Hv + h) * (kD * kD) + (size_t)(32 * quarter) * kD + j;
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[i] = M0[(size_t)i * kD];
@@ -1280,7 +1279,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             *reinterpret_cast<uint4*>(sm.aop + 2 * kSPart + off) = p2;
         }
     };
-    if (compute) split_s();
+    split_s();
 
     constexpr uint32_t kIdesc256 = umma_idesc(128, 256), kIdesc192 = umma_idesc(128, 192);
     constexpr uint32_t kIdesc128 = umma_idesc(128, 128), kIdesc64 = umma_idesc(128, 64);
@@ -1313,7 +1312,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     for (; c < nch; ++c) {
         // --- the chunk's first products: S parts x [W parts | Q]
         bool got = true;
-        if (compute) async_proxy_fence();  // the S parts just written, for the tensor cores
+        async_proxy_fence();  // the S parts just written, for the tensor cores
         if (issuer) got = wait_parity(&sm.bar_a, (uint32_t)c & 1u);
         tc_fence_before();
         if (__syncthreads_or(got ? 0 : 1)) {
@@ -1359,7 +1358,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
 
         got = wait_parity(&sm.mma_g, (uint32_t)c & 1u);
-        if (compute) got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
+        got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
         if (issuer && got) {
             ++waits_g;
             if (c + 1 < nch) {  // the BW buffer is free again
@@ -1375,7 +1374,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         // --- E = U - W M and g Q M for this thread's 16 tokens
         const float* gq = reinterpret_cast<const float*>(sm.imgC);
         const float gC = gq[2 * kC];
-        if (compute) {
+        {
             const float* gk = gq + kC;
             const float4* ut = reinterpret_cast<const float4*>(sm.imgC + kR2GBytes) + j;
             uint4 emid0;  // E_mid of the first 8 tokens (stored with the second 8)
@@ -1471,7 +1470,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
         if (issuer) ++waits_u;
         tc_fence_after();
-        if (compute) {
+        {
             uint32_t r0[16], r1[16];
             tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(32 * quarter), r0);
             tmem_ld16_issue(tmem + lane_base + kTmemDU + (uint32_t)(32 * quarter + 16), r1);
@@ -1485,7 +1484,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
         // The next S parts (the first products are complete: the state update's commit
         // covers them), written while the outputs' products run.
-        if (compute && c + 1 < nch) split_s();
+        if (c + 1 < nch) split_s();
         // The outputs' products read the E parts in TMEM, which the next first products
         // overwrite.
         got = wait_parity(&sm.mma_o, (uint32_t)c & 1u);
@@ -1505,7 +1504,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
 
     if (ok) {
-        if (compute) {
+        {
             store_outputs(0);  // the last chunk's
             store_outputs(1);
             float* MD = a.pool + ((size_t)sm.dst * a.Hv + h) * (kD * kD) + (size_t)(32 * quarter) * kD + j;
