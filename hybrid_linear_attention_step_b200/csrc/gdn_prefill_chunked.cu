@@ -1308,18 +1308,24 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
     };
 
+    // Two CTA barriers per chunk: before the first products (the S parts are written)
+    // and before the state update's products (the E parts are written).  Every other
+    // hand-off is an mbarrier that each thread waits on itself; what those waits saw is
+    // carried to the next barrier, which stops the walk if any ran out.
+    bool carry = true;
     int c = 0;
     for (; c < nch; ++c) {
         // --- the chunk's first products: S parts x [W parts | Q]
-        bool got = true;
+        bool got = carry;
         async_proxy_fence();  // the S parts just written, for the tensor cores
-        if (issuer) got = wait_parity(&sm.bar_a, (uint32_t)c & 1u);
+        if (issuer) got = wait_parity(&sm.bar_a, (uint32_t)c & 1u) && got;
         tc_fence_before();
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
             break;
         }
         tc_fence_after();
+        carry = true;
         // The chunk's first products, issued by thread 0 in three batches (one per S
         // part) with its warp's share of the previous chunk's outputs stored in between;
         // the other warps store theirs while the products run.
@@ -1358,7 +1364,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
 
         got = wait_parity(&sm.mma_g, (uint32_t)c & 1u);
-        got = wait_parity(&sm.bar_c, (uint32_t)c & 1u) && got;
         if (issuer && got) {
             ++waits_g;
             if (c + 1 < nch) {  // the BW buffer is free again
@@ -1366,9 +1371,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 ++issued_a;
             }
         }
-        if (__syncthreads_or(got ? 0 : 1)) {
-            ok = false;
-            break;
+        {
+            const bool gc = wait_parity(&sm.bar_c, (uint32_t)c & 1u);
+            if (issuer && gc) ++done_c;
+            got = got && gc;
         }
         tc_fence_after();
         // --- E = U - W M and g Q M for this thread's 16 tokens
@@ -1423,11 +1429,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
         out_t0 = c * kC;
         out_n = min(kC, a.L - out_t0);
-        got = true;
-        if (issuer) {
-            ++done_c;
-            got = wait_parity(&sm.bar_b, (uint32_t)c & 1u);
-        }
+        if (issuer) got = wait_parity(&sm.bar_b, (uint32_t)c & 1u) && got;
         tc_fence_before();
         if (__syncthreads_or(got ? 0 : 1)) {
             ok = false;
@@ -1463,12 +1465,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             umma_commit(&sm.mma_o);
             ++issued_u, ++issued_o;
         }
-        got = wait_parity(&sm.mma_u, (uint32_t)c & 1u);
-        if (__syncthreads_or(got ? 0 : 1)) {
-            ok = false;
-            break;
+        {
+            const bool gu = wait_parity(&sm.mma_u, (uint32_t)c & 1u);
+            if (issuer && gu) ++waits_u;
+            carry = gu;
         }
-        if (issuer) ++waits_u;
         tc_fence_after();
         {
             uint32_t r0[16], r1[16];
@@ -1486,22 +1487,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         // covers them), written while the outputs' products run.
         if (c + 1 < nch) split_s();
         // The outputs' products read the E parts in TMEM, which the next first products
-        // overwrite.
-        got = wait_parity(&sm.mma_o, (uint32_t)c & 1u);
-        tc_fence_before();
-        if (__syncthreads_or(got ? 0 : 1)) {
-            ok = false;
-            break;
-        }
-        tc_fence_after();
-        if (issuer) {
-            ++waits_o;
-            if (c + 1 < nch) {  // K^T and the P tile are consumed
-                issue_b(c + 1);
-                ++issued_b;
+        // overwrite, and the outputs are read from their accumulator next chunk.
+        {
+            const bool go = wait_parity(&sm.mma_o, (uint32_t)c & 1u);
+            if (issuer && go) {
+                ++waits_o;
+                if (c + 1 < nch) {  // K^T and the P tile are consumed
+                    issue_b(c + 1);
+                    ++issued_b;
+                }
             }
+            carry = carry && go;
         }
+        tc_fence_before();
     }
+    if (ok) ok = !__syncthreads_or(carry ? 0 : 1);  // the last chunk's waits
+    tc_fence_after();
 
     if (ok) {
         {
