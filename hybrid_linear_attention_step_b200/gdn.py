@@ -93,10 +93,24 @@ def status_string(status: int) -> str:
     return load_library().gdn_status_string(int(status)).decode()
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, dev: Optional[int] = None) -> int:
+    """The launch stream's handle: torch's current stream when ``stream`` is None.  With
+    ``dev`` (the index of the call's tensors' device) the stream must belong to that
+    device: the library launches on the calling thread's current device and takes the
+    pointers as they are, so another device's buffers would be read from the wrong GPU.
+    torch's current stream belongs to the current device; a raw handle is checked
+    against the current device."""
     if stream is None:
         stream = torch.cuda.current_stream()
-    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+    if hasattr(stream, "cuda_stream"):
+        if dev is not None and stream.device_index != dev:
+            raise ValueError(f"the tensors are on cuda:{dev} but the launch stream is on cuda:{stream.device_index}"
+                             f" (the current device, unless a stream was given); call inside torch.cuda.device({dev})")
+        return int(stream.cuda_stream)
+    if dev is not None and torch.cuda.current_device() != dev:
+        raise ValueError(f"the tensors are on cuda:{dev} but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}; call inside torch.cuda.device({dev})")
+    return int(stream)
 
 
 def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
@@ -109,15 +123,27 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
     return t.data_ptr()
 
 
+def _one_device(*tensors) -> int:
+    """The CUDA device index of a call's tensors, which must all be on one device (the
+    launch stream's: see _stream_handle)."""
+    devs = {t.get_device() for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError("the tensors of one call must be on one CUDA device, got devices "
+                         + ", ".join(str(d) for d in sorted(devs)))
+    return devs.pop()
+
+
 def _ptr_or_null(t: Optional[torch.Tensor], name: str) -> Optional[int]:
     return None if t is None else _dev(t, name, torch.int32)
 
 
-def _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=None):
+def _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=None, extra=(), stream=None):
     """Pointers and sizes for the decode and prefill entry points.  The library sees plain
     pointers, so every tensor's shape is checked against pool and q here: a mismatch
     would otherwise read or write past a buffer.  dst_idx holds dst_per_request entries
-    per request (T by default; 1 for a prefill)."""
+    per request (T by default; 1 for a prefill).  ``extra`` tensors of the call (error
+    word, workspace) join the one-device check; returns the pointers and sizes, and the
+    launch stream's handle."""
     if pool.dim() != 4 or q.dim() != 4 or v.dim() != 4:
         raise ValueError("pool, q, k, v must be 4-D")
     num_slots, Hv, dk, dv = pool.shape
@@ -133,12 +159,13 @@ def _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_requ
     per = T if dst_per_request is None else dst_per_request
     if src_idx.numel() != B or dst_idx.numel() != B * per:
         raise ValueError(f"src_idx must hold B = {B} entries and dst_idx B * {per}")
-    return (_dev(pool, "pool", torch.float32), int(num_slots),
+    args = (_dev(pool, "pool", torch.float32), int(num_slots),
             _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32),
             _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
             _dev(alpha, "alpha", torch.float32), _dev(beta, "beta", torch.float32),
             _dev(out, "out", torch.float32),
             int(B), int(T), int(Hk), int(Hv), int(dk), int(dv), _DTYPES[q.dtype])
+    return args, _stream_handle(stream, _one_device(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, *extra))
 
 
 def gdn_decode_step(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor,
@@ -151,8 +178,8 @@ def gdn_decode_step(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Te
     q, k [B, T, Hk, dk] and v [B, T, Hv, dv] bf16 or fp32; alpha, beta [B, T, Hv] fp32;
     out [B, T, Hv, dv] fp32.  Returns the status; raises GdnError on failure when ``check``.
     """
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
-    status = load_library().gdn_decode_step(*args, _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    args, sh = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, extra=(err_word,), stream=stream)
+    status = load_library().gdn_decode_step(*args, _ptr_or_null(err_word, "err_word"), sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_decode_step")
     return status
@@ -177,8 +204,9 @@ class PreparedDecodeStep:
                  alpha: torch.Tensor, beta: torch.Tensor, out: torch.Tensor,
                  err_word: Optional[torch.Tensor] = None, variant=None, stream=None, flags: int = 0):
         lib = load_library()
-        args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
+        args, sh = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, extra=(err_word,), stream=stream)
         err = _ptr_or_null(err_word, "err_word")
+        self._device = pool.get_device()
         if flags and variant is not None:
             raise ValueError("flags go with the automatic kernel choice: pass variant=None")
         if flags:
@@ -193,14 +221,14 @@ class PreparedDecodeStep:
             self._fn, self._name = lib.gdn_decode_step_variant, "gdn_decode_step_variant"
             args = args + (err, int(variant))
         self._args = args
-        self._stream = None if stream is None else _stream_handle(stream)
+        self._stream = None if stream is None else sh
         self._keep = (pool, src_idx, dst_idx, q, k, v, alpha, beta, out, err_word, stream)
 
     def __call__(self, stream=None, check: bool = True) -> int:
         if stream is None and self._stream is not None:
-            handle = self._stream
+            handle = self._stream  # a stream of the buffers' device, checked once
         else:
-            handle = _stream_handle(stream)
+            handle = _stream_handle(stream, self._device)
         status = self._fn(*self._args, handle)
         if check and status != GDN_OK:
             raise GdnError(status, self._name)
@@ -215,9 +243,8 @@ def gdn_decode_step_variant(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: 
     ("auto", "stream", "tile", "column")."""
     if isinstance(variant, str):
         variant = VARIANTS[variant]
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out)
-    status = load_library().gdn_decode_step_variant(*args, _ptr_or_null(err_word, "err_word"), int(variant),
-                                                    _stream_handle(stream))
+    args, sh = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, extra=(err_word,), stream=stream)
+    status = load_library().gdn_decode_step_variant(*args, _ptr_or_null(err_word, "err_word"), int(variant), sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_decode_step_variant")
     return status
@@ -231,9 +258,9 @@ def gdn_decode_step_fused(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: to
     include/gdn_step.h): GDN_FUSE_GATES makes alpha_or_x / beta_or_y the raw x, y;
     GDN_FUSE_QK_NORM L2-normalises q and k inside the kernel; GDN_SHARED_SOURCES tells the
     kernels that many requests share source slots (an ordering hint, same results)."""
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha_or_x, beta_or_y, out)
-    status = load_library().gdn_decode_step_fused(*args, int(flags), _ptr_or_null(err_word, "err_word"),
-                                                  _stream_handle(stream))
+    args, sh = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha_or_x, beta_or_y, out, extra=(err_word,),
+                            stream=stream)
+    status = load_library().gdn_decode_step_fused(*args, int(flags), _ptr_or_null(err_word, "err_word"), sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_decode_step_fused")
     return status
@@ -246,8 +273,9 @@ def gdn_prefill(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torch.Tensor
     """Enqueue a prefill (see gdn_prefill in include/gdn_step.h): q, k [B, L, Hk, dk],
     v [B, L, Hv, dv], alpha/beta [B, L, Hv], out [B, L, Hv, dv]; only the state after the
     last token is stored, to pool[dst_idx[b]] (dst_idx [B])."""
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1)
-    status = load_library().gdn_prefill(*args, _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    args, sh = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1,
+                            extra=(err_word,), stream=stream)
+    status = load_library().gdn_prefill(*args, _ptr_or_null(err_word, "err_word"), sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_prefill")
     return status
@@ -265,10 +293,11 @@ def gdn_prefill_chunked(pool: torch.Tensor, src_idx: torch.Tensor, dst_idx: torc
     ``workspace`` is a CUDA tensor of at least gdn_prefill_workspace_bytes(...) bytes.
     ``err_word`` (int32 CUDA tensor) is required: a copy or tensor-core wait that runs out is
     reported only there."""
-    args = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1)
+    wp, ep = _dev(workspace, "workspace"), _dev(err_word, "err_word", torch.int32)
+    args, sh = _decode_args(pool, src_idx, dst_idx, q, k, v, alpha, beta, out, dst_per_request=1,
+                            extra=(err_word, workspace), stream=stream)
     nbytes = workspace.numel() * workspace.element_size()
-    status = load_library().gdn_prefill_chunked(*args, _dev(workspace, "workspace"), nbytes,
-                                                _dev(err_word, "err_word", torch.int32), _stream_handle(stream))
+    status = load_library().gdn_prefill_chunked(*args, wp, nbytes, ep, sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_prefill_chunked")
     return status
@@ -285,10 +314,11 @@ def gdn_commit(accept_len: torch.Tensor, committed: torch.Tensor, cur: torch.Ten
     B, T = cur.shape
     if accept_len.numel() != B or committed.numel() != B:
         raise ValueError("accept_len and committed must hold B entries")
-    status = load_library().gdn_commit(
-        _dev(accept_len, "accept_len", torch.int32), _dev(committed, "committed", torch.int32),
-        _dev(cur, "cur", torch.int32), int(B), int(T), int(num_slots),
-        _ptr_or_null(err_word, "err_word"), _stream_handle(stream))
+    ptrs = (_dev(accept_len, "accept_len", torch.int32), _dev(committed, "committed", torch.int32),
+            _dev(cur, "cur", torch.int32))
+    err = _ptr_or_null(err_word, "err_word")
+    sh = _stream_handle(stream, _one_device(accept_len, committed, cur, err_word))
+    status = load_library().gdn_commit(*ptrs, int(B), int(T), int(num_slots), err, sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_commit")
     return status
@@ -304,10 +334,10 @@ def gdn_check_step(src_idx: torch.Tensor, dst_idx: torch.Tensor, num_slots: int,
         raise ValueError("dst_idx must hold B*T entries")
     if scratch.numel() < num_slots:
         raise ValueError("scratch must hold num_slots int32 entries")
-    status = load_library().gdn_check_step(
-        _dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32), int(B), int(T),
-        int(num_slots), _dev(scratch, "scratch", torch.int32), _dev(err_word, "err_word", torch.int32),
-        _stream_handle(stream))
+    ptrs = (_dev(src_idx, "src_idx", torch.int32), _dev(dst_idx, "dst_idx", torch.int32))
+    sp, ep = _dev(scratch, "scratch", torch.int32), _dev(err_word, "err_word", torch.int32)
+    sh = _stream_handle(stream, _one_device(src_idx, dst_idx, scratch, err_word))
+    status = load_library().gdn_check_step(*ptrs, int(B), int(T), int(num_slots), sp, ep, sh)
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_check_step")
     return status
@@ -316,8 +346,8 @@ def gdn_check_step(src_idx: torch.Tensor, dst_idx: torch.Tensor, num_slots: int,
 def gdn_wait_selftest(limit_ns: int, err_word: torch.Tensor, stream=None, check: bool = True) -> int:
     """Enqueue the bounded-wait self-test (see gdn_wait_selftest in include/gdn_step.h):
     a wait on an mbarrier nothing arrives on, which records GDN_ERR_TIMEOUT after limit_ns."""
-    status = load_library().gdn_wait_selftest(int(limit_ns), _dev(err_word, "err_word", torch.int32),
-                                              _stream_handle(stream))
+    ep = _dev(err_word, "err_word", torch.int32)
+    status = load_library().gdn_wait_selftest(int(limit_ns), ep, _stream_handle(stream, _one_device(err_word)))
     if check and status != GDN_OK:
         raise GdnError(status, "gdn_wait_selftest")
     return status
@@ -326,8 +356,8 @@ def gdn_wait_selftest(limit_ns: int, err_word: torch.Tensor, stream=None, check:
 def gdn_get_error(err_word: torch.Tensor, stream=None) -> int:
     """Synchronise the stream, return the device error word's status code and clear it."""
     code = ctypes.c_int32(-1)
-    status = load_library().gdn_get_error(_dev(err_word, "err_word", torch.int32), ctypes.byref(code),
-                                          _stream_handle(stream))
+    ep = _dev(err_word, "err_word", torch.int32)
+    status = load_library().gdn_get_error(ep, ctypes.byref(code), _stream_handle(stream, _one_device(err_word)))
     if status != GDN_OK:
         raise GdnError(status, "gdn_get_error")
     return int(code.value)

@@ -215,3 +215,33 @@ def test_fused_flags_are_checked_on_the_host(lib):
         assert f(*args, flags, None, None) == 0, flags
     for flags in (8, 16, 12, -1):
         assert f(*args, flags, None, None) == 1, flags
+
+
+def test_calls_take_tensors_of_one_device_the_current_one(monkeypatch):
+    """The binding refuses, before any launch, a call whose tensors sit on more than one
+    device, or whose launch stream (torch's current one, a given torch stream, or for a
+    raw handle the current device) belongs to another device: the library would launch
+    there with another GPU's pointers."""
+    import types
+
+    import torch
+
+    from hybrid_linear_attention_step_b200 import gdn
+
+    on = lambda i: types.SimpleNamespace(get_device=lambda: i)
+    assert gdn._one_device(on(0), on(0), None) == 0
+    assert gdn._one_device(on(1), on(1)) == 1
+    with pytest.raises(ValueError, match="one CUDA device"):
+        gdn._one_device(on(0), on(1))
+    stream = lambda i: types.SimpleNamespace(cuda_stream=1000 + i, device_index=i)
+    assert gdn._stream_handle(stream(1), 1) == 1001
+    with pytest.raises(ValueError, match="launch stream is on cuda:0"):
+        gdn._stream_handle(stream(0), 1)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda: stream(0))
+    assert gdn._stream_handle(None, 0) == 1000
+    with pytest.raises(ValueError, match="launch stream is on cuda:0"):
+        gdn._stream_handle(None, 1)
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    assert gdn._stream_handle(12345, 0) == 12345  # a raw handle: checked against the current device
+    with pytest.raises(ValueError, match="current CUDA device is cuda:0"):
+        gdn._stream_handle(12345, 1)
