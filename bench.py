@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel
 # source it was taken on (sha256 of gdn_step.cu).
 NCU_TRAFFIC = {"kernel": "gdn_tile1_kernel<128,128,64,128,5,bf16>",
-               "source_sha256": "0984bccc532caada70117c89e186038080876014904470c22dd5bdd2f1c75da4",
-               "bytes_per_launch": 541174528 + 483733504}
+               "source_sha256": "e539aa9e13cdaa93079eab8dca666256fe2a79d72834bf08a2c25f04e3b9ed12",
+               "bytes_per_launch": 541153280 + 484916224}
 
 # Kernel that serves the large decode for each --variant ("auto" picks the
 # single-token register-tile kernel: 64-column blocks, 128 threads, 5 CTAs/SM).

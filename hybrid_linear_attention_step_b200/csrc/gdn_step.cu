@@ -1205,13 +1205,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 constexpr int kMaxDevices = 64;
 
 int sm_count() {
-    static int cache[kMaxDevices] = {0};
+    // Per-device SM counts, filled on first use; atomics because host threads may call
+    // the library concurrently (every writer stores the same value).
+    static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-    if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+    if (dev < kMaxDevices) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev < kMaxDevices) cache[dev] = n;
+    if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
