@@ -37,9 +37,12 @@
  * No scaling or normalisation of q and k happens inside the step.
  *
  * Ownership and execution.  Every pointer is device memory owned by the caller;
- * the library allocates nothing, frees nothing and keeps no state between calls.
- * All work is enqueued on `stream` (0 = legacy default stream); no call
- * synchronises except gdn_get_error.
+ * the library allocates nothing and frees nothing.  Between calls it keeps only
+ * per-device constants read on first use (the SM count, a symbol address, the
+ * tensor-map encoder), which concurrent host threads fill safely, and the one
+ * device array of gdn_check_step_noalloc (see there).  All work is enqueued on
+ * `stream` (0 = legacy default stream) of the calling thread's current device;
+ * no call synchronises except gdn_get_error.
  *
  * Errors.  Each entry returns a gdn_status.  Bad sizes, a null pointer or an
  * unknown dtype return GDN_ERR_INVALID_ARG before anything is enqueued; a failed
