@@ -250,8 +250,12 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void mbar_init(uint64_t* bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(1) : "memory");
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count = 1) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -1157,6 +1161,7 @@ struct SmemS {
     unsigned char imgB[kImgB];      // [K lo | K hi] | [P_mid | P_hi]
     unsigned char imgC[kImgC];      // g_t, g_C / g_t, g_C | U^T
     uint64_t bar_a, bar_b, bar_c, mma_g, mma_u, mma_o;
+    uint64_t e01, e23;  // quarters 0-1 / 2-3 have written their E parts
     uint32_t tmem;
     int src, dst, status;
 };
@@ -1228,6 +1233,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         mbar_init(&sm.mma_g);
         mbar_init(&sm.mma_u);
         mbar_init(&sm.mma_o);
+        mbar_init(&sm.e01, kScanThreads / 2);
+        mbar_init(&sm.e23, kScanThreads / 2);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -1308,10 +1315,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
     };
 
-    // Two CTA barriers per chunk: before the first products (the S parts are written)
-    // and before the state update's products (the E parts are written).  Every other
-    // hand-off is an mbarrier that each thread waits on itself; what those waits saw is
-    // carried to the next barrier, which stops the walk if any ran out.
+    // One CTA barrier per chunk, before the first products (the S parts are written).
+    // Every other hand-off is an mbarrier: the E parts of token quarters 0-1, then of
+    // 2-3 (the state update's products on the first start while the second are formed),
+    // and the copy and MMA completions, which each thread waits on itself.  What those
+    // waits saw is carried to the next barrier, which stops the walk if any ran out.
     bool carry = true;
     int c = 0;
     for (; c < nch; ++c) {
@@ -1380,6 +1388,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         // --- E = U - W M and g Q M for this thread's 16 tokens
         const float* gq = reinterpret_cast<const float*>(sm.imgC);
         const float gC = gq[2 * kC];
+        // Quarters 0-1 (tokens 0..31) first: the state update's products on their E parts
+        // run while quarters 2-3 form theirs.
+        if (quarter >= 2) got = wait_parity(&sm.e01, (uint32_t)c & 1u) && got;
         {
             const float* gk = gq + kC;
             const float4* ut = reinterpret_cast<const float4*>(sm.imgC + kR2GBytes) + j;
@@ -1427,22 +1438,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             }
             tmem_wait_st();
         }
+        tc_fence_before();
+        mbar_arrive(quarter < 2 ? &sm.e01 : &sm.e23);
         out_t0 = c * kC;
         out_n = min(kC, a.L - out_t0);
-        if (issuer) got = wait_parity(&sm.bar_b, (uint32_t)c & 1u) && got;
-        tc_fence_before();
-        if (__syncthreads_or(got ? 0 : 1)) {
-            ok = false;
-            break;
-        }
-        tc_fence_after();
-        // --- state update first (the chain waits for it), then the outputs' products
+        // --- state update (committed first: the chain waits for it), then the outputs' products
         if (issuer) {
-            ++done_b;
-            if (c + 1 < nch) {  // U^T and the gate factors are consumed
-                issue_c(c + 1);
-                ++issued_c;
-            }
             // B = K, MN-major: features 64 to a row, tokens one row each (16 tokens per
             // MMA: 2048 bytes), the second feature half one tile on.
             const uint32_t bK = smem_u32(sm.imgB), bP = bK + 2 * kSwTile;
@@ -1451,10 +1452,21 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             auto epart = [&](int p, int ks) -> uint32_t {
                 return tmem + (uint32_t)(16 * ks) + (p < 4 ? (uint32_t)(p * kC) : 8u);
             };
-            for (int part = 0; part < 3; ++part)
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    umma_bf16_ta(tmem + kTmemDU, epart(part, ks), umma_desc_sw128(bK + 2048u * ks, kSwTile, 1024),
-                                 kIdesc128 | kIdescBmn, (part | ks) != 0 ? 1u : 0u);
+            auto issue_du = [&](int k0) {  // K-steps k0, k0 + 1 (the tokens of two quarters)
+                for (int ks = k0; ks < k0 + 2; ++ks)
+                    for (int part = 0; part < 3; ++part)
+                        umma_bf16_ta(tmem + kTmemDU, epart(part, ks),
+                                     umma_desc_sw128(bK + 2048u * ks, kSwTile, 1024), kIdesc128 | kIdescBmn,
+                                     (part | ks) != 0 ? 1u : 0u);
+            };
+            const bool g01 = wait_parity(&sm.e01, (uint32_t)c & 1u);
+            const bool gb = wait_parity(&sm.bar_b, (uint32_t)c & 1u);
+            if (gb) ++done_b;
+            tc_fence_after();
+            issue_du(0);
+            const bool g23 = wait_parity(&sm.e23, (uint32_t)c & 1u);
+            tc_fence_after();
+            issue_du(2);
             umma_commit(&sm.mma_u);
             for (int ks = 0; ks < kC / 16; ++ks)
                 umma_bf16_ta(tmem + kTmemDO, epart(3, ks), umma_desc(bP + 256 * ks, kSbo), kIdesc128,
@@ -1464,11 +1476,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                              kIdesc64, 1u);
             umma_commit(&sm.mma_o);
             ++issued_u, ++issued_o;
+            got = got && g01 && gb && g23;
+            if (got && c + 1 < nch) {  // U^T and the gate factors are consumed
+                issue_c(c + 1);
+                ++issued_c;
+            }
         }
         {
             const bool gu = wait_parity(&sm.mma_u, (uint32_t)c & 1u);
             if (issuer && gu) ++waits_u;
-            carry = gu;
+            carry = gu && got;
         }
         tc_fence_after();
         {
